@@ -1,0 +1,413 @@
+/*
+ * nvfp4_oracle.c — plain, single-threaded CPU oracle for the NVFP4 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY: loaded by tests/, __graft_entry__.smoke() and bench.py's
+ * CPU baseline.  No product code path may call it.  It shares nothing with the CUDA
+ * sources.  Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math (see build_oracle.py);
+ * every fp32 operation below is one IEEE-754 binary32 operation rounded to nearest even
+ * (x86-64 SSE arithmetic, no contraction into fused multiply-add).
+ *
+ * Sources are cited as "page title, section".  Where the pages leave a step open the
+ * reading taken is stated as READING in the comment beside it.
+ */
+#include "nvfp4_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------------------ */
+/* bf16 -> fp32 widening is exact: the bf16 bits are the top half of the fp32 bits.     */
+static float bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* E2M1: 1 sign bit, 2 exponent bits, 1 mantissa bit; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
+ * (the NVFP4 element grid).  Code bit 3 is the sign.                                      */
+static const double kE2M1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+float orc_e2m1_decode(uint8_t code) {
+    double m = kE2M1Mag[code & 7u];
+    return (float)((code & 8u) ? -m : m);
+}
+
+/* Round to nearest on the E2M1 grid, ties to the code with an even mantissa bit
+ * ("Pi0.5 Thor NVFP4 End-to-End Results", §Implemented Path: native FP4 conversion is
+ * round-to-nearest-even).  Magnitudes above 6 saturate to 6 (satfinite).
+ * READING: the sign of the input is kept, so values that round to zero give +0 (0x0) or
+ * -0 (0x8) by their sign, as an IEEE-style conversion does.  Inputs are finite.        */
+uint8_t orc_e2m1_encode(float v) {
+    uint8_t sign = signbit(v) ? 8u : 0u;
+    double a = fabs((double)v);
+    if (a >= 6.0) return (uint8_t)(sign | 7u); /* satfinite: everything from 6 up is 6 */
+    int best = 0;
+    double best_d = a; /* distance to magnitude 0 */
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(a - kE2M1Mag[c]);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) != 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | (uint8_t)best);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* E4M3 (bias 7): normal (1 + m/8) * 2^(e-7) for e = 1..15, except e = 15, m = 7 which is
+ * NaN; subnormal m * 2^-9; max finite 448 (0x7E).  The block scale is the unsigned form
+ * (sign bit 0) ("Pi0.5 ...", §Encoder Attention QKV NVFP4 + Scale-Factor Zero-Init: the
+ * bytes 0x7F/0xFF decode as NaN).                                                       */
+float orc_e4m3_decode(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return (float)(s ? -mag : mag);
+}
+
+/* Round to nearest E4M3 value, ties to the even code, magnitudes above 448 saturate to
+ * 448 (satfinite).  Finite codes 0x00..0x7E are strictly increasing in value, so the
+ * two candidates are found by bisection.  Sign kept (the block scale is never negative). */
+uint8_t orc_e4m3_encode(float t) {
+    uint8_t sign = signbit(t) ? 0x80u : 0u;
+    double a = fabs((double)t);
+    if (isnan(t)) return (uint8_t)(sign | 0x7Fu);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);
+    int lo = 0, hi = 0x7E; /* invariant: dec(lo) <= a < dec(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if ((double)orc_e4m3_decode((uint8_t)mid) <= a) lo = mid;
+        else hi = mid;
+    }
+    double dl = a - (double)orc_e4m3_decode((uint8_t)lo);
+    double dh = (double)orc_e4m3_decode((uint8_t)hi) - a;
+    int c = (dl < dh) ? lo : (dh < dl) ? hi : ((lo & 1) == 0 ? lo : hi);
+    return (uint8_t)(sign | (uint8_t)c);
+}
+
+/* Array forms of the codecs (one call per array instead of per element). */
+void orc_e2m1_encode_n(const float *v, size_t n, uint8_t *out) {
+    for (size_t i = 0; i < n; ++i) out[i] = orc_e2m1_encode(v[i]);
+}
+void orc_e4m3_encode_n(const float *v, size_t n, uint8_t *out) {
+    for (size_t i = 0; i < n; ++i) out[i] = orc_e4m3_encode(v[i]);
+}
+void orc_e4m3_decode_n(const uint8_t *c, size_t n, float *out) {
+    for (size_t i = 0; i < n; ++i) out[i] = orc_e4m3_decode(c[i]);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Scale-factor layout ("Pi0.5 ...", §Encoder Attention QKV NVFP4 + Scale-Factor
+ * Zero-Init: tile-interleaved SFA/SFB layouts round K up to 64-element atoms; padding
+ * entries must be zero).
+ * READING: the tile atom is 128 rows x 4 scale blocks = 512 bytes; inside it, row r and
+ * block c sit at (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4; atoms are ordered with the
+ * K-atom index fastest, then the 128-row group.  Rows are padded to 128.                */
+size_t orc_sf_bytes(int rows, int K) {
+    size_t row_groups = ((size_t)rows + 127) / 128;
+    size_t k_atoms = ((size_t)K + 63) / 64;
+    return row_groups * k_atoms * 512;
+}
+
+size_t orc_sf_offset(int row, int kblk, int K) {
+    size_t k_atoms = ((size_t)K + 63) / 64;
+    size_t atom = (size_t)(row / 128) * k_atoms + (size_t)(kblk / 4);
+    return atom * 512 + (size_t)(row % 32) * 16 + (size_t)((row % 128) / 32) * 4 + (size_t)(kblk % 4);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* One block of 16 values ("GROOT N1.7 ...", §What is in the tier: one UE4M3 scale per
+ * 16 elements, computed at run time; E2M1 codes; fp32 per-tensor global scale g).
+ *   a = max|y|;  d = 6*g;  t = a/d;  s = E4M3(t);  S = dec(s)*g
+ *   dec(s) == 0  -> every code is +0 and the scale byte is 0
+ *   otherwise    r = 1/S;  code_i = E2M1(y_i * r)
+ * READING: a/(6g) is one IEEE division, y*(1/S) one reciprocal then one multiply, every
+ * step rounded to fp32 nearest-even (the pages fix no order; this one is reproducible).
+ * Codes are packed two per byte, element 2j in the low nibble.                          */
+uint8_t orc_quantize_block16(const float *y, float g, uint8_t *codes8) {
+    float a = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float m = fabsf(y[i]);
+        if (m > a) a = m;
+    }
+    float d = 6.0f * g;
+    float t = a / d;
+    uint8_t s = orc_e4m3_encode(t);
+    float ds = orc_e4m3_decode(s);
+    if (ds == 0.0f) {
+        memset(codes8, 0, 8);
+        return s;
+    }
+    float S = ds * g;
+    float r = 1.0f / S;
+    for (int j = 0; j < 8; ++j) {
+        float v0 = y[2 * j] * r;
+        float v1 = y[2 * j + 1] * r;
+        codes8[j] = (uint8_t)(orc_e2m1_encode(v0) | (orc_e2m1_encode(v1) << 4));
+    }
+    return s;
+}
+
+void orc_quantize_rows(const float *y, int rows, int K, int ldy, float g,
+                       uint8_t *codes, uint8_t *sf) {
+    int nblk = (K + 15) / 16;
+    size_t row_bytes = (size_t)nblk * 8;
+    float blk[16];
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? y[(size_t)r * ldy + k] : 0.0f;
+            }
+            uint8_t s = orc_quantize_block16(blk, g, codes + (size_t)r * row_bytes + (size_t)b * 8);
+            sf[orc_sf_offset(r, b, K)] = s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Norm front-ends, one row at a time ("GROOT N1.7 ...", §What is in the tier: AdaLN and
+ * the pre-FFN LayerNorm emit FP4 directly; "Pi0.5 ...", §Implemented Path: AdaRMSNorm
+ * before QKV and Gate+Up; §Vectorized SigLIP LayerNorms: LayerNorm to NVFP4).
+ *   LayerNorm : n = (x - mu) * rstd;          y = n * gamma + beta
+ *   RMSNorm   : y = (x * rstd_rms) * gamma
+ *   AdaLN     : y = n * (1 + scale) + shift
+ *   AdaRMSNorm: y = (x * rstd_rms) * (1 + scale) [+ shift]
+ * READING: row statistics are accumulated in fp64 in index order (mean, then the
+ * population variance about it; mean of squares for RMS), rounded once to fp32:
+ * mu_f = (float)mu, rstd_f = (float)(1 / sqrt(var + eps)).  The elementwise steps are
+ * fp32 operations in the order written, (1 + scale) formed first.  A NULL gamma reads
+ * as 1, a NULL beta / scale / shift as 0.                                               */
+static float ld_x(const void *x, int in_fp32, size_t i) {
+    return in_fp32 ? ((const float *)x)[i] : bf16_to_f32(((const uint16_t *)x)[i]);
+}
+
+void orc_norm_rows(const void *x, int in_fp32, int rows, int K, int ldx, int kind,
+                   const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,
+                   const uint16_t *mod_shift, float eps, float *y) {
+    for (int r = 0; r < rows; ++r) {
+        size_t base = (size_t)r * ldx;
+        float *yr = y + (size_t)r * K;
+        if (kind == ORC_NORM_NONE) {
+            for (int k = 0; k < K; ++k) yr[k] = ld_x(x, in_fp32, base + k);
+            continue;
+        }
+        float mu_f = 0.0f, rstd_f;
+        if (kind == ORC_NORM_LAYERNORM || kind == ORC_NORM_ADALN) {
+            double s = 0.0;
+            for (int k = 0; k < K; ++k) s += (double)ld_x(x, in_fp32, base + k);
+            double mu = s / K;
+            double q = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double dv = (double)ld_x(x, in_fp32, base + k) - mu;
+                q += dv * dv;
+            }
+            double var = q / K;
+            mu_f = (float)mu;
+            rstd_f = (float)(1.0 / sqrt(var + (double)eps));
+        } else {
+            double q = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double xv = (double)ld_x(x, in_fp32, base + k);
+                q += xv * xv;
+            }
+            rstd_f = (float)(1.0 / sqrt(q / K + (double)eps));
+        }
+        for (int k = 0; k < K; ++k) {
+            float xv = ld_x(x, in_fp32, base + k);
+            float ga = gamma ? bf16_to_f32(gamma[k]) : 1.0f;
+            float be = beta ? bf16_to_f32(beta[k]) : 0.0f;
+            float sc = mod_scale ? bf16_to_f32(mod_scale[k]) : 0.0f;
+            float sh = mod_shift ? bf16_to_f32(mod_shift[k]) : 0.0f;
+            float out;
+            switch (kind) {
+            case ORC_NORM_LAYERNORM: {
+                float n = (xv - mu_f) * rstd_f;
+                float t = n * ga;
+                out = t + be;
+                break;
+            }
+            case ORC_NORM_ADALN: {
+                float n = (xv - mu_f) * rstd_f;
+                float opl = 1.0f + sc;
+                float t = n * opl;
+                out = t + sh;
+                break;
+            }
+            case ORC_NORM_RMSNORM: {
+                float n = xv * rstd_f;
+                out = n * ga;
+                break;
+            }
+            default: { /* ORC_NORM_ADARMS */
+                float n = xv * rstd_f;
+                float opl = 1.0f + sc;
+                float t = n * opl;
+                out = mod_shift ? t + sh : t;
+                break;
+            }
+            }
+            yr[k] = out;
+        }
+    }
+}
+
+/* Fused norm -> FP4 is, by the pages' contract, identical to the two-step chain
+ * ("GROOT N1.7 ...", §What is in the tier: bit-identical to the two-step chain).
+ * READING: the intermediate y is not rounded to bf16/fp16 between the steps.           */
+void orc_quantize_norm(const void *x, int in_fp32, int rows, int K, int ldx, int kind,
+                       const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,
+                       const uint16_t *mod_shift, float eps, float g,
+                       uint8_t *codes, uint8_t *sf) {
+    float *y = (float *)malloc(sizeof(float) * (size_t)K);
+    size_t esz = in_fp32 ? 4 : 2;
+    int nblk = (K + 15) / 16;
+    for (int r = 0; r < rows; ++r) {
+        const char *xr = (const char *)x + (size_t)r * ldx * esz;
+        orc_norm_rows(xr, in_fp32, 1, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, y);
+        /* quantize this row as row r of the output */
+        float blk[16];
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? y[k] : 0.0f;
+            }
+            uint8_t s = orc_quantize_block16(blk, g, codes + (size_t)r * nblk * 8 + (size_t)b * 8);
+            sf[orc_sf_offset(r, b, K)] = s;
+        }
+    }
+    free(y);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Offline weight quantization ("Pi0.5 ...", §Implemented Path: weights are quantized
+ * once to NVFP4 E2M1 plus block scales).  Blocks run along K, as for activations.
+ * READING: the per-tensor global scale is amax(|W|) / (6 * 448) so that the largest
+ * block scale lands on the E4M3 maximum; an all-zero tensor takes g = 1.
+ * Optional pairwise interleave ("Pi0.5 ...", §Fused GeGLU Epilogue for the P1 Encoder
+ * FFN: gate and up rows pairwise interleaved along N): rows [0, N/2) are gate, rows
+ * [N/2, N) are up; packed row 2j = gate row j, packed row 2j+1 = up row j.             */
+float orc_quantize_weight(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up,
+                          uint8_t *codes, uint8_t *sf) {
+    float amax = 0.0f;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            float m = fabsf(bf16_to_f32(w[(size_t)n * ldw + k]));
+            if (m > amax) amax = m;
+        }
+    float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    float *y = (float *)malloc(sizeof(float) * (size_t)K);
+    int nblk = (K + 15) / 16;
+    for (int r = 0; r < N; ++r) {
+        int src = r;
+        if (interleave_gate_up) src = (r % 2 == 0) ? r / 2 : N / 2 + r / 2;
+        for (int k = 0; k < K; ++k) y[k] = bf16_to_f32(w[(size_t)src * ldw + k]);
+        float blk[16];
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? y[k] : 0.0f;
+            }
+            uint8_t s = orc_quantize_block16(blk, g, codes + (size_t)r * nblk * 8 + (size_t)b * 8);
+            sf[orc_sf_offset(r, b, K)] = s;
+        }
+    }
+    free(y);
+    return g;
+}
+
+/* Dequantized value of element k of row `row`: val(code) * dec(scale) * g, exact in fp64. */
+static double deq_elem(const uint8_t *codes, const uint8_t *sf, float g, int row, int k, int K) {
+    int nblk = (K + 15) / 16;
+    uint8_t byte = codes[(size_t)row * nblk * 8 + (size_t)k / 2];
+    uint8_t c = (k % 2 == 0) ? (byte & 15u) : (byte >> 4);
+    double s = (double)orc_e4m3_decode(sf[orc_sf_offset(row, k / 16, K)]);
+    return (double)orc_e2m1_decode(c) * s * (double)g;
+}
+
+void orc_dequantize(const uint8_t *codes, const uint8_t *sf, float g, int rows, int K,
+                    double *out) {
+    for (int r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k) out[(size_t)r * K + k] = deq_elem(codes, sf, g, r, k, K);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* tanh-form GELU, 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))), in fp64. */
+double orc_gelu_tanh(double z) {
+    const double k = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * z * (1.0 + tanh(k * (z + 0.044715 * z * z * z)));
+}
+
+/* Block-scaled GEMM with fused epilogue ("GROOT N1.7 ...", §What is in the tier: every
+ * DiT GEMM is NVFP4 x NVFP4 with fused bf16 bias / bias+residual / bias+tanh-GELU+FP4
+ * output epilogues; "Pi0.5 ...", §Half-Width Fused GeGLU Epilogue and §Fused GeGLU FFN
+ * in the Decoder: gelu(gate) * up on pairwise-interleaved columns, quantized once, GELU
+ * on the fp32 accumulator rather than on a rounded GEMM output).
+ *   acc[m,n] = sum_k Adeq[m,k] * Wdeq[n,k]          (fp64, k ascending)
+ *   v[m,n]   = acc + bias[n] + residual[m,n]        (terms present per epilogue)
+ *   BIAS_GELU: h = gelu(v), N_out = N;   GEGLU: h[m,j] = gelu(v[m,2j]) * v[m,2j+1], N_out = N/2
+ *   FP4 output = the block quantizer applied to (float)h along n with g_out.
+ * Dequantized operands include their global scales, so acc already carries gA * gW.    */
+void orc_gemm(const uint8_t *a_codes, const uint8_t *a_sf, float gA, int M,
+              const uint8_t *w_codes, const uint8_t *w_sf, float gW, int N, int K,
+              int epi, const uint16_t *bias, const uint16_t *residual, int ldr,
+              const int *m_idx, int n_rows, double *v_out, double *h_out,
+              float g_out, uint8_t *out_codes, uint8_t *out_sf) {
+    if (!m_idx) n_rows = M;
+    double *arows = (double *)malloc(sizeof(double) * (size_t)n_rows * K);
+    double *wrow = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int i = 0; i < n_rows; ++i) {
+        int m = m_idx ? m_idx[i] : i;
+        for (int k = 0; k < K; ++k) arows[(size_t)i * K + k] = deq_elem(a_codes, a_sf, gA, m, k, K);
+    }
+    int use_bias = (epi == ORC_EPI_BIAS || epi == ORC_EPI_BIAS_RESIDUAL || epi == ORC_EPI_BIAS_GELU ||
+                    epi == ORC_EPI_GEGLU) && bias != NULL;
+    int use_res = (epi == ORC_EPI_RESIDUAL || epi == ORC_EPI_BIAS_RESIDUAL);
+    for (int n = 0; n < N; ++n) {
+        for (int k = 0; k < K; ++k) wrow[k] = deq_elem(w_codes, w_sf, gW, n, k, K);
+        for (int i = 0; i < n_rows; ++i) {
+            int m = m_idx ? m_idx[i] : i;
+            const double *ar = arows + (size_t)i * K;
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k) acc += ar[k] * wrow[k];
+            if (use_bias) acc += (double)bf16_to_f32(bias[n]);
+            if (use_res) acc += (double)bf16_to_f32(residual[(size_t)m * ldr + n]);
+            v_out[(size_t)i * N + n] = acc;
+        }
+    }
+    if (epi == ORC_EPI_BIAS_GELU || epi == ORC_EPI_GEGLU) {
+        int n_out = (epi == ORC_EPI_GEGLU) ? N / 2 : N;
+        float *hf = (float *)malloc(sizeof(float) * (size_t)n_out);
+        int oblk = (n_out + 15) / 16;
+        for (int i = 0; i < n_rows; ++i) {
+            int m = m_idx ? m_idx[i] : i;
+            const double *v = v_out + (size_t)i * N;
+            for (int j = 0; j < n_out; ++j) {
+                double h = (epi == ORC_EPI_GEGLU) ? orc_gelu_tanh(v[2 * j]) * v[2 * j + 1]
+                                                   : orc_gelu_tanh(v[j]);
+                if (h_out) h_out[(size_t)i * n_out + j] = h;
+                hf[j] = (float)h;
+            }
+            if (out_codes && out_sf) {
+                float blk[16];
+                for (int b = 0; b < oblk; ++b) {
+                    for (int t = 0; t < 16; ++t) {
+                        int j = b * 16 + t;
+                        blk[t] = (j < n_out) ? hf[j] : 0.0f;
+                    }
+                    uint8_t s = orc_quantize_block16(blk, g_out,
+                                                     out_codes + (size_t)m * oblk * 8 + (size_t)b * 8);
+                    out_sf[orc_sf_offset(m, b, n_out)] = s;
+                }
+            }
+        }
+        free(hf);
+    }
+    free(wrow);
+    free(arows);
+}
