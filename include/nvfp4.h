@@ -1,0 +1,196 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4.so: the NVFP4 linear layer of a VLA action head on B200
+ * (sm_100a): bf16 -> {LayerNorm | RMSNorm | AdaLN | AdaRMSNorm} -> dynamic NVFP4 quantize,
+ * offline NVFP4 weight quantize, and a block-scaled NVFP4 GEMM (tcgen05 kind::mxf4nvf4)
+ * with fused bias / residual / tanh-GELU->FP4 / GeGLU->FP4 epilogues.
+ *
+ * Sources are cited as "page title, section":
+ *   [GROOT]  "GROOT N1.7 update: Thor NVFP4 + FA4 performance tier"
+ *   [PI05]   "Pi0.5 Thor NVFP4 End-to-End Results"
+ *
+ * Formats (shared by every entry point):
+ *   FP4 tensor of `rows` x K elements:
+ *     codes : uint8 [rows, K/2], row stride K/2 bytes; element 2j of a row in the low
+ *             nibble of byte j, element 2j+1 in the high nibble; E2M1 code, bit 3 = sign,
+ *             magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}.
+ *     sf    : uint8 UE4M3 block scales, one per (row, 16-element K block), in 512-byte
+ *             atoms of 128 rows x 4 blocks; atoms ordered K fastest, then 128-row group;
+ *             inside an atom row r, block c is at (r%32)*16 + ((r%128)/32)*4 + c%4.
+ *             Rows are padded to 128 and K to 64 elements; nvfp4_sf_bytes() gives the size.
+ *             Padding bytes must be zero ([PI05] §Encoder Attention QKV NVFP4 +
+ *             Scale-Factor Zero-Init): zero the buffer once at allocation (nvfp4_sf_zero);
+ *             the quantizers write only real entries.
+ *     global_scale g (fp32): an element decodes as val(code) * dec(sf) * g.
+ *   bf16 tensors are row-major with the stated leading dimension (in elements).
+ *
+ * Conventions:
+ *   - Every pointer inside a call is a DEVICE pointer unless marked "host".  The caller
+ *     allocates and owns every buffer.  Device pointers must be 16-byte aligned and leading
+ *     dimensions multiples of 8 elements.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream),
+ *     allocate nothing and never synchronise, except nvfp4_quantize_weight (returns the
+ *     global scale to the host) and nvfp4_get_device_status.
+ *   - Errors are returned as nvfp4_status; nothing throws across the ABI and no call falls
+ *     back to another precision or a host path ([PI05] §Implemented Path: unsupported
+ *     shapes, missing kernels or failed launches raise; none selects another tier).
+ *   - Global scales must be finite and within [2^-100, 2^100].
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nvfp4_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,       /* NULL pointer, bad enum, bad scale, ld < K ...     */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* K or N outside the documented constraints        */
+    NVFP4_ERR_MISALIGNED = 3,        /* pointer not 16-byte aligned / ld not a multiple of 8 */
+    NVFP4_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required          */
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 5,/* current device is not sm_100                     */
+    NVFP4_ERR_CUDA = 6,              /* a CUDA runtime/driver call or launch failed      */
+    NVFP4_ERR_TIMEOUT = 7            /* a kernel's bounded wait expired (device status)  */
+} nvfp4_status;
+
+typedef enum {
+    NVFP4_NORM_NONE = 0,      /* y = x (plain quantizer)                               */
+    NVFP4_NORM_LAYERNORM = 1, /* y = (x - mu) * rstd * gamma + beta                    */
+    NVFP4_NORM_RMSNORM = 2,   /* y = (x * rstd_rms) * gamma                            */
+    NVFP4_NORM_ADALN = 3,     /* y = (x - mu) * rstd * (1 + scale) + shift             */
+    NVFP4_NORM_ADARMS = 4     /* y = (x * rstd_rms) * (1 + scale) [+ shift]            */
+} nvfp4_norm;
+
+typedef enum {
+    NVFP4_EPI_NONE = 0,          /* out = acc * gA * gW                       -> bf16   */
+    NVFP4_EPI_BIAS = 1,          /* + bias[n]                                 -> bf16   */
+    NVFP4_EPI_RESIDUAL = 2,      /* + residual[m, n]                          -> bf16   */
+    NVFP4_EPI_BIAS_RESIDUAL = 3, /* + bias[n] + residual[m, n]                -> bf16   */
+    NVFP4_EPI_BIAS_GELU = 4,     /* gelu_tanh(acc*gA*gW + bias[n])            -> FP4    */
+    NVFP4_EPI_GEGLU = 5          /* gelu_tanh(v[m,2j]) * v[m,2j+1], v = acc*gA*gW (+bias) -> FP4, width N/2 */
+} nvfp4_epilogue;
+
+typedef enum { NVFP4_IN_BF16 = 0, NVFP4_IN_FP32 = 1 } nvfp4_in_dtype;
+
+/* An FP4 operand: device codes / sf in the formats above, host-side global scale. */
+typedef struct {
+    const uint8_t *codes;
+    const uint8_t *sf;
+    float global_scale;
+    int rows;
+    int K;
+} nvfp4_tensor;
+
+/* ---- helpers ----------------------------------------------------------------------- */
+
+/* NVFP4_OK if the current device is sm_100 and this library's kernels load on it;
+ * NVFP4_ERR_UNSUPPORTED_DEVICE otherwise.  Call once before capture ([GROOT] §Shared-code
+ * changes: the frontend probes its bindings up front instead of failing inside capture). */
+nvfp4_status nvfp4_probe(void);
+
+/* Static, never NULL. */
+const char *nvfp4_status_string(nvfp4_status s);
+
+/* Bytes of a scale-factor buffer for rows x K elements: ceil(rows/128)*ceil(K/64)*512. */
+size_t nvfp4_sf_bytes(int rows, int K);
+
+/* Byte offset of the scale of (row, K block kblk) in that buffer (layout above). */
+size_t nvfp4_sf_offset(int row, int kblk, int K);
+
+/* Zeroes a scale-factor buffer (cudaMemsetAsync); once per allocation is enough. */
+nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream);
+
+/* Workspace bytes nvfp4_gemm needs for this shape (split-K partials and tile tickets);
+ * 0 if none.  The workspace must be zeroed once at allocation; every call leaves its
+ * ticket words zero again (after NVFP4_ERR_TIMEOUT, zero it again). */
+size_t nvfp4_gemm_workspace_bytes(int M, int N, int K);
+
+/* Reads and clears the library's device status word after synchronising `stream`:
+ * NVFP4_OK, or NVFP4_ERR_TIMEOUT if a kernel's bounded wait expired since the last read. */
+nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
+
+/* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
+
+/* Per row of x [M, K] (leading dimension ldx, bf16 or fp32): the norm `kind`, then the
+ * per-16 block quantizer with global scale `global_scale`, emitting codes [M, K/2] and
+ * sf (nvfp4_sf_bytes(M, K), pre-zeroed).  ([GROOT] §What is in the tier: AdaLN and the
+ * pre-FFN LayerNorm emit FP4 directly, bit-identical to the two-step chain; dynamic
+ * per-16 activation quantization with no calibration pass.  [PI05] §Vectorized SigLIP
+ * LayerNorms: register-resident single pass with 16-byte loads; §Implemented Path:
+ * AdaRMSNorm + NVFP4/SFA in one launch, dynamic quantization of the attention output.)
+ *
+ * Per block of 16 normalized values y:  a = max|y|, s = E4M3_rn_satfinite(a / (6 g)),
+ * S = dec(s) g; dec(s) == 0 -> all codes +0; else code_i = E2M1_rn_satfinite(y_i * (1/S)).
+ * Row statistics: fp64 sums, mean and 1/sqrt(var + eps) rounded once to fp32.
+ * gamma/beta/mod_scale/mod_shift: bf16 [K] or NULL (gamma NULL reads 1, others 0).
+ * Constraints: M >= 0 (M == 0 is a no-op), 16 <= K <= 32768, K % 16 == 0, ldx >= K. */
+nvfp4_status nvfp4_quantize_norm(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx,
+                                 nvfp4_norm kind, const void *gamma, const void *beta,
+                                 const void *mod_scale, const void *mod_shift, float eps,
+                                 float global_scale, uint8_t *codes, uint8_t *sf,
+                                 nvfp4_stream_t stream);
+
+/* The first step of the two-step chain alone: the same norm, written as fp32 y [M, K]
+ * (dense).  nvfp4_quantize_norm(y, NVFP4_IN_FP32, ..., NVFP4_NORM_NONE, ...) is the second
+ * step; the fused call equals the chain bit for bit. */
+nvfp4_status nvfp4_norm_f32(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx,
+                            nvfp4_norm kind, const void *gamma, const void *beta,
+                        const void *mod_scale, const void *mod_shift, float eps, float *y,
+                        nvfp4_stream_t stream);
+
+/* ---- offline weight quantize --------------------------------------------------------- */
+
+/* W bf16 [N, K] (ldw) -> codes [N, K/2] + sf (nvfp4_sf_bytes(N, K), pre-zeroed) with the
+ * per-tensor global scale g = amax(|W|) / (6 * 448) (1 if W is all zero), returned in
+ * *global_scale_out (host).  interleave_gate_up = 1 packs rows [0, N/2) (gate) and
+ * [N/2, N) (up) pairwise: output row 2j = gate row j, row 2j+1 = up row j ([PI05]
+ * §Fused GeGLU Epilogue for the P1 Encoder FFN).  `scratch`: device, >= 256 bytes.
+ * Synchronises `stream`.  ([PI05] §Implemented Path: weights quantized once at load.) */
+nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw,
+                                   int interleave_gate_up, uint8_t *codes, uint8_t *sf,
+                                   float *global_scale_out, void *scratch,
+                                   nvfp4_stream_t stream);
+
+/* ---- block-scaled NVFP4 GEMM with fused epilogue ------------------------------------ */
+
+/* acc[m, n] = sum_k dec(A)[m, k] * dec(W)[n, k] over the E2M1 codes and UE4M3 block scales
+ * (tcgen05.mma kind::mxf4nvf4, fp32 accumulation in tensor memory), then the epilogue
+ * `epi` on v = acc * gA * gW (+ bias[n]) (+ residual[m, n]) ([GROOT] §What is in the tier:
+ * fused bf16 bias / bias+residual / bias+tanh-GELU+FP4-output epilogues; [PI05] §Fused
+ * GeGLU FFN in the Decoder: GELU on the fp32 accumulator, gate/up interleaved pairwise).
+ *   A: M x K activations, W: N x K weights (A->rows == M, W->rows == N, both ->K == K).
+ *   bias: bf16 [N] or NULL; residual: bf16 [M, ldr] (RESIDUAL / BIAS_RESIDUAL only).
+ *   bf16 epilogues write out_bf16 [M, ldo]; FP4 epilogues (BIAS_GELU, GEGLU) write
+ *   out_codes [M, N_out/2] and out_sf (nvfp4_sf_bytes(M, N_out), pre-zeroed) quantized
+ *   with out_global_scale, N_out = N (BIAS_GELU) or N/2 (GEGLU).
+ *   workspace: >= nvfp4_gemm_workspace_bytes(M, N, K) bytes, zeroed once at allocation.
+ * Constraints: M >= 0 (0 is a no-op), K % 32 == 0 (TMA 16-byte rows; a K % 64 tail is
+ * covered by the zero scale padding, [PI05] §Encoder Attention QKV NVFP4 + Scale-Factor
+ * Zero-Init), N % 64 == 0. */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
+                        nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
+                        void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,
+                        float out_global_scale, void *workspace, size_t ws_bytes,
+                        nvfp4_stream_t stream);
+
+/* Schedule-pinned variant of nvfp4_gemm for tuning sweeps and tests: block_n in
+ * {64, 128, 256} output columns per CTA, splits >= 1 K partitions (each a whole number of
+ * 256-element K tiles; 0 = let the library choose both).  Same contract otherwise; the
+ * workspace must hold nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits) bytes. */
+nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
+                           nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
+                           void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,
+                           float out_global_scale, void *workspace, size_t ws_bytes,
+                           int block_n, int splits, nvfp4_stream_t stream);
+
+size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int splits);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

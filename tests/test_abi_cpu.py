@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and exports every
+function include/nvfp4.h declares, its layout helpers agree with the oracle, and argument
+validation rejects bad calls before touching the device."""
+import ctypes as C
+
+import pytest
+
+from vla_action_head_b200 import build, nvfp4
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return nvfp4.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = nvfp4.header_functions()
+    assert {"nvfp4_quantize_norm", "nvfp4_quantize_weight", "nvfp4_gemm"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert L.nvfp4_status_string(s)
+    assert L.nvfp4_status_string(99) == b"unknown status"
+
+
+def test_sf_layout_matches_oracle(L, orc):
+    for rows, K in ((1, 16), (41, 1536), (130, 4320), (968, 2048), (300, 96)):
+        assert L.nvfp4_sf_bytes(rows, K) == orc.sf_bytes(rows, K)
+        for r in range(0, rows, max(1, rows // 37)):
+            for b in range(0, K // 16, max(1, K // 16 // 23)):
+                assert L.nvfp4_sf_offset(r, b, K) == orc.sf_offset(r, b, K)
+
+
+def test_workspace_sizes(L):
+    assert L.nvfp4_gemm_workspace_bytes_ex(968, 2560, 2048, 256, 1) == 0
+    ws = L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 128, 4)
+    assert ws >= 4 * 41 * 1536 * 4
+    assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 96, 1) == 0  # N % 96 != 0
+
+
+def _t(codes=0x1000, sf=0x2000, g=1.0, rows=4, K=64):
+    return nvfp4._Tensor(codes, sf, g, rows, K)
+
+
+def test_gemm_validation(L):
+    A, W = _t(rows=4, K=64), _t(rows=64, K=64)
+    out = C.c_void_p(0x3000)
+    g = L.nvfp4_gemm
+    ok_args = dict(epi=0, bias=None, res=None, ldr=0, out=out, ldo=64)
+
+    def call(a=A, w=W, M=4, N=64, K=64, epi=0, bias=None, res=None, ldr=0, out=out, ldo=64,
+             oc=None, osf=None, og=1.0, ws=None, wsb=0):
+        return g(C.byref(a) if a is not None else None, C.byref(w) if w is not None else None, M, N, K,
+                 epi, bias, res, ldr, out, ldo, oc, osf, og, ws, wsb, None)
+
+    assert call(a=None) == 1
+    assert call(M=5) == 1                      # A->rows != M
+    assert call(epi=9) == 1
+    assert call(N=32, w=_t(rows=32, K=64)) == 2          # N % 64
+    assert call(K=48, a=_t(rows=4, K=48), w=_t(rows=64, K=48)) == 2  # K % 32
+    assert call(epi=1) == 1                    # bias required
+    assert call(epi=2) == 1                    # residual required
+    assert call(epi=4) == 1                    # FP4 epilogue needs out_codes / out_sf
+    assert call(a=_t(g=0.0)) == 1              # global scale out of range
+    assert call(a=_t(g=float("inf"))) == 1
+    assert call(ldo=60) == 1                   # ldo < N
+    assert call(out=C.c_void_p(0x3008)) == 3   # misaligned output
+    assert call(a=_t(codes=0x1004)) == 3       # misaligned codes
+    assert call(ldo=68) == 3                   # ld not a multiple of 8
+    # valid arguments reach the device check: no GPU here
+    assert call() in (5, 6)
+
+
+def test_norm_and_weight_validation(L):
+    q = L.nvfp4_quantize_norm
+    x, c, s = C.c_void_p(0x1000), C.c_void_p(0x2000), C.c_void_p(0x4000)
+    assert q(None, 0, 4, 64, 64, 0, None, None, None, None, 1e-6, 1.0, c, s, None) == 1
+    assert q(x, 0, 4, 72, 72, 0, None, None, None, None, 1e-6, 1.0, c, s, None) == 2  # K % 16
+    assert q(x, 0, 4, 64, 60, 0, None, None, None, None, 1e-6, 1.0, c, s, None) == 1  # ldx < K
+    assert q(x, 0, 4, 64, 64, 7, None, None, None, None, 1e-6, 1.0, c, s, None) == 1  # kind
+    assert q(x, 0, 4, 64, 64, 0, None, None, None, None, 1e-6, -1.0, c, s, None) == 1  # scale
+    assert q(C.c_void_p(0x1002), 0, 4, 64, 64, 0, None, None, None, None, 1e-6, 1.0, c, s, None) == 3
+    assert q(x, 0, 4, 64, 64, 0, None, None, None, None, 1e-6, 1.0, c, s, None) in (5, 6)
+    w = L.nvfp4_quantize_weight
+    gs = C.c_float()
+    assert w(x, 64, 64, 64, 0, c, s, None, x, None) == 1
+    assert w(x, 63, 64, 64, 1, c, s, C.byref(gs), x, None) == 2  # interleave needs even N
+    assert w(x, 64, 64, 64, 0, c, s, C.byref(gs), x, None) in (5, 6)

@@ -1,0 +1,97 @@
+"""GPU parity of the block-scaled NVFP4 GEMM and its fused epilogues against the oracle.
+
+Operands are quantized by the oracle and uploaded, so the GEMM is checked alone: bf16
+outputs meet the spec bar (relative error <= 1e-2 where |ref| > 1e-2 max|ref|,
+cosine >= 0.99999); FP4 outputs meet the boundary-only mismatch bar in parity.py.  Every
+tile width (64/128/256) and several split-K factors are pinned explicitly, over shapes
+that span several tiles and ragged M / K tails."""
+import numpy as np
+import pytest
+
+from parity import check_fp4_output, check_gemm_bf16, dev_bf16, host, to_gpu_fp4
+from vla_action_head_b200 import nvfp4, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _probe():
+    nvfp4.probe()
+
+
+def _operands(orc, wl, M, N, K, inter=False):
+    x = synth.bf16_normal(synth.seed_of(wl, synth.X), (M, K))
+    w = synth.bf16_normal(synth.seed_of(wl, synth.W0), (N, K), 0.0, 0.02)
+    ac, asf = orc.quantize_norm(x, "none", g=1.0)
+    wc, wsf, gw = orc.quantize_weight(w, interleave_gate_up=inter)
+    return (ac, asf, 1.0), (wc, wsf, gw)
+
+
+def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0):
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, wl, M, N, K)
+    bias = synth.bf16_normal(synth.seed_of(wl, synth.BIAS0), (N,), 0.0, 0.01)
+    res = synth.bf16_normal(synth.seed_of(wl, synth.RESIDUAL), (M, N))
+    ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res, g_out=g_out)
+    A = to_gpu_fp4(ac, asf, ga, M, K)
+    W = to_gpu_fp4(wc, wsf, gw, N, K)
+    uses_bias = epi in ("bias", "bias_residual", "bias_gelu")
+    uses_res = epi in ("residual", "bias_residual")
+    out = nvfp4.gemm(A, W, epi, bias=dev_bf16(bias) if uses_bias else None,
+                     residual=dev_bf16(res) if uses_res else None, out_global_scale=g_out,
+                     block_n=bn, splits=sp)
+    if epi in ("bias_gelu", "geglu"):
+        n_out = N // 2 if epi == "geglu" else N
+        return check_fp4_output(orc, host(out.codes), host(out.sf), ref["codes"], ref["sf"], ref["h"],
+                                g_out, M, n_out, what=(M, N, K, epi, bn, sp))
+    return check_gemm_bf16(host(out), ref["v"], what=(M, N, K, epi, bn, sp))
+
+
+SHAPES = [(41, 512, 256), (1, 64, 64), (7, 192, 96), (50, 256, 1024), (130, 384, 320), (300, 256, 512),
+          (41, 1536, 1536)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_default_schedule_bias(orc, M, N, K):
+    _run(orc, M, N, K, "bias")
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("sp", [1, 2, 3])
+def test_every_tile_and_split(orc, bn, sp):
+    _run(orc, 41, 512, 768, "bias_residual", bn=bn, sp=sp)
+    _run(orc, 130, 256, 1024, "none", bn=bn, sp=sp)
+
+
+@pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
+@pytest.mark.parametrize("M,sp", [(41, 1), (41, 4), (200, 1)])
+def test_epilogues(orc, epi, M, sp):
+    _run(orc, M, 512, 512, epi, bn=128, sp=sp)
+
+
+def test_k_tail_zero_padding(orc):
+    """K % 64 == 32: the last MMA K step reads TMA zero-fill and zero scale padding."""
+    _run(orc, 41, 128, 96, "bias", bn=64, sp=1)
+    _run(orc, 41, 128, 4320, "bias", bn=128, sp=2)
+
+
+def test_zero_activations_give_bias(orc):
+    M, N, K = 41, 256, 512
+    ac = np.zeros((M, K // 2), np.uint8)
+    asf = np.zeros(orc.sf_bytes(M, K), np.uint8)
+    (_, _, _), (wc, wsf, gw) = _operands(orc, 12, M, N, K)
+    bias = synth.bf16_normal(3, (N,), 0.0, 0.5)
+    out = nvfp4.gemm(to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K), "bias",
+                     bias=dev_bf16(bias))
+    assert np.array_equal(host(out), np.broadcast_to(bias, (M, N)))
+
+
+def test_determinism_split_k(orc):
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 13, 41, 1536, 6144)
+    A, W = to_gpu_fp4(ac, asf, ga, 41, 6144), to_gpu_fp4(wc, wsf, gw, 1536, 6144)
+    o1 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=6))
+    o2 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=6))
+    assert np.array_equal(o1, o2)
+
+
+def test_device_status_clean():
+    nvfp4.device_status()

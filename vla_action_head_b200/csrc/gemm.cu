@@ -1,0 +1,425 @@
+// gemm.cu — block-scaled NVFP4 GEMM on sm_100a tensor cores with fused epilogues.
+//
+//   acc[m, n] = sum_k e(A)[m, k] sA[m, k/16] e(W)[n, k] sW[n, k/16]      (fp32, in TMEM)
+//   v = acc * gA * gW (+ bias[n]) (+ residual[m, n])  ->  bf16, or tanh-GELU / GeGLU -> FP4
+// ("GROOT N1.7 update: Thor NVFP4 + FA4 performance tier", §What is in the tier: every DiT
+// GEMM block-scaled NVFP4 with fused bf16 bias / bias+residual / bias+tanh-GELU+FP4
+// epilogues; "Pi0.5 Thor NVFP4 End-to-End Results", §Half-Width Fused GeGLU Epilogue and
+// §Fused GeGLU FFN in the Decoder: gelu(gate)*up on pairwise-interleaved columns, 16
+// values per output scale block, GELU on the fp32 accumulator.)
+//
+// One CTA computes a 128 x BN output tile over one K range (split-K for small M, where the
+// GEMM streams weights and needs every SM pulling them).  Warp roles:
+//   warp 0      TMA producer: 2-D tiled loads of the A / W code tiles (128-byte swizzle) and
+//               1-D bulk loads of their scale-factor atoms into a STAGES-deep ring; the
+//               weight half of the first stages is issued before the programmatic-launch
+//               wait because weights never depend on the previous kernel.
+//   warp 1      tensor-memory allocation; one thread issues tcgen05.cp (scales smem->TMEM)
+//               and tcgen05.mma kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64 each).
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one row per thread), then
+//               either the fused epilogue directly, or split-K partials to the workspace
+//               with an arrival ticket; the last CTA of a tile reduces the partials in
+//               split order (deterministic) and runs the epilogue.
+// Every wait is bounded (see sm100.cuh); an expired wait records a status and the CTA
+// unwinds: copies and MMAs in flight are drained, tensor memory is freed.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gemm.h"
+#include "norm.h"
+#include "quant.cuh"
+#include "sm100.cuh"
+
+namespace nvfp4 {
+
+__device__ uint32_t g_device_status = 0;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kABytes = 128 * 128;  // one A stage: 128 rows x 128 bytes (256 FP4 values)
+constexpr int kSfAtom = 512;        // 128 rows x 4 scale blocks
+
+template <int BN>
+struct Cfg {
+    static constexpr int kSfbGroups = BN >= 128 ? BN / 128 : 1;
+    static constexpr int kBBytes = BN * 128;
+    static constexpr int kSfaBytes = 4 * kSfAtom;
+    static constexpr int kSfbBytes = kSfbGroups * 4 * kSfAtom;
+    // tensor-memory columns: accumulator, then 16 columns of A scales, then B scales
+    static constexpr int kColSfa = BN;
+    static constexpr int kColSfb = BN + 16;
+    static constexpr int kColsUsed = BN + 16 + 16 * kSfbGroups;
+    static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
+                                     : kColsUsed <= 256 ? 256 : 512;
+};
+
+template <int BN, int STAGES>
+struct Smem {
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kOffA + STAGES * kABytes;
+    static constexpr int kOffSfa = kOffB + STAGES * Cfg<BN>::kBBytes;
+    static constexpr int kOffSfb = kOffSfa + STAGES * Cfg<BN>::kSfaBytes;
+    static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes;
+    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 1) * 8;
+    static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ void named_barrier_epi() {
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float z) {
+    const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+    const float z3 = z * z * z;
+    return 0.5f * z * (1.0f + tanhf(k0 * (z + 0.044715f * z3)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// bounded wait that ignores the abort flag (used while draining before teardown)
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+    int dummy = 0;
+    return mbar_wait(bar, parity, &dummy, &g_device_status, kStatusTimeoutDrain);
+}
+
+// Epilogue of one 32-column chunk held by this thread (row m, columns n .. n + 31).
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs &p, int m, int n, float *v) {
+    const int epi = p.epi;
+    const bool has_bias = p.bias != nullptr &&
+                          (epi == kEpiBias || epi == kEpiBiasResidual || epi == kEpiBiasGelu || epi == kEpiGeglu);
+    const bool has_res = (epi == kEpiResidual || epi == kEpiBiasResidual);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], p.alpha);
+    if (has_bias) {
+        const uint4 *bq = reinterpret_cast<const uint4 *>(p.bias + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 u = __ldg(bq + j);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                v[8 * j + 2 * t] = __fadd_rn(v[8 * j + 2 * t], bf16lo(w[t]));
+                v[8 * j + 2 * t + 1] = __fadd_rn(v[8 * j + 2 * t + 1], bf16hi(w[t]));
+            }
+        }
+    }
+    if (has_res) {
+        const uint4 *rq = reinterpret_cast<const uint4 *>(p.residual + static_cast<size_t>(m) * p.ldr + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 u = rq[j];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                v[8 * j + 2 * t] = __fadd_rn(v[8 * j + 2 * t], bf16lo(w[t]));
+                v[8 * j + 2 * t + 1] = __fadd_rn(v[8 * j + 2 * t + 1], bf16hi(w[t]));
+            }
+        }
+    }
+    if (epi == kEpiBiasGelu) {
+        const float d6g = __fmul_rn(6.0f, p.g_out);
+        const int k_atoms_out = (p.N + 63) >> 6;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float y[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) y[i] = gelu_tanh_f(v[16 * h + i]);
+            uint2 c;
+            const uint32_t s = quantize_block16(y, p.g_out, d6g, c);
+            const int col = n + 16 * h;
+            *reinterpret_cast<uint2 *>(p.out_codes + static_cast<size_t>(m) * (p.N >> 1) + (col >> 1)) = c;
+            p.out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
+        }
+    } else if (epi == kEpiGeglu) {
+        const float d6g = __fmul_rn(6.0f, p.g_out);
+        const int n_out = p.N >> 1;
+        const int k_atoms_out = (n_out + 63) >> 6;
+        float y[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(gelu_tanh_f(v[2 * j]), v[2 * j + 1]);
+        uint2 c;
+        const uint32_t s = quantize_block16(y, p.g_out, d6g, c);
+        const int col = n >> 1;  // first output column of this block
+        *reinterpret_cast<uint2 *>(p.out_codes + static_cast<size_t>(m) * (n_out >> 1) + (col >> 1)) = c;
+        p.out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
+    } else {
+        uint4 *oq = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(m) * p.ldo + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            oq[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                               pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+    }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs p) {
+    using C = Cfg<BN>;
+    using S = Smem<BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + S::kOffBar;             // STAGES barriers
+    const uint32_t bar_empty = bar_full + STAGES * 8;         // STAGES barriers
+    const uint32_t bar_acc = bar_empty + STAGES * 8;          // 1 barrier
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + S::kOffMisc);
+    // misc[0] = tensor-memory base, misc[1] = abort flag, misc[2] = split-K ticket,
+    // misc[3] = accumulator-valid decision of the epilogue warps
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
+    const int n0 = n_tile * BN, m0 = m_tile * 128;
+    const int kt_begin = split * p.kt_per_split;
+    const int kt_end = min(p.k_tiles, kt_begin + p.kt_per_split);
+    const int nkt = kt_end - kt_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_acc, 1);
+        misc[1] = 0;
+        misc[2] = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t *>(misc)), C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    // Let the next kernel in the stream start its own weight prefetch.
+    pdl_launch_dependents();
+
+    auto nkb_of = [&](int kt) { return min(4, p.k_atoms - 4 * kt); };
+    auto stage_bytes = [&](int kt) {
+        return p.a_box_rows * 128u + static_cast<uint32_t>(C::kBBytes) +
+               static_cast<uint32_t>(nkb_of(kt)) * kSfAtom * (1 + C::kSfbGroups);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------ producer ------------------------------
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_a = policy_evict_last();
+            auto load_w = [&](int j) {
+                const int s = j % STAGES, kt = kt_begin + j;
+                const uint32_t full = bar_full + 8 * s;
+                const uint32_t nb = static_cast<uint32_t>(nkb_of(kt)) * kSfAtom;
+                tma_load_2d(sbase + S::kOffB + s * C::kBBytes, &tmB, kt * 128, n0, full, pol_w);
+#pragma unroll
+                for (int gi = 0; gi < C::kSfbGroups; ++gi) {
+                    const size_t grp = static_cast<size_t>(n0 / 128 + gi);
+                    bulk_load(sbase + S::kOffSfb + s * C::kSfbBytes + gi * 4 * kSfAtom,
+                              p.sfb + (grp * p.k_atoms + 4 * kt) * kSfAtom, nb, full, pol_w);
+                }
+            };
+            auto load_a = [&](int j) {
+                const int s = j % STAGES, kt = kt_begin + j;
+                const uint32_t full = bar_full + 8 * s;
+                const uint32_t nb = static_cast<uint32_t>(nkb_of(kt)) * kSfAtom;
+                tma_load_2d(sbase + S::kOffA + s * kABytes, &tmA, kt * 128, m0, full, pol_a);
+                bulk_load(sbase + S::kOffSfa + s * C::kSfaBytes,
+                          p.sfa + (static_cast<size_t>(m_tile) * p.k_atoms + 4 * kt) * kSfAtom, nb, full, pol_a);
+            };
+            const int pre = min(STAGES, nkt);
+            for (int j = 0; j < pre; ++j) {
+                mbar_arrive_expect_tx(bar_full + 8 * (j % STAGES), stage_bytes(kt_begin + j));
+                load_w(j);
+            }
+            pdl_wait();  // A and its scales come from the previous kernel
+            for (int j = 0; j < pre; ++j) load_a(j);
+            int issued = pre;
+            for (int j = pre; j < nkt; ++j) {
+                const int s = j % STAGES;
+                if (!mbar_wait(bar_empty + 8 * s, ((j / STAGES) - 1) & 1, abort_flag, &g_device_status, kStatusTimeoutEmpty)) break;
+                mbar_arrive_expect_tx(bar_full + 8 * s, stage_bytes(kt_begin + j));
+                load_w(j);
+                load_a(j);
+                issued = j + 1;
+            }
+            // drain: every issued stage must have landed before the CTA may exit
+            for (int j = max(0, issued - STAGES); j < issued; ++j)
+                drain_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------ MMA issuer ------------------------------
+            constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
+            const uint32_t t_acc = tmem;
+            const uint32_t t_sfa = tmem + C::kColSfa;
+            const uint32_t t_sfb = tmem + C::kColSfb;
+            const uint32_t sfb_sub = (BN == 64) ? static_cast<uint32_t>((n0 & 127) >> 5) : 0u;
+            for (int j = 0; j < nkt; ++j) {
+                const int s = j % STAGES, kt = kt_begin + j;
+                if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull)) break;
+                tc_fence_after();
+                const int nkb = nkb_of(kt);
+                const uint32_t a_s = sbase + S::kOffA + s * kABytes;
+                const uint32_t b_s = sbase + S::kOffB + s * C::kBBytes;
+                const uint32_t sfa_s = sbase + S::kOffSfa + s * C::kSfaBytes;
+                const uint32_t sfb_s = sbase + S::kOffSfb + s * C::kSfbBytes;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    tc_cp_32x128b_warpx4(t_sfa + 4 * kb, desc_sf_32x128b(sfa_s + kb * kSfAtom));
+#pragma unroll
+                    for (int gi = 0; gi < C::kSfbGroups; ++gi)
+                        tc_cp_32x128b_warpx4(t_sfb + 4 * C::kSfbGroups * kb + 4 * gi,
+                                             desc_sf_32x128b(sfb_s + gi * 4 * kSfAtom + kb * kSfAtom));
+                }
+                for (int kb = 0; kb < nkb; ++kb) {
+                    tc_mma_mxf4nvf4(t_acc, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb),
+                                    idesc, t_sfa + 4 * kb, t_sfb + 4 * C::kSfbGroups * kb + sfb_sub,
+                                    (j > 0 || kb > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs finished reading it
+            }
+            tc_commit(bar_acc);  // always: completion of every MMA issued above
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;  // tensor-memory sub-partition this warp may read
+        const int row = q * 32 + lane;
+        const int m = m0 + row;
+        const bool row_ok = m < p.M;
+        const bool done = drain_wait(bar_acc, 0);
+        // one decision for all four epilogue warps (tcgen05.ld and the named barriers below
+        // must be reached uniformly)
+        named_barrier_epi();
+        if (threadIdx.x == 64) misc[3] = (done && !*abort_flag) ? 1u : 0u;
+        named_barrier_epi();
+        const bool acc_ok = misc[3] != 0u;
+        tc_fence_after();
+        pdl_wait();
+        if (acc_ok) {
+            const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+            if (p.splits == 1) {
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float v[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                        epilogue_chunk(p, m, n0 + c0, v);
+                    }
+                }
+            } else {
+                // split-K: partial tile to the workspace, then an arrival ticket
+                float *part = p.partials + (static_cast<size_t>(split) * p.M) * p.N;
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float4 *dst = reinterpret_cast<float4 *>(part + static_cast<size_t>(m) * p.N + n0 + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            __stcg(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+                    }
+                }
+                __threadfence();
+                named_barrier_epi();
+                uint32_t *ticket = p.tickets + (static_cast<size_t>(m_tile) * p.n_tiles + n_tile);
+                if (threadIdx.x == 64) misc[2] = atomicAdd(ticket, 1u);
+                named_barrier_epi();
+                if (misc[2] == static_cast<uint32_t>(p.splits - 1)) {
+                    __threadfence();
+                    if (row_ok) {
+                        for (int c0 = 0; c0 < BN; c0 += 32) {
+                            float v[32];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+                            for (int sp = 0; sp < p.splits; ++sp) {
+                                const float4 *src = reinterpret_cast<const float4 *>(
+                                    p.partials + (static_cast<size_t>(sp) * p.M + m) * p.N + n0 + c0);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const float4 u = __ldcg(src + j);
+                                    v[4 * j] = __fadd_rn(v[4 * j], u.x);
+                                    v[4 * j + 1] = __fadd_rn(v[4 * j + 1], u.y);
+                                    v[4 * j + 2] = __fadd_rn(v[4 * j + 2], u.z);
+                                    v[4 * j + 3] = __fadd_rn(v[4 * j + 3], u.w);
+                                }
+                            }
+                            epilogue_chunk(p, m, n0 + c0, v);
+                        }
+                    }
+                    if (threadIdx.x == 64) *ticket = 0u;  // ready for the next call
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+    using S = Smem<BN, STAGES>;
+    static bool attr_set = false;  // per device is enough in practice; set idempotently
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             S::kBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_tiles, (p.M + 127) / 128, p.splits);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = S::kBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, STAGES>, ta, tb, p);
+}
+
+}  // namespace
+
+cudaError_t probe_gemm_kernels() {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, gemm_kernel<128, 5>);
+}
+
+cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out) {
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(out, g_device_status, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    const uint32_t zero = 0;
+    return cudaMemcpyToSymbol(g_device_status, &zero, sizeof(uint32_t));
+}
+
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
+                        cudaStream_t s) {
+    switch (block_n) {
+    case 64: return launch_bn<64, 6>(ta, tb, p, s);
+    case 128: return launch_bn<128, 5>(ta, tb, p, s);
+    case 256: return launch_bn<256, 3>(ta, tb, p, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,44 @@
+// gemm.h — internal interface between the C ABI (api.cu) and the GEMM kernel (gemm.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace nvfp4 {
+
+enum { kEpiNone = 0, kEpiBias = 1, kEpiResidual = 2, kEpiBiasResidual = 3, kEpiBiasGelu = 4, kEpiGeglu = 5 };
+
+struct GemmArgs {
+    int M, N, K;
+    int k_atoms;       // ceil(K / 64): scale atoms per 128-row group
+    int k_tiles;       // ceil(K / 256): pipeline K tiles
+    int kt_per_split;  // K tiles per split
+    int splits;
+    int n_tiles;
+    uint32_t a_box_rows;  // rows per A TMA box (min(128, M rounded up to 8))
+    const uint8_t *sfa;
+    const uint8_t *sfb;
+    float alpha;  // gA * gW
+    int epi;
+    const uint16_t *bias;
+    const uint16_t *residual;
+    int ldr;
+    uint16_t *out;
+    int ldo;
+    uint8_t *out_codes;
+    uint8_t *out_sf;
+    float g_out;
+    float *partials;    // split-K: [splits, M, N] fp32
+    uint32_t *tickets;  // split-K: one word per output tile
+};
+
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
+                        cudaStream_t s);
+
+// Reads the device status word and clears it (after synchronising `s`).
+cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out);
+
+}  // namespace nvfp4

@@ -1,0 +1,29 @@
+// norm.h — internal interface between the C ABI (api.cu) and the norm / quantizer kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+struct NormArgs {
+    const void *x;
+    int M, K, ldx;
+    int kind;  // nvfp4_norm
+    const uint16_t *gamma, *beta, *scale, *shift;
+    float eps;
+    float g;                    // global decode scale (activation path)
+    const uint32_t *amax_bits;  // weight path: g = amax / 2688 computed from this word
+    int interleave;             // weight path: pairwise gate/up row interleave
+    uint8_t *codes;
+    uint8_t *sf;
+    float *y_out;  // non-NULL: write the normalized fp32 y instead of quantizing
+};
+
+cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s);
+cudaError_t launch_weight_amax(const uint16_t *w, int N, int K, int ldw, uint32_t *amax_bits, cudaStream_t s);
+cudaError_t probe_norm_kernels();
+cudaError_t probe_gemm_kernels();
+
+}  // namespace nvfp4

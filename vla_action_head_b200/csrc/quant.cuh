@@ -1,0 +1,55 @@
+// quant.cuh — the per-16 NVFP4 block quantizer and the scale-factor layout, as device
+// functions shared by the norm front-end, the weight quantizer and the GEMM epilogues.
+//
+// Block quantizer ("GROOT N1.7 update: Thor NVFP4 + FA4 performance tier", §What is in the
+// tier: one UE4M3 scale per 16 elements computed at run time; "Pi0.5 Thor NVFP4 End-to-End
+// Results", §Implemented Path: native E2M1 conversion, round-to-nearest-even):
+//   a = max|y|;  t = a / (6 g);  s = E4M3_rn_satfinite(t);  S = dec(s) g
+//   dec(s) == 0 -> all codes +0;  else  code_i = E2M1_rn_satfinite(y_i * (1 / S))
+// Every step is one fp32 operation rounded to nearest even (explicit _rn intrinsics, so
+// the compiler cannot contract or reassociate them).
+#pragma once
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace nvfp4 {
+
+// Scale-factor byte offset: 512-byte atoms of 128 rows x 4 blocks (K rounded up to 64
+// elements), atoms ordered K fastest then 128-row group; inside an atom row r, block c at
+// (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4 ("Pi0.5 ...", §Encoder Attention QKV NVFP4 +
+// Scale-Factor Zero-Init: tile-interleaved layouts round K up to 64-element atoms).
+__host__ __device__ __forceinline__ size_t sf_offset(int row, int kblk, int k_atoms) {
+    const size_t atom = static_cast<size_t>(row >> 7) * k_atoms + (kblk >> 2);
+    return atom * 512 + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (kblk & 3);
+}
+
+// Quantizes y[0..15]; d6g = 6 * g (fp32).  Writes 8 code bytes (element 0 in the low
+// nibble of byte 0) and returns the scale byte.
+__device__ __forceinline__ uint32_t quantize_block16(const float *y, float g, float d6g,
+                                                     uint2 &codes) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(y[i]));
+    const float t = __fdiv_rn(a, d6g);
+    const uint32_t s = cvt_e4m3_rn_satfinite(t);
+    const float ds = e4m3_to_f32(s);
+    if (ds == 0.0f) {
+        codes = make_uint2(0u, 0u);
+        return s;
+    }
+    const float S = __fmul_rn(ds, g);
+    const float r = __frcp_rn(S);
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], r);
+    codes.x = cvt_e2m1x8(v);
+    codes.y = cvt_e2m1x8(v + 8);
+    return s;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+}  // namespace nvfp4

@@ -1,0 +1,228 @@
+"""Python binding of libnvfp4.so (include/nvfp4.h).
+
+Argument marshalling only: torch supplies device memory and the current CUDA stream; every
+step of the computation runs in the library's sm_100a kernels.  There is no fallback: if
+the library is missing or the device is not sm_100, calls raise.
+
+Raw entry points keep their C names (`nvfp4_quantize_norm`, `nvfp4_quantize_weight`,
+`nvfp4_gemm`, ...) and take plain integers / pointers.  The lower-case helpers
+(`quantize_norm`, `quantize_weight`, `gemm`, ...) accept torch tensors and allocate outputs.
+"""
+import ctypes as C
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
+
+NORM = {"none": 0, "layernorm": 1, "rmsnorm": 2, "adaln": 3, "adarms": 4}
+EPI = {"none": 0, "bias": 1, "residual": 2, "bias_residual": 3, "bias_gelu": 4, "geglu": 5}
+IN_BF16, IN_FP32 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned",
+          4: "workspace", 5: "unsupported device", 6: "CUDA error", 7: "timeout"}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, call, status):
+        super().__init__(f"{call} failed: {status} ({STATUS.get(status, '?')})")
+        self.status = status
+
+
+class _Tensor(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("sf", C.c_void_p), ("global_scale", C.c_float),
+                ("rows", C.c_int), ("K", C.c_int)]
+
+
+_lib = None
+P, I, F, SZ = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+
+
+def lib():
+    """Loads libnvfp4.so (built in-tree by vla_action_head_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run vla_action_head_b200.build.build()")
+        L = C.CDLL(LIB_PATH)
+        sig = {
+            "nvfp4_probe": (I, []),
+            "nvfp4_status_string": (C.c_char_p, [I]),
+            "nvfp4_sf_bytes": (SZ, [I, I]),
+            "nvfp4_sf_offset": (SZ, [I, I, I]),
+            "nvfp4_sf_zero": (I, [P, I, I, P]),
+            "nvfp4_gemm_workspace_bytes": (SZ, [I, I, I]),
+            "nvfp4_gemm_workspace_bytes_ex": (SZ, [I, I, I, I, I]),
+            "nvfp4_get_device_status": (I, [P]),
+            "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
+            "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
+            "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
+            "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
+                               F, P, SZ, P]),
+            "nvfp4_gemm_ex": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P,
+                                  P, F, P, SZ, I, I, P]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions():
+    """Names of the functions include/nvfp4.h declares."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:nvfp4_status|size_t|const char \*)\s*(nvfp4_\w+)\(", txt, re.M)))
+
+
+def _check(call, st):
+    if st != 0:
+        raise NVFP4Error(call, st)
+
+
+# ---- torch-facing helpers ---------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return C.c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+@dataclass
+class NVFP4Tensor:
+    """FP4 codes [rows, K/2] (uint8), scale bytes (uint8, nvfp4_sf_bytes), global scale."""
+    codes: "object"
+    sf: "object"
+    global_scale: float
+    rows: int
+    K: int
+
+    def c(self):
+        return _Tensor(self.codes.data_ptr(), self.sf.data_ptr(), self.global_scale, self.rows, self.K)
+
+
+def sf_bytes(rows, K):
+    return int(lib().nvfp4_sf_bytes(rows, K))
+
+
+def empty_fp4(rows, K, device="cuda", global_scale=1.0):
+    """Output buffers for an FP4 tensor; the scale buffer is zeroed (padding must be 0)."""
+    torch = _torch()
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=device)
+    sf = torch.zeros(sf_bytes(rows, K), dtype=torch.uint8, device=device)
+    return NVFP4Tensor(codes, sf, global_scale, rows, K)
+
+
+def quantize_norm(x, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
+                  global_scale=1.0, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:
+    torch = _torch()
+    M, K = x.shape
+    dt = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    if out is None:
+        out = empty_fp4(M, K, x.device, global_scale)
+    st = lib().nvfp4_quantize_norm(_ptr(x), dt, M, K, x.stride(0), NORM[kind], _ptr(gamma), _ptr(beta),
+                                   _ptr(scale), _ptr(shift), eps, global_scale, _ptr(out.codes),
+                                   _ptr(out.sf), _stream())
+    _check("nvfp4_quantize_norm", st)
+    out.global_scale = global_scale
+    return out
+
+
+def norm_f32(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, out=None):
+    torch = _torch()
+    M, K = x.shape
+    dt = IN_FP32 if x.dtype == torch.float32 else IN_BF16
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    st = lib().nvfp4_norm_f32(_ptr(x), dt, M, K, x.stride(0), NORM[kind], _ptr(gamma), _ptr(beta),
+                              _ptr(scale), _ptr(shift), eps, _ptr(out), _stream())
+    _check("nvfp4_norm_f32", st)
+    return out
+
+
+_scratch = {}
+
+
+def quantize_weight(w, interleave_gate_up=False) -> NVFP4Tensor:
+    torch = _torch()
+    N, K = w.shape
+    out = empty_fp4(N, K, w.device)
+    dev = w.device.index if w.device.index is not None else torch.cuda.current_device()
+    if dev not in _scratch:
+        _scratch[dev] = torch.zeros(256, dtype=torch.uint8, device=w.device)
+    g = C.c_float(0.0)
+    st = lib().nvfp4_quantize_weight(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)),
+                                     _ptr(out.codes), _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]),
+                                     _stream())
+    _check("nvfp4_quantize_weight", st)
+    out.global_scale = g.value
+    return out
+
+
+class Workspace:
+    """Caller-owned GEMM workspace: zeroed once when (re)allocated, reused across calls."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes):
+        torch = _torch()
+        if nbytes == 0:
+            return None, 0
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=self.device)
+        return self.buf, self.buf.numel()
+
+
+_default_ws = {}
+
+
+def gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None,
+         out_global_scale=1.0, workspace: Optional[Workspace] = None, block_n=0, splits=0):
+    """a: M x K, w: N x K.  bf16 epilogues return bf16 [M, N]; FP4 epilogues an NVFP4Tensor."""
+    torch = _torch()
+    M, N, K = a.rows, w.rows, a.K
+    e = EPI[epi]
+    fp4 = e in (4, 5)
+    if out is None:
+        if fp4:
+            out = empty_fp4(M, N // 2 if e == 5 else N, a.codes.device, out_global_scale)
+        else:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=a.codes.device)
+    if workspace is None:
+        dev = a.codes.device.index if a.codes.device.index is not None else torch.cuda.current_device()
+        workspace = _default_ws.setdefault(dev, Workspace(a.codes.device))
+    need = lib().nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits)
+    ws, ws_bytes = workspace.get(need)
+    ta, tw = a.c(), w.c()
+    ldr = residual.stride(0) if residual is not None else 0
+    if fp4:
+        st = lib().nvfp4_gemm_ex(C.byref(ta), C.byref(tw), M, N, K, e, _ptr(bias), _ptr(residual), ldr,
+                                 None, 0, _ptr(out.codes), _ptr(out.sf), out_global_scale, _ptr(ws),
+                                 ws_bytes, block_n, splits, _stream())
+        out.global_scale = out_global_scale
+    else:
+        st = lib().nvfp4_gemm_ex(C.byref(ta), C.byref(tw), M, N, K, e, _ptr(bias), _ptr(residual), ldr,
+                                 _ptr(out), out.stride(0), None, None, 1.0, _ptr(ws), ws_bytes, block_n,
+                                 splits, _stream())
+    _check("nvfp4_gemm", st)
+    return out
+
+
+def probe():
+    _check("nvfp4_probe", lib().nvfp4_probe())
+
+
+def device_status():
+    """Raises NVFP4Error(TIMEOUT) if a kernel's bounded wait expired since the last check."""
+    _check("nvfp4_get_device_status", lib().nvfp4_get_device_status(_stream()))
