@@ -27,15 +27,15 @@ def _operands(orc, wl, M, N, K, inter=False):
     return (ac, asf, 1.0), (wc, wsf, gw)
 
 
-def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0):
+def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0, geglu_bias=False):
     (ac, asf, ga), (wc, wsf, gw) = _operands(orc, wl, M, N, K)
-    bias = synth.bf16_normal(synth.seed_of(wl, synth.BIAS0), (N,), 0.0, 0.01)
-    res = synth.bf16_normal(synth.seed_of(wl, synth.RESIDUAL), (M, N))
+    uses_bias = epi in ("bias", "bias_residual", "bias_gelu") or (epi == "geglu" and geglu_bias)
+    uses_res = epi in ("residual", "bias_residual")
+    bias = synth.bf16_normal(synth.seed_of(wl, synth.BIAS0), (N,), 0.0, 0.01) if uses_bias else None
+    res = synth.bf16_normal(synth.seed_of(wl, synth.RESIDUAL), (M, N)) if uses_res else None
     ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res, g_out=g_out)
     A = to_gpu_fp4(ac, asf, ga, M, K)
     W = to_gpu_fp4(wc, wsf, gw, N, K)
-    uses_bias = epi in ("bias", "bias_residual", "bias_gelu")
-    uses_res = epi in ("residual", "bias_residual")
     out = nvfp4.gemm(A, W, epi, bias=dev_bf16(bias) if uses_bias else None,
                      residual=dev_bf16(res) if uses_res else None, out_global_scale=g_out,
                      block_n=bn, splits=sp)
@@ -66,6 +66,12 @@ def test_every_tile_and_split(orc, bn, sp):
 @pytest.mark.parametrize("M,sp", [(41, 1), (41, 4), (200, 1)])
 def test_epilogues(orc, epi, M, sp):
     _run(orc, M, 512, 512, epi, bn=128, sp=sp)
+
+
+@pytest.mark.parametrize("g_out", [1.0, 0.02])
+def test_geglu_with_bias_and_scale(orc, g_out):
+    _run(orc, 50, 1024, 1024, "geglu", bn=256, sp=1, g_out=g_out, geglu_bias=True)
+    _run(orc, 50, 1024, 1024, "bias_gelu", bn=64, sp=2, g_out=g_out)
 
 
 def test_k_tail_zero_padding(orc):

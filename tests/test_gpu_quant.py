@@ -48,7 +48,9 @@ def _crafted_blocks():
     rng = np.random.default_rng(0)
     r = rng.standard_normal((256, 16)).astype(np.float32)
     r *= np.exp(rng.uniform(-12, 9, (256, 1))).astype(np.float32)
-    return np.concatenate([np.stack(rows), r]).astype(np.float32)
+    out = np.concatenate([np.stack(rows), r]).astype(np.float32)
+    pad = (-len(out)) % 4
+    return np.concatenate([out, np.zeros((pad, 16), np.float32)])
 
 
 @pytest.mark.parametrize("g", [1.0, 0.37, 2.0 ** -20])

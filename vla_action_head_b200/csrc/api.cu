@@ -123,6 +123,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 5) return NVFP4_ERR_INVALID_ARG;
     if (K % 32 != 0 || N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!scale_ok(A->global_scale) || !scale_ok(W->global_scale)) return NVFP4_ERR_INVALID_ARG;
+    if (M == 0) return NVFP4_OK;  // nothing to read or write
     const bool fp4_out = (epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
     const bool need_bias = (epi == NVFP4_EPI_BIAS || epi == NVFP4_EPI_BIAS_RESIDUAL || epi == NVFP4_EPI_BIAS_GELU);
     const bool need_res = (epi == NVFP4_EPI_RESIDUAL || epi == NVFP4_EPI_BIAS_RESIDUAL);
@@ -143,7 +144,6 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if ((bias && !aligned16(bias)) || (need_res && !aligned16(residual))) return NVFP4_ERR_MISALIGNED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-    if (M == 0) return NVFP4_OK;
 
     Schedule sc;
     if (block_n == 0 && splits == 0) {
@@ -202,6 +202,7 @@ nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, 
     if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32) return NVFP4_ERR_INVALID_ARG;
     if (static_cast<int>(kind) < 0 || static_cast<int>(kind) > 4) return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0 || K > (dt == NVFP4_IN_FP32 ? 16384 : 32768)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return NVFP4_OK;  // nothing to read or write
     if (x == nullptr || ldx < K) return NVFP4_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return NVFP4_ERR_INVALID_ARG;
     if (y_out == nullptr) {
@@ -215,7 +216,6 @@ nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, 
         if (pp != nullptr && !aligned16(pp)) return NVFP4_ERR_MISALIGNED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-    if (M == 0) return NVFP4_OK;
     NormArgs a = {};
     a.x = x;
     a.M = M;
