@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 linear path on B200: prints ONE JSON line (rank 0).
+
+Step = one forward pass of a stack of L distinct DiT layers at M = 41 tokens, hidden 1536
+(per layer: AdaLN->FP4, QKV GEMM +bias, context quantize, attention-output GEMM
++bias+residual, LayerNorm->FP4, FFN-up GEMM +bias+tanh-GELU->FP4, FFN-down GEMM
++bias+residual: 7 kernels), replayed from a CUDA graph.  L = 24 puts 382 MB of distinct
+weights behind each step, 3x the 126 MB L2, so every layer streams its weights from HBM.
+Metric: microseconds per layer (lower is better), plus the weight-stream GB/s it implies.
+
+Side measurements in the same line: the GEMM kernel's roofline (CUDA events around graph
+replays of each DiT GEMM over L distinct weight copies), the M = 968 prefill layer's
+TFLOPS (tensor-bound), the 18-layer action-expert stack, the M sweep on 1536 -> 6144, and
+the oracle on the host cores (cpu_baseline).
+
+--impl reference times the oracle (the reference arm of this build) on the same workload.
+Multi-GPU (torchrun): independent replicas, one per rank; timing is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear µs/layer & weight-stream GB/s at M=41; TFLOPS at M=968"
+UNIT = "µs/layer"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0  # nominal dense ratio, 9 PF / 2.25 PF
+DIT = dict(M=41, H=1536, F=6144)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=24)
+    ap.add_argument("--no-side", action="store_true", help="skip the side measurements")
+    ap.add_argument("--profile-case", default=None,
+                    help="run one small case for ncu (dit-gemms | prefill-gemms | norm) and exit")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampler (every 100 ms) bracketing a timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, v):
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+def gemm_bytes(M, N, K, epi):
+    """Algorithmic bytes of one GEMM: A and W codes + scales, output, bias, residual."""
+    b = M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16
+    if epi == "geglu":
+        b += M * (N // 2) // 2 + M * (N // 2) // 16
+    elif epi == "bias_gelu":
+        b += M * N // 2 + M * N // 16
+    else:
+        b += 2 * M * N
+    if epi in ("bias", "bias_residual", "bias_gelu"):
+        b += 2 * N
+    if epi in ("residual", "bias_residual"):
+        b += 2 * M * N
+    return b
+
+
+def time_graph(g, reps, stream):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps  # ms per replay
+
+
+def capture(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def gemm_ring_time(A, lins, epi, outs, ws, stream, reps=20, res=None):
+    """Average time (ms) of one GEMM launch over a graph of len(lins) distinct weights."""
+    from vla_action_head_b200 import nvfp4
+
+    def body():
+        for i, lin in enumerate(lins):
+            nvfp4.gemm(A, lin.w, epi, bias=lin.bias, residual=res, out=outs[i % len(outs)], workspace=ws)
+    body()  # sizes the workspace before capture
+    g = capture(body, stream)
+    ms = time_graph(g, reps, stream)
+    del g
+    return ms / len(lins)
+
+
+# ---------------------------------------------------------------------------------------
+def cpu_baseline_dit(steps=1):
+    """The oracle (single-threaded C, fp64 GEMM) on one full DiT layer at M = 41."""
+    import numpy as np
+    import torch
+
+    from oracle import oracle as orc
+    from vla_action_head_b200 import synth
+
+    M, H, F = DIT["M"], DIT["H"], DIT["F"]
+    s = lambda tid: synth.seed_of(2, tid)  # noqa: E731
+    cpu = lambda seed, shape, m, sd: synth.bf16_normal_torch(seed, shape, m, sd, device="cpu").view(  # noqa: E731
+        torch.int16).numpy().view(np.uint16)
+    x = cpu(s(synth.X), (M, H), 0, 1)
+    ctx = cpu(s(synth.CONTEXT), (M, H), 0, 1)
+    sc, sh = cpu(s(synth.MOD_SCALE), (H,), 0, 0.1), cpu(s(synth.MOD_SHIFT), (H,), 0, 0.1)
+    ga, be = cpu(s(synth.GAMMA), (H,), 1, 0.1), cpu(s(synth.BETA), (H,), 0, 0.1)
+    shapes = [(3 * H, H), (H, H), (F, H), (H, F)]
+    W = [orc.quantize_weight(cpu(s(synth.W0 + i), shp, 0, 0.02)) for i, shp in enumerate(shapes)]
+    B = [cpu(s(synth.BIAS0 + i), (shp[0],), 0, 0.01) for i, shp in enumerate(shapes)]
+
+    def bf16(v):
+        return synth.f32_to_bf16_bits(v.astype(np.float32))
+
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        a1, a1s = orc.quantize_norm(x, "adaln", scale=sc, shift=sh, eps=1e-6)
+        orc.gemm(a1, a1s, 1.0, M, W[0][0], W[0][1], W[0][2], 3 * H, H, epi="bias", bias=B[0])
+        c, cs = orc.quantize_norm(ctx, "none")
+        h = bf16(orc.gemm(c, cs, 1.0, M, W[1][0], W[1][1], W[1][2], H, H, epi="bias_residual", bias=B[1],
+                          residual=x)["v"])
+        a2, a2s = orc.quantize_norm(h, "layernorm", gamma=ga, beta=be, eps=1e-5)
+        u = orc.gemm(a2, a2s, 1.0, M, W[2][0], W[2][1], W[2][2], F, H, epi="bias_gelu", bias=B[2])
+        orc.gemm(u["codes"], u["sf"], 1.0, M, W[3][0], W[3][1], W[3][2], H, F, epi="bias_residual",
+                 bias=B[3], residual=h)
+    dt = time.perf_counter() - t0
+    return dt / steps * 1e6  # us per layer
+
+
+def reference_arm(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    # each step is one full DiT layer on the oracle (~1.6 s); the run is bounded to ~3 min by
+    # timing at most as many of the K steps as fit, which the line states in its sample
+    t0 = time.perf_counter()
+    cpu_baseline_dit(1)
+    per = time.perf_counter() - t0
+    for _ in range(max(0, min(args.warmup, int(30 / per)) - 1)):
+        cpu_baseline_dit(1)
+    n = max(1, min(args.steps, int(150 / max(per, 1e-3))))
+    us = cpu_baseline_dit(n)
+    line = {"metric": METRIC, "value": round(us, 1), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(us / 1e3, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "one DiT layer, M=41, hidden 1536, FFN 6144 (oracle, fp64 GEMM)",
+                       "global_batch": DIT["M"], "parallelism": "replicas" if ws > 1 else "single"},
+            "cpu_baseline": {"value": round(us, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"one full DiT layer per step; {n} of {args.steps} steps timed"},
+            "e2e": {"value": round(us, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------
+def profile_case(name):
+    """Small, short runs of single kernels for ncu (a few launches, a few hundred MB)."""
+    import torch
+
+    from vla_action_head_b200 import layers, nvfp4
+    torch.cuda.set_device(0)
+    nvfp4.probe()
+    if name == "dit-gemms":
+        lay = layers.DiTLayer(**DIT)
+        x = torch.randn(DIT["M"], DIT["H"], device="cuda").to(torch.bfloat16)
+        y = torch.empty_like(x)
+        for _ in range(3):
+            lay.forward(x, x, y)
+    elif name == "prefill-gemms":
+        lay = layers.PrefillLayer()
+        x = torch.randn(968, 2048, device="cuda").to(torch.bfloat16)
+        y = torch.empty_like(x)
+        for _ in range(3):
+            lay.forward(x, x, y)
+    elif name == "norm":
+        x = torch.randn(968, 2048, device="cuda").to(torch.bfloat16)
+        g = torch.ones(2048, device="cuda").to(torch.bfloat16)
+        for _ in range(3):
+            nvfp4.quantize_norm(x, "rmsnorm", gamma=g)
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    print(json.dumps({"profile_case": name, "ok": True}))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return reference_arm(args)
+    if args.profile_case:
+        return profile_case(args.profile_case)
+    import torch
+
+    from vla_action_head_b200 import build, layers, nvfp4, synth
+    build.build()
+    ws_n, rank, local = dist_setup()
+    nvfp4.probe()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.Stream()
+    pk, pk_kind = peaks()
+    L, M, H, F = args.layers, DIT["M"], DIT["H"], DIT["F"]
+
+    # ---- the DiT stack (main metric) ----
+    with torch.cuda.stream(stream):
+        wsp = nvfp4.Workspace(dev)
+        stack = [layers.DiTLayer(**DIT, layer=i, device=dev, ws=wsp) for i in range(L)]
+        x0 = synth.bf16_normal_torch(synth.seed_of(2, synth.X), (M, H), device=dev)
+        ctx = synth.bf16_normal_torch(synth.seed_of(2, synth.CONTEXT), (M, H), device=dev)
+        buf = [x0.clone(), torch.empty_like(x0)]
+    torch.cuda.synchronize()
+
+    def stack_fwd():
+        for i, lay in enumerate(stack):
+            lay.forward(buf[i % 2], ctx, buf[(i + 1) % 2])
+
+    with torch.cuda.stream(stream):
+        stack_fwd()  # eager pass: sizes the workspace, loads the kernels
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    g_stack = capture(stack_fwd, stream)
+
+    def run_steps(n, with_copies=None):
+        for _ in range(n):
+            if with_copies:
+                buf[0].copy_(with_copies[0], non_blocking=True)
+            g_stack.replay()
+            if with_copies:
+                with_copies[1].copy_(buf[L % 2], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    clk = Clocks(local)
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        run_steps(max(1, 200 // max(1, L // 24)))  # ~soak so the sampler sees the load
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        run_steps(args.steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    clocks = clk.stop()
+    ms_total = max_over_ranks(ws_n, e0.elapsed_time(e1))
+    nvfp4.device_status()
+    us_layer = ms_total * 1e3 / (args.steps * L * ws_n)
+    w_bytes = sum(l.weight_bytes() for l in stack[0].linears())
+    gbs_weights = w_bytes / (us_layer * 1e-6) / 1e9
+
+    # ---- end to end through the same API with host buffers ----
+    xh = torch.empty((M, H), dtype=torch.bfloat16).pin_memory()
+    yh = torch.empty((M, H), dtype=torch.bfloat16).pin_memory()
+    xh.copy_(x0.cpu())
+    with torch.cuda.stream(stream):
+        run_steps(2, (xh, yh))
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        run_steps(args.steps, (xh, yh))
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    ms_e2e = max_over_ranks(ws_n, e0.elapsed_time(e1))
+    us_layer_e2e = ms_e2e * 1e3 / (args.steps * L * ws_n)
+
+    line = {"metric": METRIC, "value": round(us_layer, 3), "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3) -> fp32 acc; bf16 io",
+            "data": "synthetic",
+            "config": {"workload": f"DiT layer stack, {L} distinct layers per step, M=41 tokens, hidden 1536, "
+                                   "FFN 6144, AdaLN/LayerNorm->NVFP4, 4 NVFP4 GEMMs with fused epilogues",
+                       "global_batch": M, "layers_per_step": L, "parallelism": f"replicas x{ws_n}",
+                       "l2": f"inputs larger than L2: {L} x {w_bytes / 1e6:.1f} MB distinct weights per step",
+                       "graph": "CUDA graph replay, programmatic dependent launch"},
+            "weight_stream_gbs": round(gbs_weights, 1),
+            "clocks": clocks,
+            "gpu_launches": args.steps * L * layers.DiTLayer.launches,
+            "e2e": {"value": round(us_layer_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": M * H * 2,
+                    "d2h_bytes_per_step": M * H * 2}}
+
+    del g_stack
+    if not args.no_side:
+        try:
+            line.update(side_measurements(stack, wsp, stream, dev, pk, pk_kind))
+        except Exception as e:  # a side measurement never hides the main line
+            line["side_error"] = repr(e)[:300]
+    if rank == 0 and ws_n == 1:
+        try:
+            us_cpu = cpu_baseline_dit(1)
+            line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                                    "sample": "one full DiT layer (M=41, hidden 1536, FFN 6144), fp64 GEMM, "
+                                              "single-threaded C"}
+        except Exception as e:  # the baseline is reported, never required
+            line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": str(e)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
+    import torch
+
+    from vla_action_head_b200 import layers, nvfp4, synth
+    M, H, F = DIT["M"], DIT["H"], DIT["F"]
+    out = {}
+    # ---- roofline of the GEMM kernel in the DiT layer (HBM-bound at M = 41) ----
+    l0 = stack[0]
+    per = {}
+    tot_b, tot_ms = 0, 0.0
+    specs = [("qkv", l0.a1, "qkv", "bias", 3 * H, H), ("attn_out", l0.ctx_q, "o", "bias_residual", H, H),
+             ("ffn_up", l0.a2, "up", "bias_gelu", F, H), ("ffn_down", l0.u, "down", "bias_residual", H, F)]
+    res = torch.zeros((M, H), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(stream):
+        for name, A, attr, epi, N, K in specs:
+            lins = [getattr(s, attr) for s in stack]
+            if epi == "bias_gelu":
+                outs = [nvfp4.empty_fp4(M, N, dev) for _ in range(2)]
+            else:
+                outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            ms = gemm_ring_time(A, lins, epi, outs, wsp, stream, res=res if "residual" in epi else None)
+            b = gemm_bytes(M, N, K, epi)
+            per[name] = {"us": round(ms * 1e3, 3), "gbs": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}
+            tot_b += b
+            tot_ms += ms
+    ach = tot_b / (tot_ms * 1e-3) / 1e9
+    out["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                       "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+                       "kernel": "gemm_kernel (4 DiT GEMMs, M=41, L2-cold weights)", "peak_kind": pk_kind,
+                       "per_gemm": per}
+    # ---- 18-layer action-expert stack (config 3 layers, one CUDA graph) ----
+    with torch.cuda.stream(stream):
+        ae = [layers.ActionExpertLayer(layer=i, device=dev, ws=wsp) for i in range(18)]
+        xa = synth.bf16_normal_torch(synth.seed_of(3, synth.X), (50, 1024), device=dev)
+        ca = synth.bf16_normal_torch(synth.seed_of(3, synth.CONTEXT), (50, 2048), device=dev)
+        ab = [xa.clone(), torch.empty_like(xa)]
+
+        def ae_fwd():
+            for i, lay in enumerate(ae):
+                lay.forward(ab[i % 2], ca, ab[(i + 1) % 2])
+        ae_fwd()
+    torch.cuda.synchronize()
+    g = capture(ae_fwd, stream)
+    ms = time_graph(g, 50, stream)
+    del g
+    ae_w = sum(l.weight_bytes() for l in ae[0].linears())
+    out["action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
+                                    "weight_stream_gbs": round(18 * ae_w / (ms * 1e-3) / 1e9, 1)}
+    del ae, xa, ca, ab
+    # ---- prefill layer at M = 968 (tensor-bound): ring of 4 distinct layers ----
+    with torch.cuda.stream(stream):
+        pre = [layers.PrefillLayer(layer=i, device=dev, ws=wsp) for i in range(4)]
+        xp = synth.bf16_normal_torch(synth.seed_of(4, synth.X), (968, 2048), device=dev)
+        yp = torch.empty_like(xp)
+
+        def pre_fwd():
+            for lay in pre:
+                lay.forward(xp, xp, yp)
+        pre_fwd()
+    torch.cuda.synchronize()
+    g = capture(pre_fwd, stream)
+    ms = time_graph(g, 10, stream) / len(pre)
+    del g
+    fl = pre[0].flops()
+    tf = fl / (ms * 1e-3) / 1e12
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    # the gate_up GEMM alone (dominant kernel of the layer)
+    with torch.cuda.stream(stream):
+        outs = [nvfp4.empty_fp4(968, 16384, dev) for _ in range(2)]
+        ms_gu = gemm_ring_time(pre[0].a2, [p.gate_up for p in pre], "geglu", outs, wsp, stream, reps=10)
+    tf_gu = 2.0 * 968 * 32768 * 2048 / (ms_gu * 1e-3) / 1e12
+    out["prefill_m968"] = {"us_per_layer": round(ms * 1e3, 2), "tflops": round(tf, 1),
+                           "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1)}
+    out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_peak, 1),
+                            "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4), "traffic": None,
+                            "kernel": "gemm_kernel gate_up 968x32768x2048 GeGLU->FP4",
+                            "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)"}
+    del pre, xp, yp, outs
+    # ---- M sweep on the 1536 -> 6144 GEMM (bias, bf16 out), 48 distinct weights ----
+    with torch.cuda.stream(stream):
+        lins = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(5, 1000 + i), (6144, 1536), 0, 0.02,
+                                                      device=dev),
+                              synth.bf16_normal_torch(synth.seed_of(5, 2000 + i), (6144,), 0, 0.01, device=dev))
+                for i in range(48)]
+    sweep = []
+    for Ms in (1, 16, 41, 128, 512, 968):
+        with torch.cuda.stream(stream):
+            xs = synth.bf16_normal_torch(synth.seed_of(5, Ms), (Ms, 1536), device=dev)
+            A = nvfp4.quantize_norm(xs, "none")
+            outs = [torch.empty((Ms, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            ms = gemm_ring_time(A, lins, "bias", outs, wsp, stream, reps=10)
+        b = gemm_bytes(Ms, 6144, 1536, "bias")
+        sweep.append({"M": Ms, "us": round(ms * 1e3, 3), "gbs": round(b / (ms * 1e-3) / 1e9, 1),
+                      "tflops": round(2.0 * Ms * 6144 * 1536 / (ms * 1e-3) / 1e12, 2)})
+    out["m_sweep_1536x6144"] = sweep
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

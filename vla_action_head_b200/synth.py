@@ -64,3 +64,40 @@ def bf16_normal(seed: int, shape, mean: float = 0.0, std: float = 1.0) -> np.nda
 
 def seed_of(workload: int, tensor_id: int) -> int:
     return 1000 * workload + tensor_id
+
+
+# ---- the same recipe evaluated with torch on a device (large timing inputs) ----------
+def _signed(c: int) -> int:
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def bf16_normal_torch(seed: int, shape, mean: float = 0.0, std: float = 1.0, device="cuda"):
+    """SplitMix64 -> Box-Muller -> bf16, computed with torch int64 / fp64 tensors on
+    `device`.  Same recipe as bf16_normal; the device's log / sin / cos may differ from
+    numpy's in the last fp64 bit, so a rare value can differ by one bf16 step.  Used for
+    timing inputs, never for a parity comparison."""
+    import torch
+    n = 1
+    for s in shape:
+        n *= int(s)
+    m = (n + 1) // 2
+
+    def lsr(z, s):  # logical shift right of the 64-bit pattern
+        return (z >> s) & ((1 << (64 - s)) - 1)
+
+    z = torch.arange(1, 2 * m + 1, dtype=torch.int64, device=device)
+    z.mul_(_signed(0x9E3779B97F4A7C15)).add_(_signed(seed & 0xFFFFFFFFFFFFFFFF))
+    z = z ^ lsr(z, 30)
+    z.mul_(_signed(0xBF58476D1CE4E5B9))
+    z = z ^ lsr(z, 27)
+    z.mul_(_signed(0x94D049BB133111EB))
+    z = z ^ lsr(z, 31)
+    u = (lsr(z, 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    del z
+    r = torch.sqrt(-2.0 * torch.log(u[0::2]))
+    th = (2.0 * torch.pi) * u[1::2]
+    out = torch.empty(2 * m, dtype=torch.float64, device=device)
+    out[0::2] = r * torch.cos(th)
+    out[1::2] = r * torch.sin(th)
+    out = (mean + std * out[:n]).to(torch.float32)
+    return out.to(torch.bfloat16).reshape(tuple(int(s) for s in shape))
