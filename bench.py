@@ -151,17 +151,19 @@ def gemm_bytes(M, N, K, epi):
 
 
 def time_graph(g, reps, stream):
+    """ms per replay; replays and events on `stream`."""
     import torch
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(2):
-        g.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(reps):
-        g.replay()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps  # ms per replay
+    return e0.elapsed_time(e1) / reps
 
 
 def capture(fn, stream):

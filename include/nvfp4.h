@@ -114,6 +114,15 @@ size_t nvfp4_gemm_workspace_bytes(int M, int N, int K);
  * NVFP4_OK, or NVFP4_ERR_TIMEOUT if a kernel's bounded wait expired since the last read. */
 nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
 
+/* Diagnostics (tracing): while `buf` (device, `words` 64-bit words) is set, each
+ * nvfp4_gemm launch takes the next free slice of it (8 words per CTA, CTA index
+ * (split * m_tiles + m_tile) * n_tiles + n_tile) and writes: globaltimer ns at entry, SM
+ * id, then globaltimer ns at set-up done, first operand stage landed, last MMA issued,
+ * accumulator ready, epilogue done.  Launches that no longer fit are not traced.  Setting
+ * a buffer (or NULL, which turns tracing off) rewinds the cursor.  Host-side state, not
+ * thread safe; captured launches keep the slice they got at capture. */
+nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
+
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
 
 /* Per row of x [M, K] (leading dimension ldx, bf16 or fp32): the norm `kind`, then the

@@ -65,6 +65,10 @@ bool make_code_map(CUtensorMap *m, const void *ptr, int rows, int row_bytes, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+unsigned long long *g_trace = nullptr;  // diagnostics: per-CTA GEMM timestamps
+size_t g_trace_words = 0;
+size_t g_trace_cursor = 0;
+
 struct Schedule {
     int block_n;
     int splits;
@@ -186,6 +190,11 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
         p.tickets = static_cast<uint32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + (tiles * 4 + 255) / 256 * 256);
     }
+    const size_t ctas = static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
+    if (g_trace != nullptr && g_trace_cursor + 8 * ctas <= g_trace_words) {
+        p.trace = g_trace + g_trace_cursor;
+        g_trace_cursor += 8 * ctas;
+    }
     CUtensorMap ta, tb;
     if (!make_code_map(&ta, A->codes, M, K / 2, static_cast<int>(p.a_box_rows)) ||
         !make_code_map(&tb, W->codes, N, K / 2, sc.block_n))
@@ -292,6 +301,13 @@ size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int split
     if (block_n == 0 && splits == 0) return nvfp4_gemm_workspace_bytes(M, N, K);
     if (block_n <= 0 || N % block_n != 0) return 0;
     return workspace_for(M, N, finish(block_n, splits, K));
+}
+
+nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
+    g_trace = buf;
+    g_trace_words = buf ? words : 0;
+    g_trace_cursor = 0;
+    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream) {

@@ -24,6 +24,7 @@
 // unwinds: copies and MMAs in flight are drained, tensor memory is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cstdlib>
 #include <cuda_runtime.h>
 
 #include "gemm.h"
@@ -79,6 +80,12 @@ __device__ __forceinline__ float gelu_tanh_f(float z) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t smid_u() {
+    uint32_t s;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
+    return s;
 }
 
 // bounded wait that ignores the abort flag (used while draining before teardown)
@@ -173,9 +180,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // misc[3] = accumulator-valid decision of the epilogue warps
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
+    const unsigned long long t_entry = globaltimer_ns();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
+    // diagnostics: [0] globaltimer at entry, [1] smid, [2..6] globaltimer at set-up done /
+    // first stage landed / last MMA issued / accumulator ready / epilogue done
+    unsigned long long *trace = nullptr;
+    if (p.trace != nullptr)
+        trace = p.trace + 8ull * ((static_cast<unsigned long long>(blockIdx.z) * gridDim.y + blockIdx.y) *
+                                  gridDim.x + blockIdx.x);
     const int n0 = n_tile * BN, m0 = m_tile * 128;
     const int kt_begin = split * p.kt_per_split;
     const int kt_end = min(p.k_tiles, kt_begin + p.kt_per_split);
@@ -201,6 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    if (trace != nullptr && threadIdx.x == 0) {
+        trace[0] = t_entry;
+        trace[1] = smid_u();
+        trace[2] = globaltimer_ns();
+    }
     // Let the next kernel in the stream start its own weight prefetch.
     pdl_launch_dependents();
 
@@ -267,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = j % STAGES, kt = kt_begin + j;
                 if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull)) break;
                 tc_fence_after();
+                if (trace != nullptr && j == 0) trace[3] = globaltimer_ns();
                 const int nkb = nkb_of(kt);
                 const uint32_t a_s = sbase + S::kOffA + s * kABytes;
                 const uint32_t b_s = sbase + S::kOffB + s * C::kBBytes;
@@ -286,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs finished reading it
             }
+            if (trace != nullptr) trace[4] = globaltimer_ns();
             tc_commit(bar_acc);  // always: completion of every MMA issued above
         }
     } else {
@@ -301,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (threadIdx.x == 64) misc[3] = (done && !*abort_flag) ? 1u : 0u;
         named_barrier_epi();
         const bool acc_ok = misc[3] != 0u;
+        if (trace != nullptr && threadIdx.x == 64) trace[5] = globaltimer_ns();
         tc_fence_after();
         pdl_wait();
         if (acc_ok) {
@@ -367,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if (trace != nullptr && threadIdx.x == 0) trace[6] = globaltimer_ns();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
@@ -392,11 +415,20 @@ cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmAr
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, STAGES>, ta, tb, p);
 }
 
 }  // namespace
+
+bool pdl_enabled() {
+    static int on = -1;
+    if (on < 0) {
+        const char *e = getenv("NVFP4_PDL");
+        on = (e != nullptr && e[0] == '0') ? 0 : 1;
+    }
+    return on == 1;
+}
 
 cudaError_t probe_gemm_kernels() {
     cudaFuncAttributes fa;

@@ -33,10 +33,14 @@ struct GemmArgs {
     float g_out;
     float *partials;    // split-K: [splits, M, N] fp32
     uint32_t *tickets;  // split-K: one word per output tile
+    unsigned long long *trace;  // optional per-CTA timestamps (diagnostics), 8 words per CTA
 };
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s);
+
+// Programmatic dependent launch for this library's kernels: on unless NVFP4_PDL=0.
+bool pdl_enabled();
 
 // Reads the device status word and clears it (after synchronising `s`).
 cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out);

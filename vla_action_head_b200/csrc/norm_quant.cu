@@ -20,6 +20,7 @@
 // §Implemented Path: AdaRMSNorm + NVFP4/SFA in one launch.)
 #include <cuda_runtime.h>
 
+#include "gemm.h"
 #include "norm.h"
 #include "quant.cuh"
 #include "sm100.cuh"
@@ -241,7 +242,7 @@ static cudaError_t launch_tpr(const NormArgs &a, int bpt, cudaStream_t s) {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     switch (bpt) {
 #define NVFP4_CASE(B) \
     case B: return cudaLaunchKernelEx(&cfg, norm_quant_kernel<TPR, B, F32>, a);

@@ -15,7 +15,7 @@ from dataclasses import dataclass
 from typing import Optional
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+LIB_PATH = os.environ.get("NVFP4_LIB") or os.path.join(HERE, "libnvfp4.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 NORM = {"none": 0, "layernorm": 1, "rmsnorm": 2, "adaln": 3, "adarms": 4}
@@ -41,7 +41,8 @@ P, I, F, SZ = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
 
 def lib():
-    """Loads libnvfp4.so (built in-tree by vla_action_head_b200.build)."""
+    """Loads libnvfp4.so (built in-tree by vla_action_head_b200.build; NVFP4_LIB overrides
+    the path, e.g. to compare builds)."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
@@ -56,6 +57,7 @@ def lib():
             "nvfp4_gemm_workspace_bytes": (SZ, [I, I, I]),
             "nvfp4_gemm_workspace_bytes_ex": (SZ, [I, I, I, I, I]),
             "nvfp4_get_device_status": (I, [P]),
+            "nvfp4_set_gemm_trace": (I, [P, SZ]),
             "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
