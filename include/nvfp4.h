@@ -187,6 +187,26 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int
                         float out_global_scale, void *workspace, size_t ws_bytes,
                         nvfp4_stream_t stream);
 
+/* nvfp4_gemm for callers that cannot allocate device memory: no workspace argument.  The
+ * paper has no counterpart to this entry point.  It serves code that is not allowed to
+ * call cudaMalloc (or any allocator) once it is running -- for example a plugin inside a
+ * host runtime that owns every device allocation, or a real-time control loop that must
+ * not allocate after start-up.  The split-K workspace instead comes from a fixed 4 MiB
+ * buffer inside this library's own device memory, which every GPU that loads the library
+ * keeps until the process exits.  The call allocates nothing; it zeroes the buffer's
+ * ticket words with cudaMemsetAsync on `stream` before the GEMM.
+ *   - Shapes whose default schedule needs more than 4 MiB of workspace return
+ *     NVFP4_ERR_WORKSPACE (nvfp4_gemm_workspace_bytes tells the need in advance).
+ *   - The first call on each device looks the buffer's address up; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one buffer, which keeps the previous call's contents: calls that
+ *     may overlap on the GPU (other streams, other host threads) race on it; serialise them.
+ * Otherwise the contract and results are those of nvfp4_gemm. */
+nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
+                                nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
+                                void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,
+                                float out_global_scale, nvfp4_stream_t stream);
+
 /* Schedule-pinned variant of nvfp4_gemm for tuning sweeps and tests: block_n in
  * {64, 128, 256} output columns per CTA, splits >= 1 K partitions (each a whole number of
  * 256-element K tiles; 0 = let the library choose both).  Same contract otherwise; the

@@ -378,6 +378,28 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int
                      workspace, ws_bytes, 0, 0, stream);
 }
 
+nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
+                                nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
+                                void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,
+                                float out_global_scale, nvfp4_stream_t stream) {
+    size_t need = 0;
+    if (A != nullptr && W != nullptr && M > 0 && N > 0 && K > 0 && N % 64 == 0)
+        need = workspace_for(M, N, choose(M, N, K));
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    if (need > 0) {
+        const nvfp4_status st = check_device();
+        if (st != NVFP4_OK) return st;
+        if (noalloc_scratch(&ws, &ws_bytes) != cudaSuccess) return NVFP4_ERR_CUDA;
+        if (need > ws_bytes) return NVFP4_ERR_WORKSPACE;  // shape needs more than the fixed scratch
+        // the split-K tickets must start at zero; the previous call's contents are still there
+        const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / choose(M, N, K).block_n);
+        if (cudaMemsetAsync(ws, 0, (tiles * 4 + 255) / 256 * 256, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
+    return gemm_impl(A, W, M, N, K, epi, bias, residual, ldr, out_bf16, ldo, out_codes, out_sf, out_global_scale, ws,
+                     ws_bytes, 0, 0, stream);
+}
+
 nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,
                            const void *bias, const void *residual, int ldr, void *out_bf16, int ldo,
                            uint8_t *out_codes, uint8_t *out_sf, float out_global_scale, void *workspace,

@@ -36,6 +36,12 @@ namespace nvfp4 {
 
 __device__ uint32_t g_device_status = 0;
 
+// Split-K workspace of nvfp4_gemm_noalloc: lives in the library's own device memory, so
+// that entry point never allocates.  Every GPU that loads the library keeps these bytes
+// until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 constexpr int kThreads = 192;
@@ -420,6 +426,27 @@ cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmAr
 }
 
 }  // namespace
+
+// Device address of g_noalloc_scratch for the current device.  Host code only sees a
+// host-side stand-in under that name, so the address is looked up once per device (with
+// that device current) and cached; no allocation is involved.
+cudaError_t noalloc_scratch(void **ptr, size_t *bytes) {
+    constexpr int kMaxDevices = 64;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = kNoAllocScratchBytes;
+    return cudaSuccess;
+}
 
 bool pdl_enabled() {
     static int on = -1;

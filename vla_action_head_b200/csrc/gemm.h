@@ -39,6 +39,10 @@ struct GemmArgs {
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s);
 
+// Device address and size of the library-owned split-K workspace used by
+// nvfp4_gemm_noalloc (looked up once per device; allocation-free).
+cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
+
 // Programmatic dependent launch for this library's kernels: on unless NVFP4_PDL=0.
 bool pdl_enabled();
 

@@ -63,6 +63,8 @@ def lib():
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
             "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
                                F, P, SZ, P]),
+            "nvfp4_gemm_noalloc": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P,
+                                       P, F, P]),
             "nvfp4_gemm_ex": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P,
                                   P, F, P, SZ, I, I, P]),
         }
