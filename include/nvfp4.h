@@ -105,9 +105,12 @@ size_t nvfp4_sf_offset(int row, int kblk, int K);
 /* Zeroes a scale-factor buffer (cudaMemsetAsync); once per allocation is enough. */
 nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream);
 
-/* Workspace bytes nvfp4_gemm needs for this shape (split-K partials and tile tickets);
- * 0 if none.  The workspace must be zeroed once at allocation; every call leaves its
- * ticket words zero again (after NVFP4_ERR_TIMEOUT, zero it again). */
+/* Workspace bytes nvfp4_gemm needs for this shape; 0 if none.  The default schedule reduces
+ * split-K partials inside a thread-block cluster (distributed shared memory) and needs no
+ * workspace; schedules that reduce through global memory (more than 8 splits, or the ones
+ * selected by negative `splits` in nvfp4_gemm_ex) need tile tickets + fp32 partials.  A
+ * workspace must be zeroed once at allocation; every call leaves its ticket words zero
+ * again (after NVFP4_ERR_TIMEOUT, zero it again). */
 size_t nvfp4_gemm_workspace_bytes(int M, int N, int K);
 
 /* Reads and clears the library's device status word after synchronising `stream`:
@@ -195,8 +198,9 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int
  * buffer inside this library's own device memory, which every GPU that loads the library
  * keeps until the process exits.  The call allocates nothing; it zeroes the buffer's
  * ticket words with cudaMemsetAsync on `stream` before the GEMM.
- *   - Shapes whose default schedule needs more than 4 MiB of workspace return
- *     NVFP4_ERR_WORKSPACE (nvfp4_gemm_workspace_bytes tells the need in advance).
+ *   - It runs the workspace-reduced schedule (nvfp4_gemm_ex with block_n = 0, splits = -1).
+ *     Shapes for which that needs more than 4 MiB return NVFP4_ERR_WORKSPACE;
+ *     nvfp4_gemm_workspace_bytes_ex(M, N, K, 0, -1) tells the need in advance.
  *   - The first call on each device looks the buffer's address up; make that first call
  *     before any stream capture.
  *   - Every call shares the one buffer, which keeps the previous call's contents: calls that
@@ -208,9 +212,12 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
                                 float out_global_scale, nvfp4_stream_t stream);
 
 /* Schedule-pinned variant of nvfp4_gemm for tuning sweeps and tests: block_n in
- * {64, 128, 256} output columns per CTA, splits >= 1 K partitions (each a whole number of
- * 256-element K tiles; 0 = let the library choose both).  Same contract otherwise; the
- * workspace must hold nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits) bytes. */
+ * {64, 128, 256} output columns per CTA and |splits| K partitions (each a whole number of
+ * 256-element K tiles).  splits > 0 reduces the partials inside a cluster when splits <= 8
+ * and M <= 128, otherwise through the workspace; splits < 0 always uses the workspace.
+ * block_n = 0 with splits = 0 takes the default schedule, with splits = -1 the default
+ * workspace-reduced schedule.  Same contract otherwise; the workspace must hold
+ * nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits) bytes. */
 nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
                            nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
                            void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,

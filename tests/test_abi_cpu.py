@@ -37,8 +37,10 @@ def test_sf_layout_matches_oracle(L, orc):
 
 def test_workspace_sizes(L):
     assert L.nvfp4_gemm_workspace_bytes_ex(968, 2560, 2048, 256, 1) == 0
-    ws = L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 128, 4)
+    assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 128, 4) == 0  # reduced in a cluster
+    ws = L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 128, -4)  # reduced through the workspace
     assert ws >= 4 * 41 * 1536 * 4
+    assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 0, -1) > 0
     assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 96, 1) == 0  # N % 96 != 0
 
 

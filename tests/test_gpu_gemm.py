@@ -56,14 +56,23 @@ def test_default_schedule_bias(orc, M, N, K):
 
 
 @pytest.mark.parametrize("bn", [64, 128, 256])
-@pytest.mark.parametrize("sp", [1, 2, 3])
+@pytest.mark.parametrize("sp", [1, 2, 3, -2, -3])
 def test_every_tile_and_split(orc, bn, sp):
+    """sp > 0: split-K reduced in a cluster over DSMEM; sp < 0: through the workspace."""
     _run(orc, 41, 512, 768, "bias_residual", bn=bn, sp=sp)
+    _run(orc, 64, 512, 768, "bias", bn=bn, sp=sp)
+    _run(orc, 100, 256, 1024, "none", bn=bn, sp=sp)
     _run(orc, 130, 256, 1024, "none", bn=bn, sp=sp)
 
 
+@pytest.mark.parametrize("sp", [4, 6, 8, -12])
+def test_deep_splits(orc, sp):
+    _run(orc, 41, 1536, 6144, "bias_residual", bn=64, sp=sp)
+    _run(orc, 50, 1024, 4096, "residual", bn=128, sp=sp)
+
+
 @pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
-@pytest.mark.parametrize("M,sp", [(41, 1), (41, 4), (200, 1)])
+@pytest.mark.parametrize("M,sp", [(41, 1), (41, 2), (41, -4), (200, 1)])
 def test_epilogues(orc, epi, M, sp):
     _run(orc, M, 512, 512, epi, bn=128, sp=sp)
 
@@ -91,11 +100,21 @@ def test_zero_activations_give_bias(orc):
     assert np.array_equal(host(out), np.broadcast_to(bias, (M, N)))
 
 
-def test_determinism_split_k(orc):
+@pytest.mark.parametrize("sp", [6, -6])
+def test_determinism_split_k(orc, sp):
     (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 13, 41, 1536, 6144)
     A, W = to_gpu_fp4(ac, asf, ga, 41, 6144), to_gpu_fp4(wc, wsf, gw, 1536, 6144)
-    o1 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=6))
-    o2 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=6))
+    o1 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=sp))
+    o2 = host(nvfp4.gemm(A, W, "none", block_n=128, splits=sp))
+    assert np.array_equal(o1, o2)
+
+
+def test_cluster_and_workspace_reductions_agree(orc):
+    """Both reductions add the partials in split order, so they agree bit for bit."""
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 14, 41, 1536, 6144)
+    A, W = to_gpu_fp4(ac, asf, ga, 41, 6144), to_gpu_fp4(wc, wsf, gw, 1536, 6144)
+    o1 = host(nvfp4.gemm(A, W, "none", block_n=64, splits=6))
+    o2 = host(nvfp4.gemm(A, W, "none", block_n=64, splits=-6))
     assert np.array_equal(o1, o2)
 
 

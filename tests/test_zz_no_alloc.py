@@ -38,10 +38,11 @@ def test_noalloc_matches_gemm_twice(M, N, K):
     import torch
     nvfp4.probe()
     L = nvfp4.lib()
-    need = L.nvfp4_gemm_workspace_bytes(M, N, K)
-    assert need > 0  # these shapes run split-K, so the fixed scratch is exercised
+    # these shapes run split-K through the workspace, so the fixed scratch is exercised
+    assert L.nvfp4_gemm_workspace_bytes_ex(M, N, K, 0, -1) > 0
     a, w, bias, res = _operands(M, N, K, 41)
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    need = L.nvfp4_gemm_workspace_bytes(M, N, K)
+    ws = torch.zeros(max(need, 16), dtype=torch.uint8, device="cuda")
     ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     st = _call(L.nvfp4_gemm, a, w, M, N, K, "bias_residual", bias, res, ref,
                [C.c_void_p(ws.data_ptr()), C.c_size_t(need)])
@@ -61,7 +62,7 @@ def test_noalloc_rejects_oversized_workspace():
     nvfp4.probe()
     L = nvfp4.lib()
     M, N, K = 128, 1024, 16384
-    need = L.nvfp4_gemm_workspace_bytes(M, N, K)
+    need = L.nvfp4_gemm_workspace_bytes_ex(M, N, K, 0, -1)
     assert need > (4 << 20)
     a, w, bias, res = _operands(M, N, K, 42)
     out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")

@@ -73,7 +73,10 @@ struct Schedule {
     int block_n;
     int splits;
     int kt_per_split;
+    bool cluster;  // split-K partials reduced over DSMEM inside a cluster (no workspace)
 };
+
+constexpr int kMaxClusterSplits = 8;  // portable cluster size
 
 int sm_count_cached() {
     static int sms = 0;
@@ -85,18 +88,52 @@ int sm_count_cached() {
     return sms;
 }
 
-// Normalises a (block_n, splits) request so that every split owns >= 1 K tile.
-Schedule finish(int block_n, int splits, int K) {
+// Normalises a (block_n, splits) request so that every split owns >= 1 K tile.  Split
+// counts up to the portable cluster size reduce inside a cluster (`use_cluster`), larger
+// ones through the caller's workspace.
+Schedule finish(int block_n, int splits, int K, bool use_cluster = true) {
     const int k_tiles = (K + 255) / 256;
     if (splits < 1) splits = 1;
     if (splits > k_tiles) splits = k_tiles;
     const int per = (k_tiles + splits - 1) / splits;
-    return Schedule{block_n, (k_tiles + per - 1) / per, per};
+    const int eff = (k_tiles + per - 1) / per;
+    return Schedule{block_n, eff, per, use_cluster && eff > 1 && eff <= kMaxClusterSplits};
 }
 
-// Default schedule.  Small M streams the weights: enough (tile, split) CTAs to put every SM
-// on the weight stream.  Large M is compute-bound: widest tile, no split.
+// Default schedule.  Small M streams the weights: pick the tile width and split factor
+// (<= 8, reduced in a cluster) that put about one CTA on every SM, preferring wider tiles
+// and fewer splits.  Large M is compute-bound: widest tile, no split.
 Schedule choose(int M, int N, int K) {
+    const int sms = sm_count_cached();
+    const int k_tiles = (K + 255) / 256;
+    const int m_tiles = (M + 127) / 128;
+    if (M <= 128) {
+        Schedule best{64, 1, k_tiles, false};
+        double best_cost = 1e30;
+        for (int bn : {128, 64}) {
+            if (N % bn != 0) continue;
+            const int n_tiles = N / bn * m_tiles;
+            for (int s = 1; s <= kMaxClusterSplits && s <= k_tiles; ++s) {
+                const Schedule c = finish(bn, s, K);
+                const int ctas = n_tiles * c.splits;
+                if (ctas > 2 * sms) continue;
+                const double cost = std::fabs(static_cast<double>(ctas - sms)) / sms + 0.03 * c.splits +
+                                    (bn == 64 ? 0.05 : 0.0);
+                if (cost < best_cost) {
+                    best_cost = cost;
+                    best = c;
+                }
+            }
+        }
+        return best;
+    }
+    const int bn = (N % 256 == 0) ? 256 : (N % 128 == 0) ? 128 : 64;
+    return finish(bn, 1, K);
+}
+
+// The workspace-reduced schedule (used by nvfp4_gemm_noalloc): enough (tile, split) CTAs
+// to put every SM on the weight stream, partials through global memory.
+Schedule choose_workspace(int M, int N, int K) {
     const int sms = sm_count_cached();
     const int k_tiles = (K + 255) / 256;
     if (M <= 128) {
@@ -104,14 +141,13 @@ Schedule choose(int M, int N, int K) {
         const int n_tiles = N / bn;
         int splits = (sms + n_tiles / 2) / n_tiles;
         if (splits > k_tiles) splits = k_tiles;
-        return finish(bn, splits, K);
+        return finish(bn, splits, K, false);
     }
-    const int bn = (N % 256 == 0) ? 256 : (N % 128 == 0) ? 128 : 64;
-    return finish(bn, 1, K);
+    return choose(M, N, K);
 }
 
 size_t workspace_for(int M, int N, const Schedule &s) {
-    if (s.splits <= 1) return 0;
+    if (s.splits <= 1 || s.cluster) return 0;
     const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / s.block_n);
     const size_t tickets = (tiles * 4 + 255) / 256 * 256;
     return tickets + static_cast<size_t>(s.splits) * M * N * sizeof(float);
@@ -152,10 +188,14 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     Schedule sc;
     if (block_n == 0 && splits == 0) {
         sc = choose(M, N, K);
+    } else if (block_n == 0 && splits == -1) {
+        sc = choose_workspace(M, N, K);
     } else {
         if (block_n != 64 && block_n != 128 && block_n != 256) return NVFP4_ERR_INVALID_ARG;
-        if (N % block_n != 0 || splits < 1) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-        sc = finish(block_n, splits, K);
+        if (N % block_n != 0 || splits == 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        // splits < 0: reduce -splits partials through the workspace instead of a cluster
+        sc = finish(block_n, splits < 0 ? -splits : splits, K, splits > 0);
+        if (sc.cluster && M > 128) sc = finish(block_n, sc.splits, K, false);
     }
     const size_t need = workspace_for(M, N, sc);
     if (need > 0) {
@@ -171,6 +211,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     p.k_tiles = (K + 255) / 256;
     p.kt_per_split = sc.kt_per_split;
     p.splits = sc.splits;
+    p.cluster = sc.cluster ? 1 : 0;
     p.n_tiles = N / sc.block_n;
     p.a_box_rows = static_cast<uint32_t>(M >= 128 ? 128 : (M + 7) / 8 * 8);
     p.sfa = A->sf;
@@ -299,8 +340,11 @@ size_t nvfp4_gemm_workspace_bytes(int M, int N, int K) {
 size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int splits) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
     if (block_n == 0 && splits == 0) return nvfp4_gemm_workspace_bytes(M, N, K);
-    if (block_n <= 0 || N % block_n != 0) return 0;
-    return workspace_for(M, N, finish(block_n, splits, K));
+    if (block_n == 0 && splits == -1) return N % 64 ? 0 : workspace_for(M, N, choose_workspace(M, N, K));
+    if (block_n <= 0 || N % block_n != 0 || splits == 0) return 0;
+    Schedule sc = finish(block_n, splits < 0 ? -splits : splits, K, splits > 0);
+    if (sc.cluster && M > 128) sc = finish(block_n, sc.splits, K, false);
+    return workspace_for(M, N, sc);
 }
 
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
@@ -384,7 +428,7 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
                                 float out_global_scale, nvfp4_stream_t stream) {
     size_t need = 0;
     if (A != nullptr && W != nullptr && M > 0 && N > 0 && K > 0 && N % 64 == 0)
-        need = workspace_for(M, N, choose(M, N, K));
+        need = workspace_for(M, N, choose_workspace(M, N, K));
     void *ws = nullptr;
     size_t ws_bytes = 0;
     if (need > 0) {
@@ -393,11 +437,11 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
         if (noalloc_scratch(&ws, &ws_bytes) != cudaSuccess) return NVFP4_ERR_CUDA;
         if (need > ws_bytes) return NVFP4_ERR_WORKSPACE;  // shape needs more than the fixed scratch
         // the split-K tickets must start at zero; the previous call's contents are still there
-        const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / choose(M, N, K).block_n);
+        const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / choose_workspace(M, N, K).block_n);
         if (cudaMemsetAsync(ws, 0, (tiles * 4 + 255) / 256 * 256, stream) != cudaSuccess) return NVFP4_ERR_CUDA;
     }
     return gemm_impl(A, W, M, N, K, epi, bias, residual, ldr, out_bf16, ldo, out_codes, out_sf, out_global_scale, ws,
-                     ws_bytes, 0, 0, stream);
+                     ws_bytes, 0, -1, stream);
 }
 
 nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,

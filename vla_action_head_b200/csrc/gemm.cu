@@ -45,7 +45,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kABytes = 128 * 128;  // one A stage: 128 rows x 128 bytes (256 FP4 values)
 constexpr int kSfAtom = 512;        // 128 rows x 4 scale blocks
 
 template <int BN>
@@ -62,16 +61,48 @@ struct Cfg {
                                      : kColsUsed <= 256 ? 256 : 512;
 };
 
-template <int BN, int STAGES>
+// Shared-memory plan: STAGES x [A tile] then STAGES x [W tile], then the scale atoms.
+// SMALL_A (M <= 64): an A stage holds 64 rows (8 KB).  The M = 128 MMA still reads a 16 KB
+// window from the stage base; its rows 64..127 fall on the next buffer (finite E2M1 bytes),
+// and their scales are the zero padding of the 128-row scale atom, so they add nothing.
+template <int BN, int STAGES, bool SMALL_A>
 struct Smem {
+    static constexpr int kA = SMALL_A ? 8192 : 16384;
     static constexpr int kOffA = 0;
-    static constexpr int kOffB = kOffA + STAGES * kABytes;
+    static constexpr int kOffB = kOffA + STAGES * kA;
     static constexpr int kOffSfa = kOffB + STAGES * Cfg<BN>::kBBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * Cfg<BN>::kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes;
     static constexpr int kOffMisc = kOffBar + (2 * STAGES + 1) * 8;
     static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    // split-K partial tile for the cluster reduction, reusing the stage buffers
+    static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
+    static_assert((SMALL_A ? 64 : 128) * kRedLd * 4 <= kOffBar, "reduction tile must fit the stages");
+    static_assert(Cfg<BN>::kBBytes >= 8192, "SMALL_A window overlaps the W tile");
 };
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA in the cluster; release/acquire orders shared-memory writes.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
 
 __device__ __forceinline__ void named_barrier_epi() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -169,12 +200,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs &p, int m, int n, 
     }
 }
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+// SMALL_A kernels are sized (shared memory, TMEM, registers) for two resident CTAs per SM.
+template <int BN, int STAGES, bool SMALL_A>
+__global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs p) {
     using C = Cfg<BN>;
-    using S = Smem<BN, STAGES>;
+    using S = Smem<BN, STAGES, SMALL_A>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -256,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = j % STAGES, kt = kt_begin + j;
                 const uint32_t full = bar_full + 8 * s;
                 const uint32_t nb = static_cast<uint32_t>(nkb_of(kt)) * kSfAtom;
-                tma_load_2d(sbase + S::kOffA + s * kABytes, &tmA, kt * 128, m0, full, pol_a);
+                tma_load_2d(sbase + S::kOffA + s * S::kA, &tmA, kt * 128, m0, full, pol_a);
                 bulk_load(sbase + S::kOffSfa + s * C::kSfaBytes,
                           p.sfa + (static_cast<size_t>(m_tile) * p.k_atoms + 4 * kt) * kSfAtom, nb, full, pol_a);
             };
@@ -294,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 if (trace != nullptr && j == 0) trace[3] = globaltimer_ns();
                 const int nkb = nkb_of(kt);
-                const uint32_t a_s = sbase + S::kOffA + s * kABytes;
+                const uint32_t a_s = sbase + S::kOffA + s * S::kA;
                 const uint32_t b_s = sbase + S::kOffB + s * C::kBBytes;
                 const uint32_t sfa_s = sbase + S::kOffSfa + s * C::kSfaBytes;
                 const uint32_t sfb_s = sbase + S::kOffSfb + s * C::kSfbBytes;
@@ -345,6 +377,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                         epilogue_chunk(p, m, n0 + c0, v);
                     }
                 }
+            } else if (p.cluster) {
+                // split-K across the cluster: this CTA's partial tile into its own shared
+                // memory (the stage buffers are free: every load landed and every MMA read it)
+                float *red = reinterpret_cast<float *>(smem);
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c0, r);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        float4 *dst = reinterpret_cast<float4 *>(red + row * S::kRedLd + c0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                    }
+                }
             } else {
                 // split-K: partial tile to the workspace, then an arrival ticket
                 float *part = p.partials + (static_cast<size_t>(split) * p.M) * p.N;
@@ -393,6 +441,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    if (p.cluster) {
+        // Deterministic split-K reduction over distributed shared memory: CTA `rank` of the
+        // cluster owns local rows rank, rank + S, ...; for each (row, 32 columns) it adds the S
+        // partials in split order 0..S-1 and runs the epilogue.
+        __syncwarp();
+        cluster_sync_all();  // partial tiles written and visible cluster-wide
+        if (warp >= 2 && misc[3] != 0u) {
+            const int S_ = p.splits;
+            const int rank = static_cast<int>(cluster_ctarank());
+            const int rows_valid = min(SMALL_A ? 64 : 128, p.M - m0);
+            constexpr int kChunks = BN / 32;
+            const float *red = reinterpret_cast<const float *>(smem);
+            for (int item = threadIdx.x - 64;; item += 128) {
+                const int i = rank + (item / kChunks) * S_;
+                const int ch = item % kChunks;
+                if (i >= rows_valid) break;
+                const uint32_t local = smem_u32(red + i * S::kRedLd + ch * 32);
+                float v[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) v[t] = 0.0f;
+                for (int sp = 0; sp < S_; ++sp) {
+                    const uint32_t src = mapa_shared(local, static_cast<uint32_t>(sp));
+                    float4 u[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) u[j] = ld_dsmem_f4(src + 16 * j);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        v[4 * j] = __fadd_rn(v[4 * j], u[j].x);
+                        v[4 * j + 1] = __fadd_rn(v[4 * j + 1], u[j].y);
+                        v[4 * j + 2] = __fadd_rn(v[4 * j + 2], u[j].z);
+                        v[4 * j + 3] = __fadd_rn(v[4 * j + 3], u[j].w);
+                    }
+                }
+                epilogue_chunk(p, m0 + i, n0 + ch * 32, v);
+            }
+        }
+        cluster_sync_all();  // nobody leaves while a peer still reads its partials
+    }
+
     tc_fence_before();
     __syncthreads();
     if (trace != nullptr && threadIdx.x == 0) trace[6] = globaltimer_ns();
@@ -402,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SMALL_A>
 cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
-    using S = Smem<BN, STAGES>;
-    static bool attr_set = false;  // per device is enough in practice; set idempotently
+    using S = Smem<BN, STAGES, SMALL_A>;
+    static bool attr_set = false;  // per process; the attribute is idempotent
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             S::kBytes);
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, STAGES, SMALL_A>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -417,12 +504,23 @@ cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmAr
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = S::kBytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (p.cluster) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = 1;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = static_cast<unsigned>(p.splits);
+        ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, STAGES>, ta, tb, p);
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, STAGES, SMALL_A>, ta, tb, p);
 }
 
 }  // namespace
@@ -459,7 +557,7 @@ bool pdl_enabled() {
 
 cudaError_t probe_gemm_kernels() {
     cudaFuncAttributes fa;
-    return cudaFuncGetAttributes(&fa, gemm_kernel<128, 5>);
+    return cudaFuncGetAttributes(&fa, gemm_kernel<128, 5, false>);
 }
 
 cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out) {
@@ -473,10 +571,13 @@ cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out) {
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s) {
+    const bool small = p.a_box_rows <= 64;
+    // M <= 64: ~100 KB of shared memory and <= 256 TMEM columns, so two CTAs share an SM and
+    // the next GEMM prefetches its weights while this one finishes.  Larger M: deep pipelines.
     switch (block_n) {
-    case 64: return launch_bn<64, 6>(ta, tb, p, s);
-    case 128: return launch_bn<128, 5>(ta, tb, p, s);
-    case 256: return launch_bn<256, 3>(ta, tb, p, s);
+    case 64: return small ? launch_bn<64, 5, true>(ta, tb, p, s) : launch_bn<64, 6, false>(ta, tb, p, s);
+    case 128: return small ? launch_bn<128, 3, true>(ta, tb, p, s) : launch_bn<128, 5, false>(ta, tb, p, s);
+    case 256: return small ? launch_bn<256, 2, true>(ta, tb, p, s) : launch_bn<256, 3, false>(ta, tb, p, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -17,6 +17,7 @@ struct GemmArgs {
     int k_tiles;       // ceil(K / 256): pipeline K tiles
     int kt_per_split;  // K tiles per split
     int splits;
+    int cluster;       // 1: the splits of a tile form a cluster and reduce over DSMEM
     int n_tiles;
     uint32_t a_box_rows;  // rows per A TMA box (min(128, M rounded up to 8))
     const uint8_t *sfa;

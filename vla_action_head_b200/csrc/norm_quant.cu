@@ -78,9 +78,10 @@ __global__ void __launch_bounds__(128) norm_quant_kernel(const NormArgs p) {
     const int nblk = p.K >> 4;
     const int k_atoms = (p.K + 63) >> 6;
 
-    // The input may be the previous kernel's output: wait for it (programmatic launch).
-    pdl_wait();
+    // Let the next kernel launch now (it prefetches its weights), then wait for our input,
+    // which may be the previous kernel's output (programmatic dependent launch).
     pdl_launch_dependents();
+    pdl_wait();
 
     const bool row_ok = row < p.M;
     int src_row = row;
