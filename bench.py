@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=24)
     ap.add_argument("--no-side", action="store_true", help="skip the side measurements")
+    ap.add_argument("--soak-steps", type=int, default=200,
+                    help="untimed steps while the clock sampler starts (0 for profiling runs)")
     ap.add_argument("--profile-case", default=None,
                     help="run one small case for ncu (dit-gemms | prefill-gemms | norm) and exit")
     return ap.parse_args()
@@ -335,7 +337,7 @@ def main():
     clk = Clocks(local)
     time.sleep(0.3)
     with torch.cuda.stream(stream):
-        run_steps(max(1, 200 // max(1, L // 24)))  # ~soak so the sampler sees the load
+        run_steps(args.soak_steps)  # so the clock sampler sees the load
     torch.cuda.synchronize()
     barrier(ws_n)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -390,7 +392,7 @@ def main():
             line.update(side_measurements(stack, wsp, stream, dev, pk, pk_kind))
         except Exception as e:  # a side measurement never hides the main line
             line["side_error"] = repr(e)[:300]
-    if rank == 0 and ws_n == 1:
+    if rank == 0 and ws_n == 1 and not args.no_side:
         try:
             us_cpu = cpu_baseline_dit(1)
             line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
