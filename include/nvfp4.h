@@ -226,6 +226,69 @@ nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, 
 
 size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int splits);
 
+/* ---- layer executor: a whole program of ops in one launch --------------------------- */
+
+/* At M <= 64 tokens a transformer layer's linear path is a chain of small dependent steps.
+ * Launched as separate kernels, each step pays a launch and a grid completion of several
+ * microseconds.  A program runs the chain in ONE persistent cooperative launch:
+ *   - every CTA walks the ops in order;
+ *   - an op starts consuming its input once the previous op's completion counter is full;
+ *   - the weight tiles of later ops stream into shared memory while earlier ops run,
+ *     since weights never depend on activations.
+ * Results are those of the standalone calls.  The norm op is nvfp4_quantize_norm; the GEMM
+ * op is nvfp4_gemm with the same epilogues, its split-K partials added in split order
+ * over distributed shared memory.  ([GROOT] §Summary and §What is in the tier: the DiT
+ * action head at M = 41 is weight-bandwidth bound and runs as one captured graph; [PI05]
+ * §Implemented Path: the whole path is CUDA-graph capturable.) */
+typedef enum { NVFP4_OP_QUANTIZE_NORM = 0, NVFP4_OP_GEMM = 1 } nvfp4_op_type;
+
+typedef struct {
+    nvfp4_op_type type;
+    int M, N, K;
+    /* NVFP4_OP_QUANTIZE_NORM: bf16 x [M, K] (ldx) -> out_codes / out_sf (pre-zeroed) */
+    const void *x;
+    int ldx;
+    nvfp4_norm norm;
+    const void *gamma, *beta, *mod_scale, *mod_shift;
+    float eps;
+    /* NVFP4_OP_GEMM: A (M x K) times W (N x K)^T, epilogue as nvfp4_gemm */
+    nvfp4_tensor A, W;
+    nvfp4_epilogue epi;
+    const void *bias, *residual;
+    int ldr;
+    void *out_bf16;
+    int ldo;
+    /* FP4 output: of the norm op, or of a BIAS_GELU / GEGLU epilogue */
+    uint8_t *out_codes, *out_sf;
+    float out_global_scale;
+} nvfp4_op;
+
+/* Host-side handle of a built program; the device data lives in `buffer`. */
+typedef struct {
+    void *buffer;
+    size_t bytes;
+    int n_ops;
+    int grid;
+    int cluster;
+    size_t ops_offset, maps_offset, done_offset;
+} nvfp4_program;
+
+/* Device bytes a program of n_ops ops needs. */
+size_t nvfp4_program_bytes(int n_ops);
+
+/* Validates the ops (the rules of the standalone calls, plus: GEMM M <= 64, N % 64 == 0,
+ * K % 32 == 0; norm K <= 4096, bf16 input), chooses each GEMM's schedule, encodes the TMA
+ * descriptors and copies the program into `buffer` (device, >= nvfp4_program_bytes(n_ops),
+ * 256-byte aligned).  Synchronous (set-up time); the buffers the ops name must stay valid
+ * for every later run. */
+nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes,
+                                 nvfp4_program *prog);
+
+/* Runs the program on `stream`: zeroes its completion counters (cudaMemsetAsync) and makes
+ * one cooperative launch.  Allocates nothing; capturable in a CUDA graph.  Runs of the same
+ * program must not overlap. */
+nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

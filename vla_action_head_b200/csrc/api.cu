@@ -7,9 +7,13 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <vector>
 
 #include "../../include/nvfp4.h"
+#include "exec.h"
 #include "gemm.h"
 #include "norm.h"
 
@@ -151,6 +155,38 @@ size_t workspace_for(int M, int N, const Schedule &s) {
     const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / s.block_n);
     const size_t tickets = (tiles * 4 + 255) / 256 * 256;
     return tickets + static_cast<size_t>(s.splits) * M * N * sizeof(float);
+}
+
+// Argument checks shared by nvfp4_gemm* and the GEMM op of a program (no device access).
+nvfp4_status validate_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,
+                           const void *bias, const void *residual, int ldr, void *out_bf16, int ldo,
+                           uint8_t *out_codes, uint8_t *out_sf, float out_global_scale) {
+    if (A == nullptr || W == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if (A->rows != M || W->rows != N || A->K != K || W->K != K) return NVFP4_ERR_INVALID_ARG;
+    if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 5) return NVFP4_ERR_INVALID_ARG;
+    if (K % 32 != 0 || N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!scale_ok(A->global_scale) || !scale_ok(W->global_scale)) return NVFP4_ERR_INVALID_ARG;
+    if (M == 0) return NVFP4_OK;
+    const bool fp4_out = (epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
+    const bool need_bias = (epi == NVFP4_EPI_BIAS || epi == NVFP4_EPI_BIAS_RESIDUAL || epi == NVFP4_EPI_BIAS_GELU);
+    const bool need_res = (epi == NVFP4_EPI_RESIDUAL || epi == NVFP4_EPI_BIAS_RESIDUAL);
+    if (need_bias && bias == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (need_res && (residual == nullptr || ldr < N)) return NVFP4_ERR_INVALID_ARG;
+    if (need_res && ldr % 8 != 0) return NVFP4_ERR_MISALIGNED;
+    if (fp4_out) {
+        if (out_codes == nullptr || out_sf == nullptr || !scale_ok(out_global_scale)) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(out_codes) || !aligned16(out_sf)) return NVFP4_ERR_MISALIGNED;
+    } else {
+        if (out_bf16 == nullptr || ldo < N) return NVFP4_ERR_INVALID_ARG;
+        if (ldo % 8 != 0 || !aligned16(out_bf16)) return NVFP4_ERR_MISALIGNED;
+    }
+    if (A->codes == nullptr || A->sf == nullptr || W->codes == nullptr || W->sf == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(A->codes) || !aligned16(A->sf) || !aligned16(W->codes) || !aligned16(W->sf))
+        return NVFP4_ERR_MISALIGNED;
+    if ((bias && !aligned16(bias)) || (need_res && !aligned16(residual))) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
 }
 
 nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,
@@ -450,6 +486,157 @@ nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, 
                            size_t ws_bytes, int block_n, int splits, nvfp4_stream_t stream) {
     return gemm_impl(A, W, M, N, K, epi, bias, residual, ldr, out_bf16, ldo, out_codes, out_sf, out_global_scale,
                      workspace, ws_bytes, block_n, splits, stream);
+}
+
+// ---- layer executor ---------------------------------------------------------------------
+static constexpr int kExecCluster = 4;
+static constexpr int kExecRing = 6;
+
+size_t nvfp4_program_bytes(int n_ops) {
+    if (n_ops <= 0) return 0;
+    const size_t maps = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
+    const size_t ops = (static_cast<size_t>(n_ops) * sizeof(ExecOp) + 255) / 256 * 256;
+    const size_t done = (static_cast<size_t>(n_ops) * 4 + 255) / 256 * 256;
+    return maps + ops + done;
+}
+
+nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes, nvfp4_program *prog) {
+    if (ops == nullptr || n_ops <= 0 || buffer == nullptr || prog == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (bytes < nvfp4_program_bytes(n_ops)) return NVFP4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    int grid = 0;
+    if (exec_grid(kExecCluster, &grid) != cudaSuccess || grid < kExecCluster) return NVFP4_ERR_CUDA;
+    const int teams = grid / kExecCluster;
+
+    std::vector<CUtensorMap> maps(static_cast<size_t>(n_ops) * 2);
+    std::vector<ExecOp> eops(static_cast<size_t>(n_ops));
+    for (int i = 0; i < n_ops; ++i) {
+        const nvfp4_op &o = ops[i];
+        ExecOp &e = eops[i];
+        std::memset(&e, 0, sizeof e);
+        if (o.type == NVFP4_OP_QUANTIZE_NORM) {
+            if (o.M <= 0 || o.K <= 0 || o.x == nullptr || o.ldx < o.K) return NVFP4_ERR_INVALID_ARG;
+            if (static_cast<int>(o.norm) < 0 || static_cast<int>(o.norm) > 4) return NVFP4_ERR_INVALID_ARG;
+            if (o.K % 16 != 0 || o.K > 4096) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+            if (o.out_codes == nullptr || o.out_sf == nullptr || !scale_ok(o.out_global_scale))
+                return NVFP4_ERR_INVALID_ARG;
+            if (!(o.eps >= 0.0f) || !std::isfinite(o.eps)) return NVFP4_ERR_INVALID_ARG;
+            if (!aligned16(o.x) || o.ldx % 8 != 0 || !aligned16(o.out_codes) || !aligned16(o.out_sf))
+                return NVFP4_ERR_MISALIGNED;
+            for (const void *pp : {o.gamma, o.beta, o.mod_scale, o.mod_shift})
+                if (pp != nullptr && !aligned16(pp)) return NVFP4_ERR_MISALIGNED;
+            e.type = kOpNorm;
+            e.units = static_cast<unsigned>(o.M);
+            e.norm.x = o.x;
+            e.norm.M = o.M;
+            e.norm.K = o.K;
+            e.norm.ldx = o.ldx;
+            e.norm.kind = static_cast<int>(o.norm);
+            e.norm.gamma = static_cast<const uint16_t *>(o.gamma);
+            e.norm.beta = static_cast<const uint16_t *>(o.beta);
+            e.norm.scale = static_cast<const uint16_t *>(o.mod_scale);
+            e.norm.shift = static_cast<const uint16_t *>(o.mod_shift);
+            e.norm.eps = o.eps;
+            e.norm.g = o.out_global_scale;
+            e.norm.codes = o.out_codes;
+            e.norm.sf = o.out_sf;
+            e.bpt = (o.K / 16 + 31) / 32;
+        } else if (o.type == NVFP4_OP_GEMM) {
+            st = validate_gemm(&o.A, &o.W, o.M, o.N, o.K, o.epi, o.bias, o.residual, o.ldr, o.out_bf16, o.ldo,
+                               o.out_codes, o.out_sf, o.out_global_scale);
+            if (st != NVFP4_OK) return st;
+            if (o.M <= 0 || o.M > 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+            const int k_tiles = (o.K + 255) / 256;
+            // schedule: tile width and split factor (dividing the cluster size) that finish the
+            // op in the fewest rounds with the shortest per-CTA K chain
+            double best = 1e30;
+            Schedule sc{64, 1, k_tiles, false};
+            for (int bn : {128, 64}) {
+                if (o.N % bn != 0) continue;
+                for (int s : {1, 2, 4}) {
+                    const Schedule c = finish(bn, s, o.K, false);
+                    if (kExecCluster % c.splits != 0) continue;
+                    const int n_tiles = o.N / bn;
+                    const int per_round = teams * (kExecCluster / c.splits);
+                    const int rounds = (n_tiles + per_round - 1) / per_round;
+                    const double cost = rounds * (1.0 + 0.08 * c.kt_per_split + (c.splits > 1 ? 0.5 : 0.0)) +
+                                        (c.kt_per_split > kExecRing ? 0.3 * (c.kt_per_split - kExecRing) : 0.0) +
+                                        (bn == 64 ? 0.02 : 0.0);
+                    if (cost < best) {
+                        best = cost;
+                        sc = c;
+                    }
+                }
+            }
+            e.type = kOpGemm;
+            e.M = o.M;
+            e.N = o.N;
+            e.K = o.K;
+            e.k_atoms = (o.K + 63) / 64;
+            e.k_tiles = k_tiles;
+            e.bn = sc.block_n;
+            e.splits = sc.splits;
+            e.kt_per_split = sc.kt_per_split;
+            e.n_tiles = o.N / sc.block_n;
+            e.units = static_cast<unsigned>(e.n_tiles);
+            e.a_box_rows = static_cast<uint32_t>((o.M + 7) / 8 * 8);
+            e.sfa = o.A.sf;
+            e.sfb = o.W.sf;
+            e.alpha = o.A.global_scale * o.W.global_scale;
+            e.epi = static_cast<int>(o.epi);
+            e.bias = static_cast<const uint16_t *>(o.bias);
+            e.residual = static_cast<const uint16_t *>(o.residual);
+            e.ldr = o.ldr;
+            e.out = static_cast<uint16_t *>(o.out_bf16);
+            e.ldo = o.ldo;
+            e.out_codes = o.out_codes;
+            e.out_sf = o.out_sf;
+            e.g_out = o.out_global_scale;
+            e.tm_a = 2 * i;
+            e.tm_b = 2 * i + 1;
+            if (getenv("NVFP4_EXEC_DEBUG") != nullptr)
+                fprintf(stderr, "nvfp4 program op %d: GEMM %dx%dx%d block_n %d splits %d k_tiles/split %d tiles %d (grid %d)\n",
+                        i, o.M, o.N, o.K, e.bn, e.splits, e.kt_per_split, e.n_tiles, grid);
+            if (!make_code_map(&maps[2 * i], o.A.codes, o.M, o.K / 2, static_cast<int>(e.a_box_rows)) ||
+                !make_code_map(&maps[2 * i + 1], o.W.codes, o.N, o.K / 2, e.bn))
+                return NVFP4_ERR_CUDA;
+        } else {
+            return NVFP4_ERR_INVALID_ARG;
+        }
+    }
+    const size_t maps_bytes = maps.size() * sizeof(CUtensorMap);
+    const size_t ops_bytes = (eops.size() * sizeof(ExecOp) + 255) / 256 * 256;
+    uint8_t *base = static_cast<uint8_t *>(buffer);
+    if (cudaMemcpy(base, maps.data(), maps_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(base + maps_bytes, eops.data(), eops.size() * sizeof(ExecOp), cudaMemcpyHostToDevice) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    prog->buffer = buffer;
+    prog->bytes = bytes;
+    prog->n_ops = n_ops;
+    prog->grid = grid;
+    prog->cluster = kExecCluster;
+    prog->maps_offset = 0;
+    prog->ops_offset = maps_bytes;
+    prog->done_offset = maps_bytes + ops_bytes;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream) {
+    if (prog == nullptr || prog->buffer == nullptr || prog->n_ops <= 0) return NVFP4_ERR_INVALID_ARG;
+    uint8_t *base = static_cast<uint8_t *>(prog->buffer);
+    ExecParams p;
+    p.ops = reinterpret_cast<const ExecOp *>(base + prog->ops_offset);
+    p.maps = reinterpret_cast<const CUtensorMap *>(base + prog->maps_offset);
+    p.done = reinterpret_cast<unsigned int *>(base + prog->done_offset);
+    p.n_ops = prog->n_ops;
+    p.cluster = prog->cluster;
+    if (device_status_address(&p.status) != cudaSuccess) return NVFP4_ERR_CUDA;
+    cudaError_t e = cudaMemsetAsync(p.done, 0, static_cast<size_t>(prog->n_ops) * 4, stream);
+    if (e == cudaSuccess) e = exec_launch(p, prog->grid, stream);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return from_cuda(e);
 }
 
 }  // extern "C"

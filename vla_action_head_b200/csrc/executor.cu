@@ -1,0 +1,510 @@
+// executor.cu — the layer executor: a whole program of norm -> NVFP4 and block-scaled GEMM
+// ops (e.g. a stack of DiT layers) in ONE persistent cooperative launch.
+//
+// At M <= 64 tokens a linear layer is a chain of small dependent steps (norm, QKV GEMM,
+// attention-output GEMM, norm, FFN up, FFN down).  As separate kernels each step pays a
+// launch and a grid completion; here every CTA walks the same program, ops are ordered by
+// per-op completion counters in global memory (release by the finishing CTAs, acquire by
+// the consumers), and the weight tiles of later ops stream into each CTA's shared-memory
+// ring while the current op waits for its input -- weights never depend on activations.
+//
+// Roles (224 threads):
+//   warp 0      weight producer: TMA loads of W code tiles + bulk loads of their scale
+//               atoms, for every GEMM unit of this CTA in program order, as far ahead as the
+//               ring allows.
+//   warp 1      MMA issuer: tcgen05.cp of the scales, tcgen05.mma kind::mxf4nvf4 block16
+//               into one of two TMEM accumulators.
+//   warp 2      activation producer: waits until the op's input is complete, then TMA loads
+//               the A code tiles + scale atoms into the same ring stages.
+//   warps 3..6  epilogue and norm workers: TMEM -> registers -> fused epilogue; split-K
+//               partials are added on the tile's owner CTA over distributed shared memory
+//               in split order (deterministic); norm ops run one row per warp.
+// GEMM work: the grid is a set of clusters of C CTAs; for an op split S ways (S | C), the
+// S CTAs that share a tile are cluster neighbours.
+// Every wait is bounded (2 s); an expired wait records a device status and unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+#include "exec.h"
+#include "gemm.h"
+#include "norm_row.cuh"
+#include "quant.cuh"
+#include "sm100.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kThreads = 224;
+constexpr int kRing = 6;
+constexpr int kStageA = 8192;   // 64 rows x 128 bytes (M <= 64)
+constexpr int kStageW = 16384;  // 128 rows x 128 bytes (block_n <= 128)
+constexpr int kStageSfa = 2048;
+constexpr int kStageSfb = 2048;
+constexpr int kStage = kStageA + kStageW + kStageSfa + kStageSfb;
+constexpr int kRedLd = 128 + 4;
+constexpr int kRedBytes = 64 * kRedLd * 4;
+constexpr int kOffRed = kRing * kStage;
+constexpr int kOffBar = kOffRed + kRedBytes;
+// barriers: full[R], empty[R], acc_full[2], acc_empty[2]
+constexpr int kOffMisc = kOffBar + (2 * kRing + 4) * 8;
+// misc words: [0] TMEM base, [1] abort flag, [2] red_in (partials received as owner),
+// [3] red_free (frees received as member)
+constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+constexpr int kTmemCols = 512;  // two 128-column accumulators + scale columns
+constexpr int kColSfa = 256;
+constexpr int kColSfb = 272;
+constexpr int kSfAtom = 512;
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned int ld_acquire_cluster_smem(uint32_t addr) {
+    unsigned int v;
+    asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_add_release_cluster(uint32_t cluster_addr, unsigned int v) {
+    asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier of the 128 epilogue threads that also ANDs a flag across them: every decision to
+// abandon the work is taken by all four warps together (a named barrier has no timeout, so
+// no warp may leave while the others still expect it).
+__device__ __forceinline__ bool bar_epi_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v))
+        : "memory");
+    return r != 0;
+}
+
+// Bounded wait until *p >= target (acquire, gpu scope).
+__device__ bool wait_counter(const unsigned int *p, unsigned int target, volatile int *abort_flag, uint32_t *status) {
+    if (ld_acquire_gpu(p) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(p) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(status, static_cast<uint32_t>(kStatusOk), static_cast<uint32_t>(kStatusTimeoutOp));
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+// Bounded wait until the local shared-memory counter at `addr` >= target (acquire, cluster).
+__device__ bool wait_smem_counter(uint32_t addr, unsigned int target, volatile int *abort_flag, uint32_t *status) {
+    if (ld_acquire_cluster_smem(addr) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (ld_acquire_cluster_smem(addr) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(status, static_cast<uint32_t>(kStatusOk), static_cast<uint32_t>(kStatusTimeoutPeer));
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+struct Unit {
+    int tile, split, kt0, kt1, owner_rank;
+};
+
+__device__ __forceinline__ int op_rounds(const ExecOp &op, int teams, int C) {
+    const int per_round = teams * (C / op.splits);
+    return (op.n_tiles + per_round - 1) / per_round;
+}
+// The GEMM unit of (team, rank) in round r, if any.
+__device__ __forceinline__ bool op_unit(const ExecOp &op, int team, int rank, int teams, int C, int r, Unit &u) {
+    const int per_team = C / op.splits;
+    const int tile = (r * teams + team) * per_team + rank / op.splits;
+    if (tile >= op.n_tiles) return false;
+    u.tile = tile;
+    u.split = rank % op.splits;
+    u.kt0 = u.split * op.kt_per_split;
+    u.kt1 = min(op.k_tiles, u.kt0 + op.kt_per_split);
+    u.owner_rank = (rank / op.splits) * op.splits;
+    return true;
+}
+
+// Kept out of line: the norm path has its own register allocation, apart from the
+// epilogue's.
+template <int BPT>
+__device__ __noinline__ void norm_row_bpt(const NormArgs &a, int row, int lane) {
+    norm_row<32, BPT, false>(a, row, lane, nullptr);
+}
+__device__ void norm_row_any(const NormArgs &a, int bpt, int row, int lane) {
+    switch (bpt) {
+    case 1: norm_row_bpt<1>(a, row, lane); break;
+    case 2: norm_row_bpt<2>(a, row, lane); break;
+    case 3: norm_row_bpt<3>(a, row, lane); break;
+    case 4: norm_row_bpt<4>(a, row, lane); break;
+    case 5: norm_row_bpt<5>(a, row, lane); break;
+    case 6: norm_row_bpt<6>(a, row, lane); break;
+    case 7: norm_row_bpt<7>(a, row, lane); break;
+    default: norm_row_bpt<8>(a, row, lane); break;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kOffBar;
+    const uint32_t bar_empty = bar_full + 8 * kRing;
+    const uint32_t bar_accf = bar_empty + 8 * kRing;
+    const uint32_t bar_acce = bar_accf + 16;
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+    const uint32_t red_in_addr = sbase + kOffMisc + 8;
+    const uint32_t red_free_addr = sbase + kOffMisc + 12;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = P.cluster;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int team = blockIdx.x / C;
+    const int teams = gridDim.x / C;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_accf + 8 * b, 1);
+            mbar_init(bar_acce + 8 * b, 1);
+        }
+        misc[1] = 0;
+        misc[2] = 0;
+        misc[3] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t *>(misc)), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cluster_sync_all();  // every CTA's counters are initialised before any remote update
+    const uint32_t tmem = misc[0];
+
+    auto nkb_of = [&](const ExecOp &op, int kt) { return min(4, op.k_atoms - 4 * kt); };
+
+    if (warp == 0 && lane == 0) {
+        // ---------------------------- weight producer ----------------------------
+        const uint64_t pol = policy_evict_first();
+        int step = 0;
+        for (int i = 0; i < P.n_ops; ++i) {
+            const ExecOp &op = P.ops[i];
+            if (op.type != kOpGemm) continue;
+            const CUtensorMap *tmB = P.maps + op.tm_b;
+            const int rounds = op_rounds(op, teams, C);
+            for (int r = 0; r < rounds; ++r) {
+                Unit u;
+                if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
+                    const int slot = step % kRing, use = step / kRing;
+                    if (use > 0 && !mbar_wait(bar_empty + 8 * slot, (use - 1) & 1, abort_flag, P.status,
+                                              kStatusTimeoutEmpty))
+                        goto done_w;
+                    const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
+                    const uint32_t full = bar_full + 8 * slot;
+                    const uint32_t st = sbase + slot * kStage;
+                    mbar_arrive_expect_tx(full, op.a_box_rows * 128u + static_cast<uint32_t>(op.bn) * 128u + 2 * nb);
+                    tma_load_2d(st + kStageA, tmB, kt * 128, u.tile * op.bn, full, pol);
+                    const size_t grp = static_cast<size_t>((u.tile * op.bn) / 128);
+                    bulk_load(st + kStageA + kStageW + kStageSfa, op.sfb + (grp * op.k_atoms + 4 * kt) * kSfAtom, nb,
+                              full, pol);
+                }
+            }
+        }
+    done_w:;
+    } else if (warp == 2 && lane == 0) {
+        // ---------------------------- activation producer ----------------------------
+        const uint64_t pol = policy_evict_last();
+        int step = 0;
+        for (int i = 0; i < P.n_ops; ++i) {
+            const ExecOp &op = P.ops[i];
+            if (op.type != kOpGemm) continue;
+            const CUtensorMap *tmA = P.maps + op.tm_a;
+            bool ready = false;
+            const int rounds = op_rounds(op, teams, C);
+            for (int r = 0; r < rounds; ++r) {
+                Unit u;
+                if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                if (!ready) {
+                    if (i > 0 && !wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status)) goto done_a;
+                    fence_proxy_async_global();  // the input was written through the generic proxy
+                    ready = true;
+                }
+                for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
+                    const int slot = step % kRing, use = step / kRing;
+                    if (use > 0 && !mbar_wait(bar_empty + 8 * slot, (use - 1) & 1, abort_flag, P.status,
+                                              kStatusTimeoutEmpty))
+                        goto done_a;
+                    const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
+                    const uint32_t full = bar_full + 8 * slot;
+                    const uint32_t st = sbase + slot * kStage;
+                    tma_load_2d(st, tmA, kt * 128, 0, full, pol);
+                    bulk_load(st + kStageA + kStageW, op.sfa + static_cast<size_t>(4 * kt) * kSfAtom, nb, full, pol);
+                }
+            }
+        }
+    done_a:;
+    } else if (warp == 1 && lane == 0) {
+        // ---------------------------- MMA issuer ----------------------------
+        int step = 0, unit_idx = 0;
+        for (int i = 0; i < P.n_ops; ++i) {
+            const ExecOp &op = P.ops[i];
+            if (op.type != kOpGemm) continue;
+            const uint32_t idesc = idesc_mxf4nvf4(128, op.bn);
+            const int rounds = op_rounds(op, teams, C);
+            for (int r = 0; r < rounds; ++r) {
+                Unit u;
+                if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                const int b = unit_idx & 1, acc_use = unit_idx >> 1;
+                if (acc_use > 0 && !mbar_wait(bar_acce + 8 * b, (acc_use - 1) & 1, abort_flag, P.status,
+                                              kStatusTimeoutAccum))
+                    goto done_m;
+                tc_fence_after();
+                const uint32_t t_acc = tmem + static_cast<uint32_t>(b * 128);
+                // a 64-row W tile reads its half of the 128-row scale atom
+                const uint32_t sub = (op.bn == 64) ? static_cast<uint32_t>(((u.tile * op.bn) & 127) >> 5) : 0u;
+                for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
+                    const int slot = step % kRing, use = step / kRing;
+                    if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
+                        goto done_m;
+                    tc_fence_after();
+                    const int nkb = nkb_of(op, kt);
+                    const uint32_t st = sbase + slot * kStage;
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * kb,
+                                             desc_sf_32x128b(st + kStageA + kStageW + kb * kSfAtom));
+                        tc_cp_32x128b_warpx4(tmem + kColSfb + 4 * kb,
+                                             desc_sf_32x128b(st + kStageA + kStageW + kStageSfa + kb * kSfAtom));
+                    }
+                    for (int kb = 0; kb < nkb; ++kb)
+                        tc_mma_mxf4nvf4(t_acc, desc_kmajor_sw128(st + 32 * kb), desc_kmajor_sw128(st + kStageA + 32 * kb),
+                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 4 * kb + sub,
+                                        (kt > u.kt0 || kb > 0) ? 1u : 0u);
+                    tc_commit(bar_empty + 8 * slot);
+                }
+                tc_commit(bar_accf + 8 * b);
+                ++unit_idx;
+            }
+        }
+    done_m:;
+    } else if (warp >= 3) {
+        // ---------------------------- epilogue / norm workers ----------------------------
+        const int e = threadIdx.x - 96;  // 0..127
+        const int ew = e >> 5;           // worker warp 0..3
+        const int q = warp & 3;          // TMEM sub-partition this warp reads
+        const int row = q * 32 + lane;
+        int unit_idx = 0;
+        unsigned int owner_uses = 0, member_uses = 0;
+        for (int i = 0; i < P.n_ops; ++i) {
+            const ExecOp &op = P.ops[i];
+            if (op.type == kOpNorm) {
+                const int rows_per_round = gridDim.x * 4;
+                if (blockIdx.x * 4 >= op.norm.M) continue;  // no rows for this CTA
+                const bool ok = (e != 0) || i == 0 || wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status);
+                if (!bar_epi_and(ok)) goto done_e;
+                for (int rr = blockIdx.x * 4 + ew; rr < op.norm.M; rr += rows_per_round) {
+                    norm_row_any(op.norm, op.bpt, rr, lane);
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence();
+                        atomicAdd(P.done + i, 1u);
+                    }
+                }
+                continue;
+            }
+            // GEMM op
+            const int rounds = op_rounds(op, teams, C);
+            bool dep_seen = false;
+            for (int r = 0; r < rounds; ++r) {
+                Unit u;
+                if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                if (!dep_seen) {
+                    // the epilogue reads residuals written by earlier ops: acquire here too
+                    const bool ok =
+                        (e != 0) || i == 0 || wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status);
+                    if (!bar_epi_and(ok)) goto done_e;
+                    dep_seen = true;
+                }
+                const int b = unit_idx & 1, acc_use = unit_idx >> 1;
+                const bool got = mbar_wait(bar_accf + 8 * b, acc_use & 1, abort_flag, P.status,
+                                           kStatusTimeoutAccum);
+                if (!bar_epi_and(got)) goto done_e;
+                tc_fence_after();
+                const int rows_valid = min(64, op.M);
+                const uint32_t t_row = tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
+                const int n0 = u.tile * op.bn;
+                if (op.splits == 1) {
+                    for (int c0 = 0; c0 < op.bn; c0 += 32) {
+                        uint32_t rg[32];
+                        tmem_ld_32x32b_x32(t_row + c0, rg);
+                        tmem_ld_wait();
+                        if (row < rows_valid) {
+                            float v[32];
+#pragma unroll
+                            for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(rg[t]);
+                            epilogue_chunk(op, row, n0 + c0, v);
+                        }
+                    }
+                    tc_fence_before();
+                    bar_epi();
+                    if (e == 0) {
+                        mbar_arrive(bar_acce + 8 * b);
+                        __threadfence();
+                        atomicAdd(P.done + i, 1u);
+                    }
+                } else {
+                    // member: wait until the previous partial in `red` has been read, then write
+                    if (!bar_epi_and(wait_smem_counter(red_free_addr, member_uses, abort_flag, P.status))) goto done_e;
+                    float *red = reinterpret_cast<float *>(smem + kOffRed);
+                    for (int c0 = 0; c0 < op.bn; c0 += 32) {
+                        uint32_t rg[32];
+                        tmem_ld_32x32b_x32(t_row + c0, rg);
+                        tmem_ld_wait();
+                        if (row < rows_valid) {
+                            float4 *dst = reinterpret_cast<float4 *>(red + row * kRedLd + c0);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                dst[j] = make_float4(__uint_as_float(rg[4 * j]), __uint_as_float(rg[4 * j + 1]),
+                                                     __uint_as_float(rg[4 * j + 2]), __uint_as_float(rg[4 * j + 3]));
+                        }
+                    }
+                    tc_fence_before();
+                    bar_epi();
+                    if (e == 0) {
+                        mbar_arrive(bar_acce + 8 * b);
+                        red_add_release_cluster(mapa_shared(red_in_addr, static_cast<uint32_t>(u.owner_rank)), 1u);
+                    }
+                    ++member_uses;
+                    if (u.split == 0) {
+                        // owner: add the S partials of the group in split order, run the epilogue
+                        ++owner_uses;
+                        if (!bar_epi_and(wait_smem_counter(red_in_addr, owner_uses * static_cast<unsigned>(op.splits), abort_flag, P.status)))
+                            goto done_e;
+                        const int chunks = op.bn / 32;
+                        for (int item = e;; item += 128) {
+                            const int i_row = item / chunks, ch = item % chunks;
+                            if (i_row >= rows_valid) break;
+                            const uint32_t local = smem_u32(red + i_row * kRedLd + ch * 32);
+                            float v[32];
+#pragma unroll
+                            for (int t = 0; t < 32; ++t) v[t] = 0.0f;
+                            for (int sp = 0; sp < op.splits; ++sp) {
+                                const uint32_t src = mapa_shared(local, static_cast<uint32_t>(u.owner_rank + sp));
+                                float4 w4[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) w4[j] = ld_dsmem_f4(src + 16 * j);
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    v[4 * j] = __fadd_rn(v[4 * j], w4[j].x);
+                                    v[4 * j + 1] = __fadd_rn(v[4 * j + 1], w4[j].y);
+                                    v[4 * j + 2] = __fadd_rn(v[4 * j + 2], w4[j].z);
+                                    v[4 * j + 3] = __fadd_rn(v[4 * j + 3], w4[j].w);
+                                }
+                            }
+                            epilogue_chunk(op, i_row, n0 + ch * 32, v);
+                        }
+                        bar_epi();
+                        if (e == 0) {
+                            for (int sp = 0; sp < op.splits; ++sp)
+                                red_add_release_cluster(
+                                    mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
+                            __threadfence();
+                            atomicAdd(P.done + i, 1u);
+                        }
+                    }
+                }
+                ++unit_idx;
+            }
+        }
+    done_e:;
+    }
+
+    // teardown: peers may still read this CTA's shared memory until everyone is done
+    __syncwarp();
+    if (*abort_flag) {
+        // an abandoned run may leave copies or MMAs in flight: give them time to land
+        // before shared and tensor memory are released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t exec_grid(int cluster, int *grid) {
+    cudaError_t e = cudaFuncSetAttribute(exec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, exec_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    *grid = n * cluster;
+    return n > 0 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+cudaError_t exec_launch(const ExecParams &p, int grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(exec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(p.cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;  // CTAs wait on one another: all must be resident
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, exec_kernel, p);
+}
+
+cudaError_t probe_exec_kernel() {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, exec_kernel);
+}
+
+}  // namespace nvfp4

@@ -458,6 +458,13 @@ cudaError_t probe_gemm_kernels() {
     return cudaFuncGetAttributes(&fa, gemm_kernel<128, 5, false>);
 }
 
+cudaError_t device_status_address(uint32_t **p) {
+    void *a = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&a, g_device_status);
+    *p = static_cast<uint32_t *>(a);
+    return e;
+}
+
 cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return e;

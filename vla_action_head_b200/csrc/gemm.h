@@ -47,6 +47,9 @@ cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 // Programmatic dependent launch for this library's kernels: on unless NVFP4_PDL=0.
 bool pdl_enabled();
 
+// Device address of the library's status word (for kernels in other translation units).
+cudaError_t device_status_address(uint32_t **p);
+
 // Reads the device status word and clears it (after synchronising `s`).
 cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out);
 

@@ -16,6 +16,8 @@ enum : uint32_t {
     kStatusTimeoutEmpty = 2,    // producer waited too long for a free stage
     kStatusTimeoutAccum = 3,    // epilogue waited too long for the accumulator
     kStatusTimeoutDrain = 4,    // teardown waited too long for copies / MMAs in flight
+    kStatusTimeoutOp = 5,       // executor: an op's input never completed
+    kStatusTimeoutPeer = 6,     // executor: a split-K partner never delivered / released
 };
 
 // Wall-clock bound of one wait (ns).  Far above any legitimate wait of these kernels.
@@ -42,6 +44,9 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;

@@ -36,6 +36,22 @@ class _Tensor(C.Structure):
                 ("rows", C.c_int), ("K", C.c_int)]
 
 
+class _Op(C.Structure):
+    _fields_ = [("type", C.c_int), ("M", C.c_int), ("N", C.c_int), ("K", C.c_int),
+                ("x", C.c_void_p), ("ldx", C.c_int), ("norm", C.c_int),
+                ("gamma", C.c_void_p), ("beta", C.c_void_p), ("mod_scale", C.c_void_p),
+                ("mod_shift", C.c_void_p), ("eps", C.c_float),
+                ("A", _Tensor), ("W", _Tensor), ("epi", C.c_int), ("bias", C.c_void_p),
+                ("residual", C.c_void_p), ("ldr", C.c_int), ("out_bf16", C.c_void_p), ("ldo", C.c_int),
+                ("out_codes", C.c_void_p), ("out_sf", C.c_void_p), ("out_global_scale", C.c_float)]
+
+
+class _Program(C.Structure):
+    _fields_ = [("buffer", C.c_void_p), ("bytes", C.c_size_t), ("n_ops", C.c_int), ("grid", C.c_int),
+                ("cluster", C.c_int), ("ops_offset", C.c_size_t), ("maps_offset", C.c_size_t),
+                ("done_offset", C.c_size_t)]
+
+
 _lib = None
 P, I, F, SZ = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
@@ -63,6 +79,9 @@ def lib():
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
             "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
                                F, P, SZ, P]),
+            "nvfp4_program_bytes": (SZ, [I]),
+            "nvfp4_program_build": (I, [C.POINTER(_Op), I, P, SZ, C.POINTER(_Program)]),
+            "nvfp4_program_run": (I, [C.POINTER(_Program), P]),
             "nvfp4_gemm_noalloc": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P,
                                        P, F, P]),
             "nvfp4_gemm_ex": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P,
@@ -230,3 +249,47 @@ def probe():
 def device_status():
     """Raises NVFP4Error(TIMEOUT) if a kernel's bounded wait expired since the last check."""
     _check("nvfp4_get_device_status", lib().nvfp4_get_device_status(_stream()))
+
+
+# ---- layer executor ----------------------------------------------------------------------
+def op_norm(x, out: NVFP4Tensor, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6):
+    """A norm -> FP4 op of a program (bf16 x [M, K] -> out)."""
+    M, K = x.shape
+    op = _Op(type=0, M=M, N=0, K=K, x=x.data_ptr(), ldx=x.stride(0), norm=NORM[kind],
+             gamma=_ptr(gamma), beta=_ptr(beta), mod_scale=_ptr(scale), mod_shift=_ptr(shift), eps=eps,
+             out_codes=out.codes.data_ptr(), out_sf=out.sf.data_ptr(), out_global_scale=out.global_scale)
+    op.keep = (x, out, gamma, beta, scale, shift)  # the program only holds raw pointers
+    return op
+
+
+def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None, out_global_scale=1.0):
+    """A GEMM op of a program; `out` is bf16 [M, N] or, for FP4 epilogues, an NVFP4Tensor."""
+    e = EPI[epi]
+    op = _Op(type=1, M=a.rows, N=w.rows, K=a.K, A=a.c(), W=w.c(), epi=e, bias=_ptr(bias),
+             residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0)
+    if e in (4, 5):
+        op.out_codes, op.out_sf, op.out_global_scale = out.codes.data_ptr(), out.sf.data_ptr(), out_global_scale
+    else:
+        op.out_bf16, op.ldo, op.out_global_scale = out.data_ptr(), out.stride(0), 1.0
+    op.keep = (a, w, bias, residual, out)  # the program only holds raw pointers
+    return op
+
+
+class Program:
+    """A built program of ops (device buffer owned here); run() makes one launch.  It keeps
+    the ops, and through them every tensor they name, alive."""
+
+    def __init__(self, ops, device="cuda"):
+        self.ops = list(ops)
+        torch = _torch()
+        n = len(ops)
+        arr = (_Op * n)(*ops)
+        nbytes = int(lib().nvfp4_program_bytes(n))
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = (self.buf.data_ptr() + 255) // 256 * 256
+        self.prog = _Program()
+        _check("nvfp4_program_build", lib().nvfp4_program_build(arr, n, C.c_void_p(base), nbytes, C.byref(self.prog)))
+        self.n_ops = n
+
+    def run(self):
+        _check("nvfp4_program_run", lib().nvfp4_program_run(C.byref(self.prog), _stream()))
