@@ -123,7 +123,10 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * id, then globaltimer ns at set-up done, first operand stage landed, last MMA issued,
  * accumulator ready, epilogue done.  Launches that no longer fit are not traced.  Setting
  * a buffer (or NULL, which turns tracing off) rewinds the cursor.  Host-side state, not
- * thread safe; captured launches keep the slice they got at capture. */
+ * thread safe; captured launches keep the slice they got at capture.
+ * nvfp4_program_run, when the buffer holds n_ops * grid * 8 words, writes 8 stamps per
+ * (op, CTA) at ((op * grid) + cta) * 8: weight tile issued, input ready, first stage
+ * landed, last MMA issued, accumulator ready, partials received, op signalled, norm rows done. */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */

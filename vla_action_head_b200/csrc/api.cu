@@ -633,6 +633,8 @@ nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream)
     p.n_ops = prog->n_ops;
     p.cluster = prog->cluster;
     if (device_status_address(&p.status) != cudaSuccess) return NVFP4_ERR_CUDA;
+    p.trace = (g_trace != nullptr && g_trace_words >= static_cast<size_t>(prog->n_ops) * prog->grid * 8) ? g_trace
+                                                                                                          : nullptr;
     cudaError_t e = cudaMemsetAsync(p.done, 0, static_cast<size_t>(prog->n_ops) * 4, stream);
     if (e == cudaSuccess) e = exec_launch(p, prog->grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();

@@ -44,6 +44,7 @@ struct ExecParams {
     int n_ops;
     int cluster;       // CTAs per cluster (the split-K reduction group size limit)
     uint32_t *status;  // the library's device status word
+    unsigned long long *trace;  // optional: 8 globaltimer stamps per (op, CTA)
 };
 
 // Largest grid (multiple of `cluster`) whose CTAs are all co-resident.

@@ -204,6 +204,12 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     const uint32_t tmem = misc[0];
 
     auto nkb_of = [&](const ExecOp &op, int kt) { return min(4, op.k_atoms - 4 * kt); };
+    // diagnostics: per (op, CTA) [0] W issued first tile, [1] A dependency seen, [2] first
+    // stage full (MMA), [3] last MMA issued, [4] accumulator ready (epilogue), [5] partials in
+    // (owner), [6] op signalled, [7] norm rows done
+    auto stamp = [&](int op_i, int k) {
+        if (P.trace != nullptr) P.trace[(static_cast<size_t>(op_i) * gridDim.x + blockIdx.x) * 8 + k] = globaltimer_ns();
+    };
 
     if (warp == 0 && lane == 0) {
         // ---------------------------- weight producer ----------------------------
@@ -225,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                     const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
                     const uint32_t full = bar_full + 8 * slot;
                     const uint32_t st = sbase + slot * kStage;
+                    if (kt == u.kt0) stamp(i, 0);
                     mbar_arrive_expect_tx(full, op.a_box_rows * 128u + static_cast<uint32_t>(op.bn) * 128u + 2 * nb);
                     tma_load_2d(st + kStageA, tmB, kt * 128, u.tile * op.bn, full, pol);
                     const size_t grp = static_cast<size_t>((u.tile * op.bn) / 128);
@@ -251,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                     if (i > 0 && !wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status)) goto done_a;
                     fence_proxy_async_global();  // the input was written through the generic proxy
                     ready = true;
+                    stamp(i, 1);
                 }
                 for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
                     const int slot = step % kRing, use = step / kRing;
@@ -290,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                     if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
                         goto done_m;
                     tc_fence_after();
+                    if (kt == u.kt0) stamp(i, 2);
                     const int nkb = nkb_of(op, kt);
                     const uint32_t st = sbase + slot * kStage;
                     for (int kb = 0; kb < nkb; ++kb) {
@@ -304,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                                         (kt > u.kt0 || kb > 0) ? 1u : 0u);
                     tc_commit(bar_empty + 8 * slot);
                 }
+                stamp(i, 3);
                 tc_commit(bar_accf + 8 * b);
                 ++unit_idx;
             }
@@ -324,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 if (blockIdx.x * 4 >= op.norm.M) continue;  // no rows for this CTA
                 const bool ok = (e != 0) || i == 0 || wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status);
                 if (!bar_epi_and(ok)) goto done_e;
+                if (e == 0) stamp(i, 1);
                 for (int rr = blockIdx.x * 4 + ew; rr < op.norm.M; rr += rows_per_round) {
                     norm_row_any(op.norm, op.bpt, rr, lane);
                     __syncwarp();
@@ -332,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                         atomicAdd(P.done + i, 1u);
                     }
                 }
+                if (e == 0) stamp(i, 7);
                 continue;
             }
             // GEMM op
@@ -352,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                                            kStatusTimeoutAccum);
                 if (!bar_epi_and(got)) goto done_e;
                 tc_fence_after();
+                if (e == 0) stamp(i, 4);
                 const int rows_valid = min(64, op.M);
                 const uint32_t t_row = tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
                 const int n0 = u.tile * op.bn;
@@ -373,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                         mbar_arrive(bar_acce + 8 * b);
                         __threadfence();
                         atomicAdd(P.done + i, 1u);
+                        stamp(i, 6);
                     }
                 } else {
                     // member: wait until the previous partial in `red` has been read, then write
@@ -402,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                         ++owner_uses;
                         if (!bar_epi_and(wait_smem_counter(red_in_addr, owner_uses * static_cast<unsigned>(op.splits), abort_flag, P.status)))
                             goto done_e;
+                        if (e == 0) stamp(i, 5);
                         const int chunks = op.bn / 32;
                         for (int item = e;; item += 128) {
                             const int i_row = item / chunks, ch = item % chunks;
@@ -432,6 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                                     mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
                             __threadfence();
                             atomicAdd(P.done + i, 1u);
+                            stamp(i, 6);
                         }
                     }
                 }
