@@ -27,16 +27,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Epilogue of one 32-column chunk held by this thread (row m, columns n .. n + 31).
+// Every field of p is read once into a local first: the byte stores of the FP4 outputs may
+// alias any memory as far as the compiler knows, and p may live in global memory.
 template <class P>
 __device__ __forceinline__ void epilogue_chunk(const P &p, int m, int n, float *v) {
-    const int epi = p.epi;
-    const bool has_bias = p.bias != nullptr &&
+    const int epi = p.epi, N = p.N, ldr = p.ldr, ldo = p.ldo;
+    const float alpha = p.alpha, g_out = p.g_out;
+    const uint16_t *const bias = p.bias;
+    const uint16_t *const residual = p.residual;
+    uint16_t *const out = p.out;
+    uint8_t *const out_codes = p.out_codes;
+    uint8_t *const out_sf = p.out_sf;
+    const bool has_bias = bias != nullptr &&
                           (epi == kEpiBias || epi == kEpiBiasResidual || epi == kEpiBiasGelu || epi == kEpiGeglu);
     const bool has_res = (epi == kEpiResidual || epi == kEpiBiasResidual);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], p.alpha);
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], alpha);
     if (has_bias) {
-        const uint4 *bq = reinterpret_cast<const uint4 *>(p.bias + n);
+        const uint4 *bq = reinterpret_cast<const uint4 *>(bias + n);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint4 u = __ldg(bq + j);
@@ -49,10 +57,10 @@ __device__ __forceinline__ void epilogue_chunk(const P &p, int m, int n, float *
         }
     }
     if (has_res) {
-        const uint4 *rq = reinterpret_cast<const uint4 *>(p.residual + static_cast<size_t>(m) * p.ldr + n);
+        const uint4 *rq = reinterpret_cast<const uint4 *>(residual + static_cast<size_t>(m) * ldr + n);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 u = rq[j];
+            const uint4 u = __ldcg(rq + j);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
@@ -62,33 +70,33 @@ __device__ __forceinline__ void epilogue_chunk(const P &p, int m, int n, float *
         }
     }
     if (epi == kEpiBiasGelu) {
-        const float d6g = __fmul_rn(6.0f, p.g_out);
-        const int k_atoms_out = (p.N + 63) >> 6;
+        const float d6g = __fmul_rn(6.0f, g_out);
+        const int k_atoms_out = (N + 63) >> 6;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             float y[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) y[i] = gelu_tanh_f(v[16 * h + i]);
             uint2 c;
-            const uint32_t s = quantize_block16(y, p.g_out, d6g, c);
+            const uint32_t s = quantize_block16(y, g_out, d6g, c);
             const int col = n + 16 * h;
-            *reinterpret_cast<uint2 *>(p.out_codes + static_cast<size_t>(m) * (p.N >> 1) + (col >> 1)) = c;
-            p.out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
+            *reinterpret_cast<uint2 *>(out_codes + static_cast<size_t>(m) * (N >> 1) + (col >> 1)) = c;
+            out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
         }
     } else if (epi == kEpiGeglu) {
-        const float d6g = __fmul_rn(6.0f, p.g_out);
-        const int n_out = p.N >> 1;
+        const float d6g = __fmul_rn(6.0f, g_out);
+        const int n_out = N >> 1;
         const int k_atoms_out = (n_out + 63) >> 6;
         float y[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(gelu_tanh_f(v[2 * j]), v[2 * j + 1]);
         uint2 c;
-        const uint32_t s = quantize_block16(y, p.g_out, d6g, c);
+        const uint32_t s = quantize_block16(y, g_out, d6g, c);
         const int col = n >> 1;  // first output column of this block
-        *reinterpret_cast<uint2 *>(p.out_codes + static_cast<size_t>(m) * (n_out >> 1) + (col >> 1)) = c;
-        p.out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
+        *reinterpret_cast<uint2 *>(out_codes + static_cast<size_t>(m) * (n_out >> 1) + (col >> 1)) = c;
+        out_sf[sf_offset(m, col >> 4, k_atoms_out)] = static_cast<uint8_t>(s);
     } else {
-        uint4 *oq = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(m) * p.ldo + n);
+        uint4 *oq = reinterpret_cast<uint4 *>(out + static_cast<size_t>(m) * ldo + n);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             oq[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),

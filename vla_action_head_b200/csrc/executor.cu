@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         const uint64_t pol = policy_evict_first();
         int step = 0;
         for (int i = 0; i < P.n_ops; ++i) {
-            const ExecOp &op = P.ops[i];
+            const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmB = P.maps + op.tm_b;
             const int rounds = op_rounds(op, teams, C);
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         const uint64_t pol = policy_evict_last();
         int step = 0;
         for (int i = 0; i < P.n_ops; ++i) {
-            const ExecOp &op = P.ops[i];
+            const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmA = P.maps + op.tm_a;
             bool ready = false;
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         // ---------------------------- MMA issuer ----------------------------
         int step = 0, unit_idx = 0;
         for (int i = 0; i < P.n_ops; ++i) {
-            const ExecOp &op = P.ops[i];
+            const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const uint32_t idesc = idesc_mxf4nvf4(128, op.bn);
             const int rounds = op_rounds(op, teams, C);
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         int unit_idx = 0;
         unsigned int owner_uses = 0, member_uses = 0;
         for (int i = 0; i < P.n_ops; ++i) {
-            const ExecOp &op = P.ops[i];
+            const ExecOp op = P.ops[i];
             if (op.type == kOpNorm) {
                 const int rows_per_round = gridDim.x * 4;
                 if (blockIdx.x * 4 >= op.norm.M) continue;  // no rows for this CTA

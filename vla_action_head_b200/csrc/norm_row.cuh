@@ -45,46 +45,70 @@ __device__ __forceinline__ double row_sum(double v, double *red) {
     }
 }
 
-// Loads the 16 params of block b (bf16) as fp32, or `dflt` when the pointer is NULL.
-__device__ __forceinline__ void load_param16(const uint16_t *p, int b, float dflt, float *out) {
-    if (p == nullptr) {
+// Pairwise fp64 sum of the 16 elements of one block (fp32 values, exact in fp64).
+template <class Elem>
+__device__ __forceinline__ double block_sum16(Elem elem) {
+    double v[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) out[i] = dflt;
-        return;
-    }
-    const uint4 *q = reinterpret_cast<const uint4 *>(p + static_cast<size_t>(b) * 16);
-    const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
-    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    for (int e = 0; e < 8; ++e) v[e] = __dadd_rn(static_cast<double>(elem(2 * e)), static_cast<double>(elem(2 * e + 1)));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        out[2 * i] = bf16lo(w[i]);
-        out[2 * i + 1] = bf16hi(w[i]);
-    }
+    for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int e = 0; e < w; ++e) v[e] = __dadd_rn(v[e], v[e + w]);
+    return v[0];
 }
 
 // Row `row` of p, handled by thread t of TPR (TPR = 32: one warp; TPR = 128: the CTA, with
 // `red` four doubles of shared memory).  TPR, BPT (blocks of 16 per thread) and F32 (fp32
 // input, else bf16) are compile-time; K <= 16 * TPR * BPT.
+//
+// Latency is what matters at tens of rows, so every global load of the row is issued
+// first: the x blocks (ld.global.cg: x may have been written earlier in the same launch by
+// other SMs), and the per-column parameters (bf16, read-only; in registers for BPT <= 4,
+// else prefetched into L1).  The fp64 sums are pairwise trees per block, so the dependent
+// chain is a few adds rather than one per element; fp64 keeps the rounded fp32 statistics
+// independent of the summation order.
 template <int TPR, int BPT, bool F32>
 __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, double *red) {
     constexpr int kWords = F32 ? 16 : 8;  // 32-bit words per 16-element block
-    const int nblk = p.K >> 4;
-    const int k_atoms = (p.K + 63) >> 6;
-    const bool row_ok = row < p.M;
+    constexpr bool kParamRegs = BPT <= 4;
+    // Every field is read once into a local: the byte stores below may alias any memory as
+    // far as the compiler knows, and `p` may live in global memory (executor programs).
+    const int M = p.M, K = p.K, ldx = p.ldx, kind = p.kind;
+    const void *const x = p.x;
+    const float eps = p.eps, g_arg = p.g;
+    const uint32_t *const amax_bits = p.amax_bits;
+    uint8_t *const codes_out = p.codes;
+    uint8_t *const sf_out = p.sf;
+    float *const y_out = p.y_out;
+    const int nblk = K >> 4;
+    const int k_atoms = (K + 63) >> 6;
+    const bool row_ok = row < M;
     int src_row = row;
-    if (p.interleave) src_row = (row & 1) ? (p.M >> 1) + (row >> 1) : (row >> 1);
+    if (p.interleave) src_row = (row & 1) ? (M >> 1) + (row >> 1) : (row >> 1);
+
+    const bool ln = (kind == kLayerNorm || kind == kAdaLN);
+    const bool ada = (kind == kAdaLN || kind == kAdaRms);
+    const bool has_a = kind != kNone;
+    const bool add_b = (kind == kLayerNorm) || (kind == kAdaLN) || (kind == kAdaRms && p.shift != nullptr);
+    // y = n * A + B with A = gamma (default 1) or 1 + scale (default scale 0), B = beta / shift
+    const uint16_t *pa = ada ? p.scale : p.gamma;
+    const uint16_t *pb = (kind == kLayerNorm) ? p.beta : p.shift;
+    const uint32_t pa_dflt = ada ? 0u : 0x3F803F80u;  // bf16 pair (0, 0) or (1, 1)
 
     uint32_t raw[BPT][kWords];
-    const char *xrow = static_cast<const char *>(p.x) +
-                       static_cast<size_t>(row_ok ? src_row : 0) * p.ldx * (F32 ? 4 : 2);
+    uint32_t wa[kParamRegs ? BPT : 1][8], wb[kParamRegs ? BPT : 1][8];
+    const char *xrow = static_cast<const char *>(x) +
+                       static_cast<size_t>(row_ok ? src_row : 0) * ldx * (F32 ? 4 : 2);
 #pragma unroll
     for (int i = 0; i < BPT; ++i) {
         const int b = t + i * TPR;
-        if (row_ok && b < nblk) {
+        const bool ok = row_ok && b < nblk;
+        if (ok) {
             const uint4 *q = reinterpret_cast<const uint4 *>(xrow + static_cast<size_t>(b) * 16 * (F32 ? 4 : 2));
 #pragma unroll
             for (int j = 0; j < kWords / 4; ++j) {
-                const uint4 u = __ldg(q + j);
+                const uint4 u = __ldcg(q + j);
                 raw[i][4 * j] = u.x;
                 raw[i][4 * j + 1] = u.y;
                 raw[i][4 * j + 2] = u.z;
@@ -94,6 +118,30 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
 #pragma unroll
             for (int j = 0; j < kWords; ++j) raw[i][j] = 0u;
         }
+        if constexpr (kParamRegs) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                wa[i][j] = pa_dflt;
+                wb[i][j] = 0u;
+            }
+            if (ok && has_a && pa != nullptr) {
+                const uint4 *q = reinterpret_cast<const uint4 *>(pa + static_cast<size_t>(b) * 16);
+                const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
+                wa[i][0] = u0.x; wa[i][1] = u0.y; wa[i][2] = u0.z; wa[i][3] = u0.w;
+                wa[i][4] = u1.x; wa[i][5] = u1.y; wa[i][6] = u1.z; wa[i][7] = u1.w;
+            }
+            if (ok && add_b && pb != nullptr) {
+                const uint4 *q = reinterpret_cast<const uint4 *>(pb + static_cast<size_t>(b) * 16);
+                const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
+                wb[i][0] = u0.x; wb[i][1] = u0.y; wb[i][2] = u0.z; wb[i][3] = u0.w;
+                wb[i][4] = u1.x; wb[i][5] = u1.y; wb[i][6] = u1.z; wb[i][7] = u1.w;
+            }
+        } else {
+            if (ok && has_a && pa != nullptr)
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(pa + static_cast<size_t>(b) * 16));
+            if (ok && add_b && pb != nullptr)
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(pb + static_cast<size_t>(b) * 16));
+        }
     }
     auto elem = [&](int i, int e) -> float {
         if constexpr (F32) return __uint_as_float(raw[i][e]);
@@ -102,48 +150,58 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
 
     // ---- row statistics (fp64) ----
     float mu_f = 0.0f, rstd_f = 1.0f;
-    const int kind = p.kind;
-    if (kind == kLayerNorm || kind == kAdaLN) {
+    if (ln) {
         double s = 0.0;
 #pragma unroll
-        for (int i = 0; i < BPT; ++i)
-#pragma unroll
-            for (int e = 0; e < 16; ++e) s = __dadd_rn(s, static_cast<double>(elem(i, e)));
+        for (int i = 0; i < BPT; ++i) s = __dadd_rn(s, block_sum16([&](int e) { return elem(i, e); }));
         s = row_sum<TPR>(s, red);
-        const double mu = __ddiv_rn(s, static_cast<double>(p.K));
+        const double mu = __ddiv_rn(s, static_cast<double>(K));
         double q = 0.0;
 #pragma unroll
         for (int i = 0; i < BPT; ++i) {
             if (t + i * TPR < nblk) {
+                double d[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const double dv = __dsub_rn(static_cast<double>(elem(i, e)), mu);
-                    q = __dadd_rn(q, __dmul_rn(dv, dv));
+                    d[e] = __dmul_rn(dv, dv);
                 }
+#pragma unroll
+                for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                    for (int e = 0; e < w; ++e) d[e] = __dadd_rn(d[e], d[e + w]);
+                q = __dadd_rn(q, d[0]);
             }
         }
         q = row_sum<TPR>(q, red);
         mu_f = static_cast<float>(mu);
         rstd_f = static_cast<float>(
-            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(p.K)), static_cast<double>(p.eps)))));
+            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(K)), static_cast<double>(eps)))));
     } else if (kind == kRmsNorm || kind == kAdaRms) {
         double q = 0.0;
 #pragma unroll
-        for (int i = 0; i < BPT; ++i)
+        for (int i = 0; i < BPT; ++i) {
+            double d[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const double xv = static_cast<double>(elem(i, e));
-                q = __dadd_rn(q, __dmul_rn(xv, xv));
+                d[e] = __dmul_rn(xv, xv);
             }
+#pragma unroll
+            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) d[e] = __dadd_rn(d[e], d[e + w]);
+            q = __dadd_rn(q, d[0]);
+        }
         q = row_sum<TPR>(q, red);
         rstd_f = static_cast<float>(
-            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(p.K)), static_cast<double>(p.eps)))));
+            __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(K)), static_cast<double>(eps)))));
     }
     if (!row_ok) return;
 
-    float g = p.g;
-    if (p.amax_bits != nullptr) {
-        const float amax = __uint_as_float(*p.amax_bits);
+    float g = g_arg;
+    if (amax_bits != nullptr) {
+        const float amax = __uint_as_float(*amax_bits);
         g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
     }
     const float d6g = __fmul_rn(6.0f, g);
@@ -154,41 +212,56 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
         const int b = t + i * TPR;
         if (b >= nblk) break;
         float y[16];
-        if (kind == kNone) {
+        if (!has_a) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) y[e] = elem(i, e);
         } else {
-            float pa[16], pb[16];
-            const bool ln = (kind == kLayerNorm || kind == kAdaLN);
-            const bool ada = (kind == kAdaLN || kind == kAdaRms);
-            if (ada) {
-                load_param16(p.scale, b, 0.0f, pa);
+            uint32_t ua[8], ub[8];
+            if constexpr (kParamRegs) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pa[e] = __fadd_rn(1.0f, pa[e]);
+                for (int j = 0; j < 8; ++j) {
+                    ua[j] = wa[i][j];
+                    ub[j] = wb[i][j];
+                }
             } else {
-                load_param16(p.gamma, b, 1.0f, pa);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    ua[j] = pa_dflt;
+                    ub[j] = 0u;
+                }
+                if (pa != nullptr) {
+                    const uint4 *q = reinterpret_cast<const uint4 *>(pa + static_cast<size_t>(b) * 16);
+                    const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
+                    ua[0] = u0.x; ua[1] = u0.y; ua[2] = u0.z; ua[3] = u0.w;
+                    ua[4] = u1.x; ua[5] = u1.y; ua[6] = u1.z; ua[7] = u1.w;
+                }
+                if (add_b && pb != nullptr) {
+                    const uint4 *q = reinterpret_cast<const uint4 *>(pb + static_cast<size_t>(b) * 16);
+                    const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
+                    ub[0] = u0.x; ub[1] = u0.y; ub[2] = u0.z; ub[3] = u0.w;
+                    ub[4] = u1.x; ub[5] = u1.y; ub[6] = u1.z; ub[7] = u1.w;
+                }
             }
-            const bool add_b = (kind == kLayerNorm) || (kind == kAdaLN) ||
-                               (kind == kAdaRms && p.shift != nullptr);
-            if (add_b) load_param16(kind == kLayerNorm ? p.beta : p.shift, b, 0.0f, pb);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 const float xv = elem(i, e);
+                float av = (e & 1) ? bf16hi(ua[e >> 1]) : bf16lo(ua[e >> 1]);
+                if (ada) av = __fadd_rn(1.0f, av);
                 const float n = ln ? __fmul_rn(__fsub_rn(xv, mu_f), rstd_f) : __fmul_rn(xv, rstd_f);
-                const float tt = __fmul_rn(n, pa[e]);
-                y[e] = add_b ? __fadd_rn(tt, pb[e]) : tt;
+                const float tt = __fmul_rn(n, av);
+                y[e] = add_b ? __fadd_rn(tt, (e & 1) ? bf16hi(ub[e >> 1]) : bf16lo(ub[e >> 1])) : tt;
             }
         }
-        if (p.y_out != nullptr) {
-            float4 *yo = reinterpret_cast<float4 *>(p.y_out + static_cast<size_t>(row) * p.K + b * 16);
+        if (y_out != nullptr) {
+            float4 *yo = reinterpret_cast<float4 *>(y_out + static_cast<size_t>(row) * K + b * 16);
 #pragma unroll
             for (int j = 0; j < 4; ++j) yo[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
             continue;
         }
         uint2 c;
         const uint32_t s = quantize_block16(y, g, d6g, c);
-        *reinterpret_cast<uint2 *>(p.codes + static_cast<size_t>(row) * (p.K >> 1) + b * 8) = c;
-        p.sf[sf_offset(row, b, k_atoms)] = static_cast<uint8_t>(s);
+        *reinterpret_cast<uint2 *>(codes_out + static_cast<size_t>(row) * (K >> 1) + b * 8) = c;
+        sf_out[sf_offset(row, b, k_atoms)] = static_cast<uint8_t>(s);
     }
 }
 

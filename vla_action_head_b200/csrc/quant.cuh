@@ -29,9 +29,14 @@ __host__ __device__ __forceinline__ size_t sf_offset(int row, int kblk, int k_at
 // nibble of byte 0) and returns the scale byte.
 __device__ __forceinline__ uint32_t quantize_block16(const float *y, float g, float d6g,
                                                      uint2 &codes) {
-    float a = 0.0f;
+    float m8[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(y[i]));
+    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fabsf(y[i]), fabsf(y[i + 8]));
+#pragma unroll
+    for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) m8[i] = fmaxf(m8[i], m8[i + w]);
+    const float a = fmaxf(0.0f, m8[0]);  // NaN inputs are ignored, as fmaxf does
     const float t = __fdiv_rn(a, d6g);
     const uint32_t s = cvt_e4m3_rn_satfinite(t);
     const float ds = e4m3_to_f32(s);
