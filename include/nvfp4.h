@@ -119,14 +119,16 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
 
 /* Diagnostics (tracing): while `buf` (device, `words` 64-bit words) is set, each
  * nvfp4_gemm launch takes the next free slice of it (8 words per CTA, CTA index
- * (split * m_tiles + m_tile) * n_tiles + n_tile) and writes: globaltimer ns at entry, SM
- * id, then globaltimer ns at set-up done, first operand stage landed, last MMA issued,
- * accumulator ready, epilogue done.  Launches that no longer fit are not traced.  Setting
+ * (split * m_tiles + m_tile) * n_tiles + n_tile) and writes globaltimer ns at: entry,
+ * split-K epilogue items done, set-up done, first operand stage landed, last MMA issued,
+ * accumulator ready, exit, split-K partials visible (words 1 and 7 stay 0 without
+ * split-K).  Launches that no longer fit are not traced.  Setting
  * a buffer (or NULL, which turns tracing off) rewinds the cursor.  Host-side state, not
  * thread safe; captured launches keep the slice they got at capture.
  * nvfp4_program_run, when the buffer holds n_ops * grid * 8 words, writes 8 stamps per
  * (op, CTA) at ((op * grid) + cta) * 8: weight tile issued, input ready, first stage
- * landed, last MMA issued, accumulator ready, partials received, op signalled, norm rows done. */
+ * landed, last MMA issued, accumulator ready, partials received, op signalled, and norm
+ * rows done (norm ops) or accumulator drained to shared memory (GEMM ops). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */

@@ -46,7 +46,12 @@ constexpr int kStage = kStageA + kStageW + kStageSfa + kStageSfb;
 constexpr int kRedLd = 128 + 4;
 constexpr int kRedBytes = 64 * kRedLd * 4;
 constexpr int kOffRed = kRing * kStage;
-constexpr int kOffBar = kOffRed + kRedBytes;
+// staged epilogue inputs of this CTA's column slice: residual rows (bf16) and bias
+constexpr int kStgLd = 128 + 8;
+constexpr int kOffStg = kOffRed + kRedBytes;
+constexpr int kStgBytes = 64 * kStgLd * 2;
+constexpr int kOffStgBias = kOffStg + kStgBytes;
+constexpr int kOffBar = kOffStgBias + 256;
 // barriers: full[R], empty[R], acc_full[2], acc_empty[2]
 constexpr int kOffMisc = kOffBar + (2 * kRing + 4) * 8;
 // misc words: [0] TMEM base, [1] abort flag, [2] red_in (partials received as owner),
@@ -206,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     auto nkb_of = [&](const ExecOp &op, int kt) { return min(4, op.k_atoms - 4 * kt); };
     // diagnostics: per (op, CTA) [0] W issued first tile, [1] A dependency seen, [2] first
     // stage full (MMA), [3] last MMA issued, [4] accumulator ready (epilogue), [5] partials in
-    // (owner), [6] op signalled, [7] norm rows done
+    // (split groups), [6] op signalled, [7] norm rows done / accumulator drained (GEMM)
     auto stamp = [&](int op_i, int k) {
         if (P.trace != nullptr) P.trace[(static_cast<size_t>(op_i) * gridDim.x + blockIdx.x) * 8 + k] = globaltimer_ns();
     };
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         const int q = warp & 3;          // TMEM sub-partition this warp reads
         const int row = q * 32 + lane;
         int unit_idx = 0;
-        unsigned int owner_uses = 0, member_uses = 0;
+        unsigned int in_expected = 0, free_expected = 0;  // split-group signals expected so far
         for (int i = 0; i < P.n_ops; ++i) {
             const ExecOp op = P.ops[i];
             if (op.type == kOpNorm) {
@@ -346,8 +351,20 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 if (e == 0) stamp(i, 7);
                 continue;
             }
-            // GEMM op
+            // GEMM op.  Every CTA of a split group finalizes its own slice of bn / S columns
+            // (a multiple of 32): it adds the S partials of those columns in split order, the
+            // first from its own shared memory or a peer's over DSMEM, and runs the epilogue.
             const int rounds = op_rounds(op, teams, C);
+            const int S = op.splits;
+            const int slice = op.bn / S;
+            const int chunks = slice / 32;
+            const bool has_bias = op.bias != nullptr && (op.epi == kEpiBias || op.epi == kEpiBiasResidual ||
+                                                         op.epi == kEpiBiasGelu || op.epi == kEpiGeglu);
+            const bool has_res = op.residual != nullptr && (op.epi == kEpiResidual || op.epi == kEpiBiasResidual);
+            const int rows_valid = min(64, op.M);
+            uint16_t *stg = reinterpret_cast<uint16_t *>(smem + kOffStg);
+            uint16_t *stg_bias = reinterpret_cast<uint16_t *>(smem + kOffStgBias);
+            float *red = reinterpret_cast<float *>(smem + kOffRed);
             bool dep_seen = false;
             for (int r = 0; r < rounds; ++r) {
                 Unit u;
@@ -359,98 +376,124 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                     if (!bar_epi_and(ok)) goto done_e;
                     dep_seen = true;
                 }
+                const int n0 = u.tile * op.bn;
+                const int c0 = u.split * slice;  // first column of this CTA's slice, in the tile
+                // stage the slice's residual rows and bias while the MMAs run
+                if (has_res) {
+                    const int per_row = slice / 8;
+                    for (int idx = e; idx < rows_valid * per_row; idx += 128) {
+                        const int rr = idx / per_row, c8 = idx % per_row;
+                        const uint4 val = __ldcg(reinterpret_cast<const uint4 *>(
+                            op.residual + static_cast<size_t>(rr) * op.ldr + n0 + c0 + 8 * c8));
+                        *reinterpret_cast<uint4 *>(stg + rr * kStgLd + 8 * c8) = val;
+                    }
+                }
+                if (has_bias && e < slice / 8)
+                    *reinterpret_cast<uint4 *>(stg_bias + 8 * e) =
+                        __ldg(reinterpret_cast<const uint4 *>(op.bias + n0 + c0 + 8 * e));
                 const int b = unit_idx & 1, acc_use = unit_idx >> 1;
                 const bool got = mbar_wait(bar_accf + 8 * b, acc_use & 1, abort_flag, P.status,
                                            kStatusTimeoutAccum);
                 if (!bar_epi_and(got)) goto done_e;
                 tc_fence_after();
                 if (e == 0) stamp(i, 4);
-                const int rows_valid = min(64, op.M);
-                const uint32_t t_row = tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
-                const int n0 = u.tile * op.bn;
-                if (op.splits == 1) {
-                    for (int c0 = 0; c0 < op.bn; c0 += 32) {
+                // peers have finished reading this CTA's previous partial
+                // (one thread waits; the barrier orders the others after its acquire)
+                if (!bar_epi_and(e != 0 || free_expected == 0 ||
+                                 wait_smem_counter(red_free_addr, free_expected, abort_flag, P.status)))
+                    goto done_e;
+                // TMEM -> shared memory (rows_valid rows, all bn columns)
+                if (q * 32 < rows_valid) {
+                    const uint32_t t_row =
+                        tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
+                    for (int cc = 0; cc < op.bn; cc += 32) {
                         uint32_t rg[32];
-                        tmem_ld_32x32b_x32(t_row + c0, rg);
+                        tmem_ld_32x32b_x32(t_row + cc, rg);
                         tmem_ld_wait();
                         if (row < rows_valid) {
-                            float v[32];
-#pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(rg[t]);
-                            epilogue_chunk(op, row, n0 + c0, v);
-                        }
-                    }
-                    tc_fence_before();
-                    bar_epi();
-                    if (e == 0) {
-                        mbar_arrive(bar_acce + 8 * b);
-                        __threadfence();
-                        atomicAdd(P.done + i, 1u);
-                        stamp(i, 6);
-                    }
-                } else {
-                    // member: wait until the previous partial in `red` has been read, then write
-                    if (!bar_epi_and(wait_smem_counter(red_free_addr, member_uses, abort_flag, P.status))) goto done_e;
-                    float *red = reinterpret_cast<float *>(smem + kOffRed);
-                    for (int c0 = 0; c0 < op.bn; c0 += 32) {
-                        uint32_t rg[32];
-                        tmem_ld_32x32b_x32(t_row + c0, rg);
-                        tmem_ld_wait();
-                        if (row < rows_valid) {
-                            float4 *dst = reinterpret_cast<float4 *>(red + row * kRedLd + c0);
+                            float4 *dst = reinterpret_cast<float4 *>(red + row * kRedLd + cc);
 #pragma unroll
                             for (int j = 0; j < 8; ++j)
                                 dst[j] = make_float4(__uint_as_float(rg[4 * j]), __uint_as_float(rg[4 * j + 1]),
                                                      __uint_as_float(rg[4 * j + 2]), __uint_as_float(rg[4 * j + 3]));
                         }
                     }
-                    tc_fence_before();
-                    bar_epi();
-                    if (e == 0) {
-                        mbar_arrive(bar_acce + 8 * b);
-                        red_add_release_cluster(mapa_shared(red_in_addr, static_cast<uint32_t>(u.owner_rank)), 1u);
-                    }
-                    ++member_uses;
-                    if (u.split == 0) {
-                        // owner: add the S partials of the group in split order, run the epilogue
-                        ++owner_uses;
-                        if (!bar_epi_and(wait_smem_counter(red_in_addr, owner_uses * static_cast<unsigned>(op.splits), abort_flag, P.status)))
-                            goto done_e;
-                        if (e == 0) stamp(i, 5);
-                        const int chunks = op.bn / 32;
-                        for (int item = e;; item += 128) {
-                            const int i_row = item / chunks, ch = item % chunks;
-                            if (i_row >= rows_valid) break;
-                            const uint32_t local = smem_u32(red + i_row * kRedLd + ch * 32);
-                            float v[32];
-#pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] = 0.0f;
-                            for (int sp = 0; sp < op.splits; ++sp) {
-                                const uint32_t src = mapa_shared(local, static_cast<uint32_t>(u.owner_rank + sp));
-                                float4 w4[8];
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) w4[j] = ld_dsmem_f4(src + 16 * j);
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) {
-                                    v[4 * j] = __fadd_rn(v[4 * j], w4[j].x);
-                                    v[4 * j + 1] = __fadd_rn(v[4 * j + 1], w4[j].y);
-                                    v[4 * j + 2] = __fadd_rn(v[4 * j + 2], w4[j].z);
-                                    v[4 * j + 3] = __fadd_rn(v[4 * j + 3], w4[j].w);
-                                }
-                            }
-                            epilogue_chunk(op, i_row, n0 + ch * 32, v);
-                        }
-                        bar_epi();
-                        if (e == 0) {
-                            for (int sp = 0; sp < op.splits; ++sp)
-                                red_add_release_cluster(
-                                    mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
-                            __threadfence();
-                            atomicAdd(P.done + i, 1u);
-                            stamp(i, 6);
-                        }
-                    }
                 }
+                tc_fence_before();
+                bar_epi();
+                if (e == 0) {
+                    mbar_arrive(bar_acce + 8 * b);  // the accumulator is free again
+                    stamp(i, 7);
+                }
+                if (S > 1) {
+                    if (e == 0)
+                        for (int sp = 0; sp < S; ++sp)
+                            red_add_release_cluster(mapa_shared(red_in_addr, static_cast<uint32_t>(u.owner_rank + sp)),
+                                                    1u);
+                    in_expected += static_cast<unsigned>(S);
+                    if (!bar_epi_and(e != 0 || wait_smem_counter(red_in_addr, in_expected, abort_flag, P.status)))
+                        goto done_e;
+                    if (e == 0) stamp(i, 5);
+                }
+                for (int item = e;; item += 128) {
+                    const int i_row = item / chunks, ch = item % chunks;
+                    if (i_row >= rows_valid) break;
+                    const int col = c0 + 32 * ch;
+                    float v[32];
+                    if (S == 1) {
+                        const float4 *src4 = reinterpret_cast<const float4 *>(red + i_row * kRedLd + col);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 w = src4[j];
+                            v[4 * j] = w.x;
+                            v[4 * j + 1] = w.y;
+                            v[4 * j + 2] = w.z;
+                            v[4 * j + 3] = w.w;
+                        }
+                    } else {
+                        const uint32_t local = smem_u32(red + i_row * kRedLd + col);
+                        uint32_t src[4];
+#pragma unroll
+                        for (int sp = 0; sp < 4; ++sp)
+                            src[sp] = mapa_shared(local, static_cast<uint32_t>(u.owner_rank + (sp < S ? sp : 0)));
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] = 0.0f;
+                        // 16 columns at a time: every partial's loads are in flight together
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            float4 w4[4][4];
+#pragma unroll
+                            for (int sp = 0; sp < 4; ++sp)
+                                if (sp < S)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) w4[sp][j] = ld_dsmem_f4(src[sp] + 64 * h + 16 * j);
+#pragma unroll
+                            for (int sp = 0; sp < 4; ++sp)
+                                if (sp < S)
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        float *vv = v + 16 * h + 4 * j;
+                                        vv[0] = __fadd_rn(vv[0], w4[sp][j].x);
+                                        vv[1] = __fadd_rn(vv[1], w4[sp][j].y);
+                                        vv[2] = __fadd_rn(vv[2], w4[sp][j].z);
+                                        vv[3] = __fadd_rn(vv[3], w4[sp][j].w);
+                                    }
+                        }
+                    }
+                    epilogue_chunk_src(op, i_row, n0 + col, v, has_bias ? stg_bias + 32 * ch : nullptr,
+                                       has_res ? stg + i_row * kStgLd + 32 * ch : nullptr);
+                }
+                bar_epi();
+                if (e == 0) {
+                    if (S > 1)
+                        for (int sp = 0; sp < S; ++sp)
+                            red_add_release_cluster(
+                                mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
+                    __threadfence();
+                    atomicAdd(P.done + i, 1u);
+                    stamp(i, 6);
+                }
+                if (S > 1) free_expected += static_cast<unsigned>(S);
                 ++unit_idx;
             }
         }

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdlib>
+#include <type_traits>
 #include <cuda_runtime.h>
 
 #include "epilogue.cuh"
@@ -78,18 +79,13 @@ struct Smem {
     static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
     // split-K partial tile for the cluster reduction, reusing the stage buffers
     static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
-    static_assert((SMALL_A ? 64 : 128) * kRedLd * 4 <= kOffBar, "reduction tile must fit the stages");
+    // owner slots of the cluster split-K reduction: S x ceil(rows / S) rows, S <= 8
+    static_assert(((SMALL_A ? 64 : 128) + 8) * kRedLd * 4 <= kOffBar, "reduction slots must fit the stages");
     static_assert(Cfg<BN>::kBBytes >= 8192, "SMALL_A window overlaps the W tile");
 };
 
 __device__ __forceinline__ void named_barrier_epi() {
     asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t smid_u() {
-    uint32_t s;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(s));
-    return s;
 }
 
 // bounded wait that ignores the abort flag (used while draining before teardown)
@@ -120,8 +116,9 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
-    // diagnostics: [0] globaltimer at entry, [1] smid, [2..6] globaltimer at set-up done /
-    // first stage landed / last MMA issued / accumulator ready / epilogue done
+    // diagnostics (globaltimer ns): [0] entry, [1] split-K epilogue items done, [2] set-up
+    // done, [3] first stage landed, [4] last MMA issued, [5] accumulator ready, [6] exit,
+    // [7] split-K partials visible
     unsigned long long *trace = nullptr;
     if (p.trace != nullptr)
         trace = p.trace + 8ull * ((static_cast<unsigned long long>(blockIdx.z) * gridDim.y + blockIdx.y) *
@@ -153,7 +150,6 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     const uint32_t tmem = misc[0];
     if (trace != nullptr && threadIdx.x == 0) {
         trace[0] = t_entry;
-        trace[1] = smid_u();
         trace[2] = globaltimer_ns();
     }
     // Let the next kernel in the stream start its own weight prefetch.
@@ -276,21 +272,7 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
                     }
                 }
             } else if (p.cluster) {
-                // split-K across the cluster: this CTA's partial tile into its own shared
-                // memory (the stage buffers are free: every load landed and every MMA read it)
-                float *red = reinterpret_cast<float *>(smem);
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(t_row + c0, r);
-                    tmem_ld_wait();
-                    if (row_ok) {
-                        float4 *dst = reinterpret_cast<float4 *>(red + row * S::kRedLd + c0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-                    }
-                }
+                // split-K across the cluster: pushed to the owners after the cluster barrier
             } else {
                 // split-K: partial tile to the workspace, then an arrival ticket
                 float *part = p.partials + (static_cast<size_t>(split) * p.M) * p.N;
@@ -313,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
                 named_barrier_epi();
                 if (misc[2] == static_cast<uint32_t>(p.splits - 1)) {
                     __threadfence();
+                    if (trace != nullptr && threadIdx.x == 64) trace[7] = globaltimer_ns();
                     if (row_ok) {
                         for (int c0 = 0; c0 < BN; c0 += 32) {
                             float v[32];
@@ -340,42 +323,89 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     }
 
     if (p.cluster) {
-        // Deterministic split-K reduction over distributed shared memory: CTA `rank` of the
-        // cluster owns local rows rank, rank + S, ...; for each (row, 32 columns) it adds the S
-        // partials in split order 0..S-1 and runs the epilogue.
-        __syncwarp();
-        cluster_sync_all();  // partial tiles written and visible cluster-wide
-        if (warp >= 2 && misc[3] != 0u) {
-            const int S_ = p.splits;
-            const int rank = static_cast<int>(cluster_ctarank());
-            const int rows_valid = min(SMALL_A ? 64 : 128, p.M - m0);
-            constexpr int kChunks = BN / 32;
-            const float *red = reinterpret_cast<const float *>(smem);
-            for (int item = threadIdx.x - 64;; item += 128) {
-                const int i = rank + (item / kChunks) * S_;
-                const int ch = item % kChunks;
-                if (i >= rows_valid) break;
-                const uint32_t local = smem_u32(red + i * S::kRedLd + ch * 32);
-                float v[32];
+        // Deterministic split-K reduction over distributed shared memory.  CTA `rank` of the
+        // cluster (= its split) owns local rows rank, rank + S, ...  (1) a cluster barrier:
+        // every CTA's MMAs are done with its stage buffers, which now hold partials; (2) every
+        // CTA pushes each of its accumulator rows into slot [split][row / S] of the row's
+        // owner (remote stores, nothing waits on them); (3) a cluster barrier: all partials
+        // landed; (4) all threads of each owner add its rows' S partials from its own shared
+        // memory in split order 0..S-1 and run the epilogue on chunks of W columns (16; 32 for
+        // GeGLU).  Nothing reads a peer after (3).  The bias and residual of each thread's
+        // first chunk are loaded before (1).
+        const int S_ = p.splits;
+        const int rank = static_cast<int>(cluster_ctarank());
+        const int rows_valid = min(SMALL_A ? 64 : 128, p.M - m0);
+        const int R = (rows_valid + S_ - 1) / S_;  // rows per owner
+        float *part = reinterpret_cast<float *>(smem);
+        if (warp < 2) pdl_wait();  // the residual may come from the previous kernel
+        auto reduce = [&](auto width) {
+            constexpr int W = decltype(width)::value;
+            constexpr int kChunks = BN / W;
+            const int e = threadIdx.x;
+            const int i0 = rank + (e / kChunks) * S_, ch0 = e % kChunks;
+            uint32_t bw0[W / 2], rw0[W / 2];
+            const bool has_bias = p.bias != nullptr, has_res = p.residual != nullptr;
+            if (i0 < rows_valid) {
+                if (has_bias) load_bf16<W>(p.bias + n0 + ch0 * W, bw0);
+                if (has_res) load_bf16<W>(p.residual + static_cast<size_t>(m0 + i0) * p.ldr + n0 + ch0 * W, rw0);
+            }
+            __syncwarp();
+            cluster_sync_all();  // (1)
+            if (trace != nullptr && threadIdx.x == 64) trace[7] = globaltimer_ns();
+            const bool acc_ok = misc[3] != 0u;
+            if (warp >= 2 && acc_ok) {
+                const int q = warp & 3;
+                const int row = q * 32 + lane;
+                if (q * 32 < rows_valid) {  // warp-uniform: tcgen05.ld is .sync.aligned
+                    const uint32_t t_row = tmem + (static_cast<uint32_t>(q * 32) << 16);
+                    const uint32_t dst = mapa_shared(smem_u32(part + ((split * R + row / S_) * S::kRedLd)),
+                                                     static_cast<uint32_t>(row % S_));
+                    for (int c0 = 0; c0 < BN; c0 += 32) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(t_row + c0, r);
+                        tmem_ld_wait();
+                        if (row < rows_valid) {
 #pragma unroll
-                for (int t = 0; t < 32; ++t) v[t] = 0.0f;
-                for (int sp = 0; sp < S_; ++sp) {
-                    const uint32_t src = mapa_shared(local, static_cast<uint32_t>(sp));
-                    float4 u[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) u[j] = ld_dsmem_f4(src + 16 * j);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        v[4 * j] = __fadd_rn(v[4 * j], u[j].x);
-                        v[4 * j + 1] = __fadd_rn(v[4 * j + 1], u[j].y);
-                        v[4 * j + 2] = __fadd_rn(v[4 * j + 2], u[j].z);
-                        v[4 * j + 3] = __fadd_rn(v[4 * j + 3], u[j].w);
+                            for (int j = 0; j < 8; ++j)
+                                st_dsmem_f4(dst + 4 * (c0 + 4 * j),
+                                            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+                        }
                     }
                 }
-                epilogue_chunk(p, m0 + i, n0 + ch * 32, v);
             }
-        }
-        cluster_sync_all();  // nobody leaves while a peer still reads its partials
+            __syncwarp();
+            cluster_sync_all();  // (3)
+            if (!acc_ok) return;
+            for (int item = e;; item += kThreads) {
+                const int li = item / kChunks, ch = item % kChunks;
+                const int i = rank + li * S_;
+                if (i >= rows_valid) break;
+                float v[W];
+#pragma unroll
+                for (int t = 0; t < W; ++t) v[t] = 0.0f;
+                for (int sp = 0; sp < S_; ++sp) {
+                    const float4 *src4 = reinterpret_cast<const float4 *>(part + (sp * R + li) * S::kRedLd + ch * W);
+#pragma unroll
+                    for (int j = 0; j < W / 4; ++j) {
+                        const float4 u = src4[j];
+                        v[4 * j] = __fadd_rn(v[4 * j], u.x);
+                        v[4 * j + 1] = __fadd_rn(v[4 * j + 1], u.y);
+                        v[4 * j + 2] = __fadd_rn(v[4 * j + 2], u.z);
+                        v[4 * j + 3] = __fadd_rn(v[4 * j + 3], u.w);
+                    }
+                }
+                if (item == e)
+                    epilogue_chunk_w<W>(p, m0 + i, n0 + ch * W, v, has_bias ? bw0 : nullptr, has_res ? rw0 : nullptr);
+                else
+                    epilogue_chunk<W>(p, m0 + i, n0 + ch * W, v);
+            }
+        };
+        if (p.epi == kEpiGeglu)
+            reduce(std::integral_constant<int, 32>());
+        else
+            reduce(std::integral_constant<int, 16>());
+        if (trace != nullptr && threadIdx.x == 64) trace[1] = globaltimer_ns();
     }
 
     tc_fence_before();

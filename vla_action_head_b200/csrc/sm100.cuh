@@ -206,6 +206,12 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void st_dsmem_f4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
 // Arrives once on an mbarrier in another CTA of the cluster (address from mapa_shared),
 // releasing this thread's prior shared-memory writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
