@@ -77,8 +77,14 @@ static cudaError_t launch_tpr(const NormArgs &a, int bpt, cudaStream_t s) {
 }
 
 // Host entry used by the C ABI.  K % 16 == 0 and the size limits are checked by the caller.
+// Few rows (up to about one per SM): a CTA per row, so each row's reductions are spread
+// over 128 threads and the per-row latency is short.  Many rows: a warp per row.
 cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s) {
     const int nblk = a.K >> 4;
+    if (a.M <= 160 && nblk <= 128 * 8) {
+        const int bpt = (nblk + 127) / 128;
+        return f32_in ? launch_tpr<128, true>(a, bpt, s) : launch_tpr<128, false>(a, bpt, s);
+    }
     if (nblk <= 32 * 8) {
         const int bpt = (nblk + 31) / 32;
         return f32_in ? launch_tpr<32, true>(a, bpt, s) : launch_tpr<32, false>(a, bpt, s);
