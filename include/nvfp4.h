@@ -96,6 +96,10 @@ nvfp4_status nvfp4_probe(void);
 /* Static, never NULL. */
 const char *nvfp4_status_string(nvfp4_status s);
 
+/* The CUDA runtime's message for the last CUDA error behind an NVFP4_ERR_CUDA returned to
+ * this thread ("no error" if there was none).  Static storage; never NULL. */
+const char *nvfp4_last_cuda_error_string(void);
+
 /* Bytes of a scale-factor buffer for rows x K elements: ceil(rows/128)*ceil(K/64)*512. */
 size_t nvfp4_sf_bytes(int rows, int K);
 
@@ -221,7 +225,9 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
  * 256-element K tiles).  splits > 0 reduces the partials inside a cluster when splits <= 8
  * and M <= 128, otherwise through the workspace; splits < 0 always uses the workspace.
  * block_n = 0 with splits = 0 takes the default schedule, with splits = -1 the default
- * workspace-reduced schedule.  Same contract otherwise; the workspace must hold
+ * workspace-reduced schedule.  The default schedule for M > 64 with N % 256 == 0 runs a
+ * persistent kernel (one CTA per SM walks the 128 x 256 output tiles); a pinned schedule
+ * always runs one tile per CTA.  Same contract otherwise; the workspace must hold
  * nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits) bytes. */
 nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
                            nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,

@@ -59,15 +59,21 @@ def _unpack(codes):
     return out
 
 
-def check_fp4_output(orc, gpu_codes, gpu_sf, ref_codes, ref_sf, h_ref, g_out, rows, K, what=""):
+def check_fp4_output(orc, gpu_codes, gpu_sf, ref_codes, ref_sf, h_ref, g_out, rows, K, what="", sel=None):
     """Acceptance of an FP4-output epilogue (tanh-GELU / GeGLU) against the oracle, whose
     activation is fp64 while the kernel's is fp32:
       - scale bytes: equal, or one E4M3 step apart, in <= 1e-3 of the blocks;
       - in blocks with equal scales, code mismatches <= 1e-3 of the elements, each at an
-        oracle value h/S within 2^-10 (relative) of an E2M1 rounding boundary."""
+        oracle value h/S within 2^-10 (relative) of an E2M1 rounding boundary.
+    sel: only these rows of the `rows`-row outputs are compared (h_ref holds just them)."""
     nblk = K // 16
     gs = orc.sf_gather(gpu_sf, rows, K).astype(np.int32)
     rs = orc.sf_gather(ref_sf, rows, K).astype(np.int32)
+    if sel is not None:
+        gs, rs = gs[sel], rs[sel]
+        gpu_codes = np.ascontiguousarray(np.asarray(gpu_codes).reshape(rows, -1)[sel])
+        ref_codes = np.ascontiguousarray(np.asarray(ref_codes).reshape(rows, -1)[sel])
+        rows = len(sel)
     dif = np.abs(gs - rs)
     assert dif.max() <= 1, (what, "scale bytes differ by more than one step")
     assert (dif != 0).mean() <= 1e-3, (what, float((dif != 0).mean()))

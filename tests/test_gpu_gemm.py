@@ -27,13 +27,14 @@ def _operands(orc, wl, M, N, K, inter=False):
     return (ac, asf, 1.0), (wc, wsf, gw)
 
 
-def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0, geglu_bias=False):
+def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0, geglu_bias=False, rows=None):
+    """rows: compare only these output rows (the oracle computes just them)."""
     (ac, asf, ga), (wc, wsf, gw) = _operands(orc, wl, M, N, K)
     uses_bias = epi in ("bias", "bias_residual", "bias_gelu") or (epi == "geglu" and geglu_bias)
     uses_res = epi in ("residual", "bias_residual")
     bias = synth.bf16_normal(synth.seed_of(wl, synth.BIAS0), (N,), 0.0, 0.01) if uses_bias else None
     res = synth.bf16_normal(synth.seed_of(wl, synth.RESIDUAL), (M, N)) if uses_res else None
-    ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res, g_out=g_out)
+    ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res, g_out=g_out, rows=rows)
     A = to_gpu_fp4(ac, asf, ga, M, K)
     W = to_gpu_fp4(wc, wsf, gw, N, K)
     out = nvfp4.gemm(A, W, epi, bias=dev_bf16(bias) if uses_bias else None,
@@ -42,8 +43,9 @@ def _run(orc, M, N, K, epi, bn=0, sp=0, wl=11, g_out=1.0, geglu_bias=False):
     if epi in ("bias_gelu", "geglu"):
         n_out = N // 2 if epi == "geglu" else N
         return check_fp4_output(orc, host(out.codes), host(out.sf), ref["codes"], ref["sf"], ref["h"],
-                                g_out, M, n_out, what=(M, N, K, epi, bn, sp))
-    return check_gemm_bf16(host(out), ref["v"], what=(M, N, K, epi, bn, sp))
+                                g_out, M, n_out, what=(M, N, K, epi, bn, sp), sel=rows)
+    got = host(out) if rows is None else host(out)[rows]
+    return check_gemm_bf16(got, ref["v"], what=(M, N, K, epi, bn, sp))
 
 
 SHAPES = [(41, 512, 256), (1, 64, 64), (7, 192, 96), (50, 256, 1024), (130, 384, 320), (300, 256, 512),
@@ -120,3 +122,20 @@ def test_cluster_and_workspace_reductions_agree(orc):
 
 def test_device_status_clean():
     nvfp4.device_status()
+
+
+# The default schedule for many rows with N % 256 == 0 runs the persistent kernel (one CTA
+# per SM walks the tiles; the scale factors go to TMEM through 128x256b copies of
+# replicated images); explicit (256, 1) runs the one-tile-per-CTA kernel.
+@pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
+def test_persistent_epilogues(orc, epi):
+    _run(orc, 300, 512, 768, epi)
+
+
+def test_persistent_multi_tile_and_tails(orc):
+    """More tiles than SMs (each CTA walks several), the M tail of 968 = 7 * 128 + 72, and
+    a last K tile with an odd number of 64-wide blocks (K = 4160)."""
+    rows = [0, 1, 63, 127, 128, 500, 767, 895, 896, 900, 960, 967]
+    _run(orc, 968, 5120, 1024, "none", rows=rows)
+    _run(orc, 968, 2048, 4160, "residual", rows=rows)
+    _run(orc, 968, 4096, 512, "geglu", rows=rows)

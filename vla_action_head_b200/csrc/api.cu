@@ -43,7 +43,13 @@ nvfp4_status check_device(int *sms = nullptr) {
     return NVFP4_OK;
 }
 
-nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;  // for nvfp4_last_cuda_error_string
+
+nvfp4_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return NVFP4_OK;
+    g_last_cuda_error = e;
+    return NVFP4_ERR_CUDA;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -82,6 +88,16 @@ struct Schedule {
 };
 
 constexpr int kMaxClusterSplits = 8;  // portable cluster size
+
+// Device address of the library's status word on the current device (looked up once).
+uint32_t *status_word() {
+    constexpr int kMaxDevices = 64;
+    static uint32_t *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (addr[dev] == nullptr && device_status_address(&addr[dev]) != cudaSuccess) addr[dev] = nullptr;
+    return addr[dev];
+}
 
 int sm_count_cached() {
     static int sms = 0;
@@ -277,7 +293,11 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if (!make_code_map(&ta, A->codes, M, K / 2, static_cast<int>(p.a_box_rows)) ||
         !make_code_map(&tb, W->codes, N, K / 2, sc.block_n))
         return NVFP4_ERR_CUDA;
-    cudaError_t e = launch_gemm(ta, tb, p, sc.block_n, stream);
+    // default schedule for many rows (256-wide tiles, no split): the persistent kernel; an
+    // explicit (block_n, splits) request runs the one-tile-per-CTA kernel
+    const bool persistent = block_n == 0 && splits == 0 && sc.block_n == 256 && sc.splits == 1 && p.a_box_rows == 128;
+    if (persistent && (p.status = status_word()) == nullptr) return NVFP4_ERR_CUDA;
+    cudaError_t e = persistent ? launch_gemm_persistent(ta, tb, p, stream) : launch_gemm(ta, tb, p, sc.block_n, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return from_cuda(e);
 }
@@ -331,12 +351,15 @@ nvfp4_status nvfp4_probe(void) {
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
     // the kernels of this library must load on the device
-    if (probe_norm_kernels() != cudaSuccess || probe_gemm_kernels() != cudaSuccess) {
+    if (probe_norm_kernels() != cudaSuccess || probe_gemm_kernels() != cudaSuccess ||
+        probe_gemm_persistent() != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
     }
     return encode_fn() != nullptr ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
+
+const char *nvfp4_last_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char *nvfp4_status_string(nvfp4_status s) {
     switch (s) {

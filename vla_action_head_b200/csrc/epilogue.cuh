@@ -35,11 +35,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // as W / 2 words of bf16 pairs each (NULL: none), already loaded.
 // Every field of p is read once into a local first: the byte stores of the FP4 outputs may
 // alias any memory as far as the compiler knows, and p may live in global memory.
-template <int W, class P>
+// EPI >= 0 fixes the epilogue kind at compile time (only that path is generated).
+template <int W, int EPI = -1, class P>
 __device__ __forceinline__ void epilogue_chunk_w(const P &p, int m, int n, float *v, const uint32_t *bw,
                                                  const uint32_t *rw) {
     static_assert(W == 16 || W == 32, "chunk width");
-    const int epi = p.epi, N = p.N, ldo = p.ldo;
+    const int epi = EPI >= 0 ? EPI : p.epi;
+    const int N = p.N, ldo = p.ldo;
     const float alpha = p.alpha, g_out = p.g_out;
     uint16_t *const out = p.out;
     uint8_t *const out_codes = p.out_codes;
@@ -116,21 +118,23 @@ __device__ __forceinline__ void load_bf16(const uint16_t *src, uint32_t *w) {
 
 // The same, with bias_n / res_mn pointing to the bias of columns n.. and the residual of
 // row m, columns n.. (global or shared memory; NULL: none).
-template <int W = 32, class P>
+template <int W = 32, int EPI = -1, class P>
 __device__ __forceinline__ void epilogue_chunk_src(const P &p, int m, int n, float *v, const uint16_t *bias_n,
                                                    const uint16_t *res_mn) {
     uint32_t bw[W / 2], rw[W / 2];
     if (bias_n != nullptr) load_bf16<W>(bias_n, bw);
     if (res_mn != nullptr) load_bf16<W>(res_mn, rw);
-    epilogue_chunk_w<W>(p, m, n, v, bias_n != nullptr ? bw : nullptr, res_mn != nullptr ? rw : nullptr);
+    epilogue_chunk_w<W, EPI>(p, m, n, v, bias_n != nullptr ? bw : nullptr, res_mn != nullptr ? rw : nullptr);
 }
 
 // The same, reading bias and residual from the arguments' global pointers.
-template <int W = 32, class P>
+template <int W = 32, int EPI = -1, class P>
 __device__ __forceinline__ void epilogue_chunk(const P &p, int m, int n, float *v) {
-    const uint16_t *const bias = p.bias;
-    const uint16_t *const residual = p.residual;
-    epilogue_chunk_src<W>(p, m, n, v, bias != nullptr ? bias + n : nullptr,
+    const int epi = EPI >= 0 ? EPI : p.epi;
+    const uint16_t *const bias =
+        (epi == kEpiBias || epi == kEpiBiasResidual || epi == kEpiBiasGelu || epi == kEpiGeglu) ? p.bias : nullptr;
+    const uint16_t *const residual = (epi == kEpiResidual || epi == kEpiBiasResidual) ? p.residual : nullptr;
+    epilogue_chunk_src<W, EPI>(p, m, n, v, bias != nullptr ? bias + n : nullptr,
                        residual != nullptr ? residual + static_cast<size_t>(m) * p.ldr + n : nullptr);
 }
 

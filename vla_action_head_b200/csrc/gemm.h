@@ -35,10 +35,17 @@ struct GemmArgs {
     float *partials;    // split-K: [splits, M, N] fp32
     uint32_t *tickets;  // split-K: one word per output tile
     unsigned long long *trace;  // optional per-CTA timestamps (diagnostics), 8 words per CTA
+    uint32_t *status;           // the library's device status word (persistent kernel)
 };
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s);
+
+// Persistent 128 x 256-tile kernel for many rows (gemm_persistent.cu): N % 256 == 0, one
+// split.  Grid: min(tiles, SMs) CTAs.
+int gemm_persistent_grid(int M, int n_tiles);
+cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s);
+cudaError_t probe_gemm_persistent();
 
 // Device address and size of the library-owned split-K workspace used by
 // nvfp4_gemm_noalloc (looked up once per device; allocation-free).

@@ -1,0 +1,323 @@
+// gemm_persistent.cu — block-scaled NVFP4 GEMM for many rows (the compute-bound regime,
+// e.g. a prefill layer at M = 968), as a persistent kernel: one CTA per SM walks 128 x 256
+// output tiles, m-tile fastest, so the 8 CTAs that share a weight tile read it close together
+// and it is fetched from HBM once (the activations stay in L2).
+//
+//   acc[m, n] = sum_k e(A)[m, k] sA[m, k/16] e(W)[n, k] sW[n, k/16]      (fp32, in TMEM)
+//   v = acc * gA * gW (+ bias[n]) (+ residual[m, n])  ->  bf16, or tanh-GELU / GeGLU -> FP4
+// ("GROOT N1.7 update: Thor NVFP4 + FA4 performance tier", §What is in the tier;
+// "Pi0.5 Thor NVFP4 End-to-End Results", §Fused GeGLU FFN in the Decoder.)
+//
+// Roles (320 threads):
+//   warp 0      producer: TMA loads of the A (128 rows) and W (256 rows) code tiles and bulk
+//               loads of their scale atoms into a 4-stage ring; the weights of the first
+//               stages are issued before the programmatic-launch wait.
+//   warp 1      MMA issuer: tcgen05.cp (32x128b.warpx4) of the scale atoms, then 4 x
+//               tcgen05.mma kind::mxf4nvf4 block16 (M = 128, N = 256, K = 64) per 256-wide K tile.
+//   warps 2..9  epilogue: two warps per TMEM sub-partition, each draining 128 of the 256
+//               accumulator columns of its 32 rows into registers; the accumulator is handed
+//               back to the MMA warp right after the drain, so the fused epilogue of one tile
+//               runs while the next tile's MMAs do.  The kernel is instantiated per epilogue
+//               kind, so each instance holds one path (and fits its registers without spills).
+//
+// The scale-copy instructions (3 per 64-wide K step, one MMA each) bound the issue rate of
+// the MMA warp.  Copying two atoms per tcgen05.cp.128x256b needs each atom 4 times in
+// shared memory; building those images (with 48 small bulk copies per stage, or with a warp
+// of loads and stores) measured slower than the plain copies, so the kernel keeps them.
+//
+// Every wait is bounded (sm100.cuh); an expired wait records a status and the CTA unwinds.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "epilogue.cuh"
+#include "gemm.h"
+#include "sm100.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kSfAtom = 512;
+constexpr int kStageA = 128 * 128;                // 128 rows x 256 FP4
+constexpr int kStageB = kBN * 128;                // 256 rows x 256 FP4
+constexpr int kStageSfa = 4 * kSfAtom;            // A atoms of the 4 k-blocks
+constexpr int kStageSfb = 8 * kSfAtom;            // W atoms: 2 row groups x 4 k-blocks
+constexpr int kOffB = kStageA;
+constexpr int kOffSfa = kOffB + kStageB;
+constexpr int kOffSfb = kOffSfa + kStageSfa;
+constexpr int kStage = kOffSfb + kStageSfb;       // 54 KB, a multiple of 1024
+constexpr int kOffBar = kStages * kStage;
+// barriers: full[kStages], empty[kStages], acc_full, acc_empty
+constexpr int kOffMisc = kOffBar + (2 * kStages + 2) * 8;
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr int kTmemCols = 512;
+constexpr int kColSfa = kBN;       // 16 columns: 4 k-blocks x 4
+constexpr int kColSfb = kBN + 16;  // 32 columns: 4 k-blocks x (2 row groups x 4)
+static_assert(kStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+// Barrier of the 256 epilogue threads that also ANDs a flag across them (every decision to
+// abandon the work is taken by all eight warps together).
+__device__ __forceinline__ bool bar_epi_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v))
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32_t *status) {
+    int dummy = 0;
+    return mbar_wait(bar, parity, &dummy, status, kStatusTimeoutDrain);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + kOffBar;
+    const uint32_t bar_empty = bar_full + 8 * kStages;
+    const uint32_t bar_accf = bar_empty + 8 * kStages;
+    const uint32_t bar_acce = bar_accf + 8;
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);  // [0] TMEM base, [1] abort
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tiles = (p.M + 127) / 128;
+    const int tiles = m_tiles * p.n_tiles;
+    const int k_tiles = p.k_tiles;
+    const int my_tiles = static_cast<int>(blockIdx.x) < tiles ? (tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+    const int steps = my_tiles * k_tiles;
+    unsigned long long *trace = p.trace != nullptr ? p.trace + 8ull * blockIdx.x : nullptr;
+    if (trace != nullptr && threadIdx.x == 0) trace[0] = globaltimer_ns();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_accf, 1);
+        mbar_init(bar_acce, 1);
+        misc[1] = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(const_cast<uint32_t *>(misc)), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    pdl_launch_dependents();
+
+    auto nkb_of = [&](int kt) { return min(4, p.k_atoms - 4 * kt); };
+    auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
+
+    if (warp == 0) {
+        // ------------------------------ producer (whole warp) ------------------------------
+        const uint64_t pol = policy_evict_last();  // A and W both fit in L2 and are re-read
+        auto expect = [&](int st) {
+            const int nkb = nkb_of(st % k_tiles);
+            const uint32_t bytes = kStageA + kStageB + static_cast<uint32_t>(nkb) * 3u * kSfAtom;
+            if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * (st % kStages), bytes);
+            __syncwarp();
+        };
+        auto issue_w = [&](int st) {
+            const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
+            const int n_tile = t / m_tiles, nkb = nkb_of(kt);
+            const uint32_t full = bar_full + 8 * s, base = sbase + s * kStage;
+            if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * kBN, full, pol);
+            if (lane < 2) {  // the k-blocks' atoms of each 128-row group are contiguous
+                const size_t grp = static_cast<size_t>(n_tile) * 2 + lane;
+                bulk_load(base + kOffSfb + lane * 4 * kSfAtom, p.sfb + (grp * p.k_atoms + 4 * kt) * kSfAtom,
+                          static_cast<uint32_t>(nkb) * kSfAtom, full, pol);
+            }
+        };
+        auto issue_a = [&](int st) {
+            const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
+            const int m_tile = t % m_tiles, nkb = nkb_of(kt);
+            const uint32_t full = bar_full + 8 * s, base = sbase + s * kStage;
+            if (lane == 0) {
+                tma_load_2d(base, &tmA, kt * 128, m_tile * 128, full, pol);
+                bulk_load(base + kOffSfa, p.sfa + (static_cast<size_t>(m_tile) * p.k_atoms + 4 * kt) * kSfAtom,
+                          static_cast<uint32_t>(nkb) * kSfAtom, full, pol);
+            }
+        };
+        const int pre = min(kStages, steps);
+        for (int st = 0; st < pre; ++st) {
+            expect(st);
+            issue_w(st);
+        }
+        pdl_wait();  // A and its scales come from the previous kernel
+        for (int st = 0; st < pre; ++st) issue_a(st);
+        int issued = pre;
+        for (int st = pre; st < steps; ++st) {
+            const int s = st % kStages, use = st / kStages;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(bar_empty + 8 * s, (use - 1) & 1, abort_flag, p.status, kStatusTimeoutEmpty);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            expect(st);
+            issue_w(st);
+            issue_a(st);
+            issued = st + 1;
+        }
+        // every issued stage must have landed before the CTA may exit
+        if (lane == 0)
+            for (int st = max(0, issued - kStages); st < issued; ++st)
+                drain_wait(bar_full + 8 * (st % kStages), (st / kStages) & 1, p.status);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------ MMA issuer ------------------------------
+            constexpr uint32_t idesc = idesc_mxf4nvf4(128, kBN);
+            int st = 0;
+            for (int i = 0; i < my_tiles; ++i) {
+                if (i > 0 && !mbar_wait(bar_acce, (i - 1) & 1, abort_flag, p.status, kStatusTimeoutAccum))
+                    break;
+                tc_fence_after();
+                bool ok = true;
+                for (int kt = 0; kt < k_tiles; ++kt, ++st) {
+                    const int s = st % kStages;
+                    if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nkb = nkb_of(kt);
+                    const uint32_t base = sbase + s * kStage;
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * kb, desc_sf_32x128b(base + kOffSfa + kb * kSfAtom));
+#pragma unroll
+                        for (int g = 0; g < 2; ++g)
+                            tc_cp_32x128b_warpx4(tmem + kColSfb + 8 * kb + 4 * g,
+                                                 desc_sf_32x128b(base + kOffSfb + g * 4 * kSfAtom + kb * kSfAtom));
+                    }
+                    for (int kb = 0; kb < nkb; ++kb)
+                        tc_mma_mxf4nvf4(tmem, desc_kmajor_sw128(base + 32 * kb), desc_kmajor_sw128(base + kOffB + 32 * kb),
+                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 8 * kb,
+                                        (kt > 0 || kb > 0) ? 1u : 0u);
+                    tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs have read it
+                }
+                tc_commit(bar_accf);  // always: completion of every MMA issued above
+                if (!ok) break;
+            }
+        }
+    } else {
+        // ------------------------------ epilogue (warps 2..9) ------------------------------
+        const int q = warp & 3;            // TMEM sub-partition this warp may read
+        const int half = (warp - 2) >> 2;  // which 128 of the 256 columns
+        const int row = q * 32 + lane;
+        const int e = threadIdx.x - 64;
+        pdl_wait();  // residuals may come from the previous kernel
+        for (int i = 0; i < my_tiles; ++i) {
+            const int t = tile_of(i);
+            const int m_tile = t % m_tiles, n_tile = t / m_tiles;
+            const bool got =
+                e != 0 || mbar_wait(bar_accf, i & 1, abort_flag, p.status, kStatusTimeoutAccum);
+            if (!bar_epi_and(got && *abort_flag == 0)) break;
+            tc_fence_after();
+            uint32_t r[4][32];
+            const uint32_t t_row =
+                tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * 128);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
+            tmem_ld_wait();
+            tc_fence_before();
+            bar_epi_and(true);
+            if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
+            const int m = m_tile * 128 + row;
+            if (m < p.M) {
+                const int n = n_tile * kBN + half * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
+                    epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
+                }
+            }
+        }
+    }
+
+    // teardown
+    __syncwarp();
+    if (*abort_flag) {
+        // an abandoned run may leave copies or MMAs in flight: give them time to land before
+        // shared and tensor memory are released
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (trace != nullptr && threadIdx.x == 0) trace[6] = globaltimer_ns();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+int gemm_persistent_grid(int M, int n_tiles) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    const int tiles = ((M + 127) / 128) * n_tiles;
+    return tiles < sms ? tiles : sms;
+}
+
+template <int EPI>
+static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e =
+            cudaFuncSetAttribute(gemm_persistent_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gemm_persistent_grid(p.M, p.n_tiles));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<EPI>, ta, tb, p);
+}
+
+cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+    switch (p.epi) {
+    case kEpiNone: return launch_epi<kEpiNone>(ta, tb, p, s);
+    case kEpiBias: return launch_epi<kEpiBias>(ta, tb, p, s);
+    case kEpiResidual: return launch_epi<kEpiResidual>(ta, tb, p, s);
+    case kEpiBiasResidual: return launch_epi<kEpiBiasResidual>(ta, tb, p, s);
+    case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(ta, tb, p, s);
+    case kEpiGeglu: return launch_epi<kEpiGeglu>(ta, tb, p, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t probe_gemm_persistent() {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, gemm_persistent_kernel<kEpiNone>);
+}
+
+}  // namespace nvfp4

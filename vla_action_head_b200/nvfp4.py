@@ -26,8 +26,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned
 
 
 class NVFP4Error(RuntimeError):
-    def __init__(self, call, status):
-        super().__init__(f"{call} failed: {status} ({STATUS.get(status, '?')})")
+    def __init__(self, call, status, detail=""):
+        super().__init__(f"{call} failed: {status} ({STATUS.get(status, '?')}){detail}")
         self.status = status
 
 
@@ -67,6 +67,7 @@ def lib():
         sig = {
             "nvfp4_probe": (I, []),
             "nvfp4_status_string": (C.c_char_p, [I]),
+            "nvfp4_last_cuda_error_string": (C.c_char_p, []),
             "nvfp4_sf_bytes": (SZ, [I, I]),
             "nvfp4_sf_offset": (SZ, [I, I, I]),
             "nvfp4_sf_zero": (I, [P, I, I, P]),
@@ -103,7 +104,10 @@ def header_functions():
 
 def _check(call, st):
     if st != 0:
-        raise NVFP4Error(call, st)
+        detail = ""
+        if STATUS.get(st) == "CUDA error":
+            detail = ": " + lib().nvfp4_last_cuda_error_string().decode()
+        raise NVFP4Error(call, st, detail)
 
 
 # ---- torch-facing helpers ---------------------------------------------------------------
