@@ -225,9 +225,9 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
  * 256-element K tiles).  splits > 0 reduces the partials inside a cluster when splits <= 8
  * and M <= 128, otherwise through the workspace; splits < 0 always uses the workspace.
  * block_n = 0 with splits = 0 takes the default schedule, with splits = -1 the default
- * workspace-reduced schedule.  The default schedule for M > 64 with N % 256 == 0 runs a
- * persistent kernel (one CTA per SM walks the 128 x 256 output tiles); a pinned schedule
- * always runs one tile per CTA.  Same contract otherwise; the workspace must hold
+ * workspace-reduced schedule.  The default schedule for M > 128 with N % 128 == 0 runs a
+ * persistent kernel (one CTA per SM walks 128 x 256 or 128 x 128 output tiles); a pinned
+ * schedule always runs one tile per CTA.  Same contract otherwise; the workspace must hold
  * nvfp4_gemm_workspace_bytes_ex(M, N, K, block_n, splits) bytes. */
 nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
                            nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,

@@ -128,8 +128,10 @@ def test_device_status_clean():
 # per SM walks the tiles; the scale factors go to TMEM through 128x256b copies of
 # replicated images); explicit (256, 1) runs the one-tile-per-CTA kernel.
 @pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
-def test_persistent_epilogues(orc, epi):
-    _run(orc, 300, 512, 768, epi)
+@pytest.mark.parametrize("N,rows", [(512, None), (10240, [0, 5, 127, 128, 255, 256, 299])])
+def test_persistent_epilogues(orc, epi, N, rows):
+    """N = 512 runs 128-wide tiles (12 of them); N = 10240 runs 256-wide ones (120)."""
+    _run(orc, 300, N, 768, epi, rows=rows)
 
 
 def test_persistent_multi_tile_and_tails(orc):

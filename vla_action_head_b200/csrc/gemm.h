@@ -41,10 +41,11 @@ struct GemmArgs {
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s);
 
-// Persistent 128 x 256-tile kernel for many rows (gemm_persistent.cu): N % 256 == 0, one
-// split.  Grid: min(tiles, SMs) CTAs.
+// Persistent 128 x block_n tile kernel for many rows (gemm_persistent.cu): block_n 256 or
+// 128, one split.  Grid: min(tiles, SMs) CTAs.
 int gemm_persistent_grid(int M, int n_tiles);
-cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s);
+cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
+                                   cudaStream_t s);
 cudaError_t probe_gemm_persistent();
 
 // Device address and size of the library-owned split-K workspace used by

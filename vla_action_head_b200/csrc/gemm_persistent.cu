@@ -37,27 +37,34 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kBN = 256;
-constexpr int kStages = 4;
 constexpr int kThreads = 320;
 constexpr int kSfAtom = 512;
-constexpr int kStageA = 128 * 128;                // 128 rows x 256 FP4
-constexpr int kStageB = kBN * 128;                // 256 rows x 256 FP4
-constexpr int kStageSfa = 4 * kSfAtom;            // A atoms of the 4 k-blocks
-constexpr int kStageSfb = 8 * kSfAtom;            // W atoms: 2 row groups x 4 k-blocks
-constexpr int kOffB = kStageA;
-constexpr int kOffSfa = kOffB + kStageB;
-constexpr int kOffSfb = kOffSfa + kStageSfa;
-constexpr int kStage = kOffSfb + kStageSfb;       // 54 KB, a multiple of 1024
-constexpr int kOffBar = kStages * kStage;
-// barriers: full[kStages], empty[kStages], acc_full, acc_empty
-constexpr int kOffMisc = kOffBar + (2 * kStages + 2) * 8;
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-constexpr int kTmemCols = 512;
-constexpr int kColSfa = kBN;       // 16 columns: 4 k-blocks x 4
-constexpr int kColSfb = kBN + 16;  // 32 columns: 4 k-blocks x (2 row groups x 4)
-static_assert(kStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+// Shared-memory and TMEM plan for a tile width BN (256, or 128 when 256-wide tiles would
+// leave SMs idle): as many stages of [A 128 x 256 FP4 | W BN x 256 FP4 | A scale atoms of
+// the 4 k-blocks | W scale atoms, per 128-row group] as fit in 216 KB.
+template <int BN>
+struct PCfg {
+    static constexpr int kGroups = BN / 128;  // 128-row scale groups of a W tile
+    static constexpr int kStageA = 128 * 128;
+    static constexpr int kStageB = BN * 128;
+    static constexpr int kStageSfa = 4 * kSfAtom;
+    static constexpr int kStageSfb = kGroups * 4 * kSfAtom;
+    static constexpr int kOffB = kStageA;
+    static constexpr int kOffSfa = kOffB + kStageB;
+    static constexpr int kOffSfb = kOffSfa + kStageSfa;
+    static constexpr int kStage = kOffSfb + kStageSfb;  // 54 KB (BN 256) / 36 KB (BN 128)
+    static constexpr int kStages = (216 * 1024) / kStage;
+    static constexpr int kOffBar = kStages * kStage;
+    // barriers: full[kStages], empty[kStages], acc_full, acc_empty
+    static constexpr int kOffMisc = kOffBar + (2 * kStages + 2) * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    static constexpr int kColSfa = BN;                        // 16 columns: 4 k-blocks x 4
+    static constexpr int kColSfb = BN + 16;                   // 4 k-blocks x (groups x 4)
+    static constexpr int kTmemCols = (kColSfb + 16 * kGroups) <= 256 ? 256 : 512;
+    static_assert(kStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
 
 // Barrier of the 256 epilogue threads that also ANDs a flag across them (every decision to
 // abandon the work is taken by all eight warps together).
@@ -79,18 +86,22 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32
     return mbar_wait(bar, parity, &dummy, status, kStatusTimeoutDrain);
 }
 
-template <int EPI>
+template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const GemmArgs p) {
+    using Cf = PCfg<BN>;
+    constexpr int kStages = Cf::kStages, kStage = Cf::kStage, kStageA = Cf::kStageA, kStageB = Cf::kStageB;
+    constexpr int kOffB = Cf::kOffB, kOffSfa = Cf::kOffSfa, kOffSfb = Cf::kOffSfb, kGroups = Cf::kGroups;
+    constexpr int kColSfa = Cf::kColSfa, kColSfb = Cf::kColSfb, kTmemCols = Cf::kTmemCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar_full = sbase + kOffBar;
+    const uint32_t bar_full = sbase + Cf::kOffBar;
     const uint32_t bar_empty = bar_full + 8 * kStages;
     const uint32_t bar_accf = bar_empty + 8 * kStages;
     const uint32_t bar_acce = bar_accf + 8;
-    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);  // [0] TMEM base, [1] abort
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + Cf::kOffMisc);  // [0] TMEM base, [1] abort
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t pol = policy_evict_last();  // A and W both fit in L2 and are re-read
         auto expect = [&](int st) {
             const int nkb = nkb_of(st % k_tiles);
-            const uint32_t bytes = kStageA + kStageB + static_cast<uint32_t>(nkb) * 3u * kSfAtom;
+            const uint32_t bytes = kStageA + kStageB + static_cast<uint32_t>(nkb) * (1u + kGroups) * kSfAtom;
             if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * (st % kStages), bytes);
             __syncwarp();
         };
@@ -140,9 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
             const int n_tile = t / m_tiles, nkb = nkb_of(kt);
             const uint32_t full = bar_full + 8 * s, base = sbase + s * kStage;
-            if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * kBN, full, pol);
-            if (lane < 2) {  // the k-blocks' atoms of each 128-row group are contiguous
-                const size_t grp = static_cast<size_t>(n_tile) * 2 + lane;
+            if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * BN, full, pol);
+            if (lane < kGroups) {  // the k-blocks' atoms of each 128-row group are contiguous
+                const size_t grp = static_cast<size_t>(n_tile) * kGroups + lane;
                 bulk_load(base + kOffSfb + lane * 4 * kSfAtom, p.sfb + (grp * p.k_atoms + 4 * kt) * kSfAtom,
                           static_cast<uint32_t>(nkb) * kSfAtom, full, pol);
             }
@@ -183,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------ MMA issuer ------------------------------
-            constexpr uint32_t idesc = idesc_mxf4nvf4(128, kBN);
+            constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
             int st = 0;
             for (int i = 0; i < my_tiles; ++i) {
                 if (i > 0 && !mbar_wait(bar_acce, (i - 1) & 1, abort_flag, p.status, kStatusTimeoutAccum))
@@ -202,13 +213,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kb = 0; kb < nkb; ++kb) {
                         tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * kb, desc_sf_32x128b(base + kOffSfa + kb * kSfAtom));
 #pragma unroll
-                        for (int g = 0; g < 2; ++g)
-                            tc_cp_32x128b_warpx4(tmem + kColSfb + 8 * kb + 4 * g,
+                        for (int g = 0; g < kGroups; ++g)
+                            tc_cp_32x128b_warpx4(tmem + kColSfb + 4 * kGroups * kb + 4 * g,
                                                  desc_sf_32x128b(base + kOffSfb + g * 4 * kSfAtom + kb * kSfAtom));
                     }
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_mxf4nvf4(tmem, desc_kmajor_sw128(base + 32 * kb), desc_kmajor_sw128(base + kOffB + 32 * kb),
-                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 8 * kb,
+                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 4 * kGroups * kb,
                                         (kt > 0 || kb > 0) ? 1u : 0u);
                     tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs have read it
                 }
@@ -219,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------ epilogue (warps 2..9) ------------------------------
         const int q = warp & 3;            // TMEM sub-partition this warp may read
-        const int half = (warp - 2) >> 2;  // which 128 of the 256 columns
+        const int half = (warp - 2) >> 2;  // which half of the BN columns
+        constexpr int kChunks = BN / 64;   // 32-column chunks per thread
         const int row = q * 32 + lane;
         const int e = threadIdx.x - 64;
         pdl_wait();  // residuals may come from the previous kernel
@@ -230,20 +242,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 e != 0 || mbar_wait(bar_accf, i & 1, abort_flag, p.status, kStatusTimeoutAccum);
             if (!bar_epi_and(got && *abort_flag == 0)) break;
             tc_fence_after();
-            uint32_t r[4][32];
+            uint32_t r[kChunks][32];
             const uint32_t t_row =
-                tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * 128);
+                tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * (BN / 2));
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
+            for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
             tmem_ld_wait();
             tc_fence_before();
             bar_epi_and(true);
             if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
             const int m = m_tile * 128 + row;
             if (m < p.M) {
-                const int n = n_tile * kBN + half * 128;
+                const int n = n_tile * BN + half * (BN / 2);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < kChunks; ++c) {
                     float v[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
@@ -281,43 +293,51 @@ int gemm_persistent_grid(int M, int n_tiles) {
     return tiles < sms ? tiles : sms;
 }
 
-template <int EPI>
+template <int BN, int EPI>
 static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(gemm_persistent_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(gemm_persistent_kernel<BN, EPI>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, PCfg<BN>::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gemm_persistent_grid(p.M, p.n_tiles));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = PCfg<BN>::kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<EPI>, ta, tb, p);
+    return cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<BN, EPI>, ta, tb, p);
 }
 
-cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+template <int BN>
+static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
     switch (p.epi) {
-    case kEpiNone: return launch_epi<kEpiNone>(ta, tb, p, s);
-    case kEpiBias: return launch_epi<kEpiBias>(ta, tb, p, s);
-    case kEpiResidual: return launch_epi<kEpiResidual>(ta, tb, p, s);
-    case kEpiBiasResidual: return launch_epi<kEpiBiasResidual>(ta, tb, p, s);
-    case kEpiBiasGelu: return launch_epi<kEpiBiasGelu>(ta, tb, p, s);
-    case kEpiGeglu: return launch_epi<kEpiGeglu>(ta, tb, p, s);
+    case kEpiNone: return launch_epi<BN, kEpiNone>(ta, tb, p, s);
+    case kEpiBias: return launch_epi<BN, kEpiBias>(ta, tb, p, s);
+    case kEpiResidual: return launch_epi<BN, kEpiResidual>(ta, tb, p, s);
+    case kEpiBiasResidual: return launch_epi<BN, kEpiBiasResidual>(ta, tb, p, s);
+    case kEpiBiasGelu: return launch_epi<BN, kEpiBiasGelu>(ta, tb, p, s);
+    case kEpiGeglu: return launch_epi<BN, kEpiGeglu>(ta, tb, p, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
+cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
+                                   cudaStream_t s) {
+    if (block_n == 256) return launch_bn<256>(ta, tb, p, s);
+    if (block_n == 128) return launch_bn<128>(ta, tb, p, s);
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t probe_gemm_persistent() {
     cudaFuncAttributes fa;
-    return cudaFuncGetAttributes(&fa, gemm_persistent_kernel<kEpiNone>);
+    return cudaFuncGetAttributes(&fa, gemm_persistent_kernel<256, kEpiNone>);
 }
 
 }  // namespace nvfp4
