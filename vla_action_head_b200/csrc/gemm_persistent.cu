@@ -8,22 +8,24 @@
 // ("GROOT N1.7 update: Thor NVFP4 + FA4 performance tier", §What is in the tier;
 // "Pi0.5 Thor NVFP4 End-to-End Results", §Fused GeGLU FFN in the Decoder.)
 //
-// Roles (320 threads):
+// Roles (384 threads):
 //   warp 0      producer: TMA loads of the A (128 rows) and W (256 rows) code tiles and bulk
 //               loads of their scale atoms into a 4-stage ring; the weights of the first
 //               stages are issued before the programmatic-launch wait.
-//   warp 1      MMA issuer: tcgen05.cp (32x128b.warpx4) of the scale atoms, then 4 x
-//               tcgen05.mma kind::mxf4nvf4 block16 (M = 128, N = 256, K = 64) per 256-wide K tile.
+//   warps 10-11 scale copiers: tcgen05.cp (32x128b.warpx4) of the stage's scale atoms into
+//               one of two TMEM scale slots, signalled to the MMA warp by tcgen05.commit.
+//   warp 1      MMA issuer: 4 x tcgen05.mma kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64)
+//               per 256-wide K tile.
 //   warps 2..9  epilogue: two warps per TMEM sub-partition, each draining 128 of the 256
 //               accumulator columns of its 32 rows into registers; the accumulator is handed
 //               back to the MMA warp right after the drain, so the fused epilogue of one tile
 //               runs while the next tile's MMAs do.  The kernel is instantiated per epilogue
 //               kind, so each instance holds one path (and fits its registers without spills).
 //
-// The scale-copy instructions (3 per 64-wide K step, one MMA each) bound the issue rate of
-// the MMA warp.  Copying two atoms per tcgen05.cp.128x256b needs each atom 4 times in
-// shared memory; building those images (with 48 small bulk copies per stage, or with a warp
-// of loads and stores) measured slower than the plain copies, so the kernel keeps them.
+// Scale copies: tcgen05.cp instructions from one thread complete one after another (about
+// 90 cycles each, measured), which made them, not the MMAs, bound a single issuing thread.
+// From separate warps they overlap (48 copies: 4490 cycles from one thread, 1011 from eight
+// warps), so two copier warps issue them and the MMA warp only issues MMAs.
 //
 // Every wait is bounded (sm100.cuh); an expired wait records a status and the CTA unwinds.
 #include <cuda.h>
@@ -37,7 +39,8 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+constexpr int kCopiers = 2;  // warps 10, 11
 constexpr int kSfAtom = 512;
 
 // Shared-memory and TMEM plan for a tile width BN (256, or 128 when 256-wide tiles would
@@ -56,12 +59,13 @@ struct PCfg {
     static constexpr int kStage = kOffSfb + kStageSfb;  // 54 KB (BN 256) / 36 KB (BN 128)
     static constexpr int kStages = (216 * 1024) / kStage;
     static constexpr int kOffBar = kStages * kStage;
-    // barriers: full[kStages], empty[kStages], acc_full, acc_empty
-    static constexpr int kOffMisc = kOffBar + (2 * kStages + 2) * 8;
+    // barriers: full[kStages], empty[kStages], acc_full, acc_empty, sf_ready[2], sf_free[2]
+    static constexpr int kOffMisc = kOffBar + (2 * kStages + 6) * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-    static constexpr int kColSfa = BN;                        // 16 columns: 4 k-blocks x 4
-    static constexpr int kColSfb = BN + 16;                   // 4 k-blocks x (groups x 4)
-    static constexpr int kTmemCols = (kColSfb + 16 * kGroups) <= 256 ? 256 : 512;
+    // scale columns: two slots (stage parity) of [A: 4 k-blocks x 4 | W: 4 k-blocks x groups x 4]
+    static constexpr int kColSf = BN;
+    static constexpr int kSfSlot = 16 + 16 * kGroups;
+    static constexpr int kTmemCols = (kColSf + 2 * kSfSlot) <= 256 ? 256 : 512;
     static_assert(kStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
@@ -93,7 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using Cf = PCfg<BN>;
     constexpr int kStages = Cf::kStages, kStage = Cf::kStage, kStageA = Cf::kStageA, kStageB = Cf::kStageB;
     constexpr int kOffB = Cf::kOffB, kOffSfa = Cf::kOffSfa, kOffSfb = Cf::kOffSfb, kGroups = Cf::kGroups;
-    constexpr int kColSfa = Cf::kColSfa, kColSfb = Cf::kColSfb, kTmemCols = Cf::kTmemCols;
+    constexpr int kColSf = Cf::kColSf, kSfSlot = Cf::kSfSlot, kTmemCols = Cf::kTmemCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -101,6 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_empty = bar_full + 8 * kStages;
     const uint32_t bar_accf = bar_empty + 8 * kStages;
     const uint32_t bar_acce = bar_accf + 8;
+    const uint32_t bar_sfr = bar_acce + 8;  // 2: scale slot copied (one arrival per copier warp)
+    const uint32_t bar_sff = bar_sfr + 16;  // 2: scale slot read by its MMAs
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + Cf::kOffMisc);  // [0] TMEM base, [1] abort
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
@@ -120,6 +126,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(bar_accf, 1);
         mbar_init(bar_acce, 1);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(bar_sfr + 8 * j, kCopiers);
+            mbar_init(bar_sff + 8 * j, 1);
+        }
         misc[1] = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -202,29 +212,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < k_tiles; ++kt, ++st) {
-                    const int s = st % kStages;
-                    if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
+                    const int s = st % kStages, slot = st & 1;
+                    if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull) ||
+                        !mbar_wait(bar_sfr + 8 * slot, (st >> 1) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nkb = nkb_of(kt);
                     const uint32_t base = sbase + s * kStage;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * kb, desc_sf_32x128b(base + kOffSfa + kb * kSfAtom));
-#pragma unroll
-                        for (int g = 0; g < kGroups; ++g)
-                            tc_cp_32x128b_warpx4(tmem + kColSfb + 4 * kGroups * kb + 4 * g,
-                                                 desc_sf_32x128b(base + kOffSfb + g * 4 * kSfAtom + kb * kSfAtom));
-                    }
+                    const uint32_t t_sf = tmem + kColSf + slot * kSfSlot;
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_mxf4nvf4(tmem, desc_kmajor_sw128(base + 32 * kb), desc_kmajor_sw128(base + kOffB + 32 * kb),
-                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 4 * kGroups * kb,
+                                        idesc, t_sf + 4 * kb, t_sf + 16 + 4 * kGroups * kb,
                                         (kt > 0 || kb > 0) ? 1u : 0u);
-                    tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs have read it
+                    tc_commit(bar_empty + 8 * s);     // frees the stage once these MMAs have read it
+                    tc_commit(bar_sff + 8 * slot);    // and the scale slot
                 }
                 tc_commit(bar_accf);  // always: completion of every MMA issued above
                 if (!ok) break;
+            }
+        }
+    } else if (warp >= 10) {
+        if (lane == 0) {
+            // --------------------------- scale copiers (warps 10, 11) ---------------------------
+            // tcgen05.cp issued from one thread run one after another; spread over two warps they
+            // overlap, and with two scale slots they overlap the MMAs of the previous stage too.
+            // Copier c takes k-blocks 2c and 2c + 1 of every stage.
+            const int c = warp - 10;
+            for (int st = 0; st < steps; ++st) {
+                const int s = st % kStages, slot = st & 1, kt = st % k_tiles;
+                if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull))
+                    break;
+                if (st >= 2 && !mbar_wait(bar_sff + 8 * slot, ((st >> 1) - 1) & 1, abort_flag, p.status,
+                                          kStatusTimeoutFull))
+                    break;
+                tc_fence_after();
+                const int nkb = nkb_of(kt);
+                const uint32_t base = sbase + s * kStage;
+                const uint32_t t_sf = tmem + kColSf + slot * kSfSlot;
+                for (int kb = 2 * c; kb < 2 * c + 2 && kb < nkb; ++kb) {
+                    tc_cp_32x128b_warpx4(t_sf + 4 * kb, desc_sf_32x128b(base + kOffSfa + kb * kSfAtom));
+#pragma unroll
+                    for (int g = 0; g < kGroups; ++g)
+                        tc_cp_32x128b_warpx4(t_sf + 16 + 4 * kGroups * kb + 4 * g,
+                                             desc_sf_32x128b(base + kOffSfb + g * 4 * kSfAtom + kb * kSfAtom));
+                }
+                tc_commit(bar_sfr + 8 * slot);  // arrives when this warp's copies have landed
             }
         }
     } else {
