@@ -14,9 +14,11 @@
 //               1-D bulk loads of their scale-factor atoms into a STAGES-deep ring; the
 //               weight half of the first stages is issued before the programmatic-launch
 //               wait because weights never depend on the previous kernel.
-//   warp 1      tensor-memory allocation; one thread issues tcgen05.cp (scales smem->TMEM)
-//               and tcgen05.mma kind::mxf4nvf4 block16 (M = 128, N = BN, K = 64 each).
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one row per thread), then
+//   warp 1      tensor-memory allocation; one thread issues tcgen05.mma kind::mxf4nvf4
+//               block16 (M = 128, N = BN, K = 64 each).
+//   warps 2..5  until the accumulator is ready: tcgen05.cp of the scale atoms (smem -> TMEM),
+//               one k-block per warp, into two scale slots; then the epilogue:
+//               tcgen05.ld of the fp32 accumulator (one row per thread), then
 //               either the fused epilogue directly, or split-K partials to the workspace
 //               with an arrival ticket; the last CTA of a tile reduces the partials in
 //               split order (deterministic) and runs the epilogue.
@@ -56,9 +58,10 @@ struct Cfg {
     static constexpr int kSfaBytes = 4 * kSfAtom;
     static constexpr int kSfbBytes = kSfbGroups * 4 * kSfAtom;
     // tensor-memory columns: accumulator, then 16 columns of A scales, then B scales
-    static constexpr int kColSfa = BN;
-    static constexpr int kColSfb = BN + 16;
-    static constexpr int kColsUsed = BN + 16 + 16 * kSfbGroups;
+    // scale columns: two slots (stage parity) of [A: 4 k-blocks x 4 | W: 4 k-blocks x groups x 4]
+    static constexpr int kColSf = BN;
+    static constexpr int kSfSlot = 16 + 16 * kSfbGroups;
+    static constexpr int kColsUsed = BN + 2 * kSfSlot;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                      : kColsUsed <= 256 ? 256 : 512;
 };
@@ -75,7 +78,7 @@ struct Smem {
     static constexpr int kOffSfa = kOffB + STAGES * Cfg<BN>::kBBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * Cfg<BN>::kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes;
-    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 1) * 8;
+    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 5) * 8;
     static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
     // split-K partial tile for the cluster reduction, reusing the stage buffers
     static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
@@ -107,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     const uint32_t bar_full = sbase + S::kOffBar;             // STAGES barriers
     const uint32_t bar_empty = bar_full + STAGES * 8;         // STAGES barriers
     const uint32_t bar_acc = bar_empty + STAGES * 8;          // 1 barrier
+    const uint32_t bar_sfr = bar_acc + 8;                     // 2: scale slot copied (4 arrivals)
+    const uint32_t bar_sff = bar_sfr + 16;                    // 2: scale slot read by its MMAs
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + S::kOffMisc);
     // misc[0] = tensor-memory base, misc[1] = abort flag, misc[2] = split-K ticket,
     // misc[3] = accumulator-valid decision of the epilogue warps
@@ -134,6 +139,10 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             mbar_init(bar_empty + 8 * s, 1);
         }
         mbar_init(bar_acc, 1);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(bar_sfr + 8 * j, 4);
+            mbar_init(bar_sff + 8 * j, 1);
+        }
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -211,32 +220,25 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             // ------------------------------ MMA issuer ------------------------------
             constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
             const uint32_t t_acc = tmem;
-            const uint32_t t_sfa = tmem + C::kColSfa;
-            const uint32_t t_sfb = tmem + C::kColSfb;
             const uint32_t sfb_sub = (BN == 64) ? static_cast<uint32_t>((n0 & 127) >> 5) : 0u;
             for (int j = 0; j < nkt; ++j) {
-                const int s = j % STAGES, kt = kt_begin + j;
-                if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull)) break;
+                const int s = j % STAGES, kt = kt_begin + j, slot = j & 1;
+                if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull) ||
+                    !mbar_wait(bar_sfr + 8 * slot, (j >> 1) & 1, abort_flag, &g_device_status, kStatusTimeoutFull))
+                    break;
                 tc_fence_after();
                 if (trace != nullptr && j == 0) trace[3] = globaltimer_ns();
                 const int nkb = nkb_of(kt);
                 const uint32_t a_s = sbase + S::kOffA + s * S::kA;
                 const uint32_t b_s = sbase + S::kOffB + s * C::kBBytes;
-                const uint32_t sfa_s = sbase + S::kOffSfa + s * C::kSfaBytes;
-                const uint32_t sfb_s = sbase + S::kOffSfb + s * C::kSfbBytes;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    tc_cp_32x128b_warpx4(t_sfa + 4 * kb, desc_sf_32x128b(sfa_s + kb * kSfAtom));
-#pragma unroll
-                    for (int gi = 0; gi < C::kSfbGroups; ++gi)
-                        tc_cp_32x128b_warpx4(t_sfb + 4 * C::kSfbGroups * kb + 4 * gi,
-                                             desc_sf_32x128b(sfb_s + gi * 4 * kSfAtom + kb * kSfAtom));
-                }
+                const uint32_t t_sf = tmem + C::kColSf + slot * C::kSfSlot;
                 for (int kb = 0; kb < nkb; ++kb) {
                     tc_mma_mxf4nvf4(t_acc, desc_kmajor_sw128(a_s + 32 * kb), desc_kmajor_sw128(b_s + 32 * kb),
-                                    idesc, t_sfa + 4 * kb, t_sfb + 4 * C::kSfbGroups * kb + sfb_sub,
+                                    idesc, t_sf + 4 * kb, t_sf + 16 + 4 * C::kSfbGroups * kb + sfb_sub,
                                     (j > 0 || kb > 0) ? 1u : 0u);
                 }
-                tc_commit(bar_empty + 8 * s);  // frees the stage once these MMAs finished reading it
+                tc_commit(bar_empty + 8 * s);   // frees the stage once these MMAs finished reading it
+                tc_commit(bar_sff + 8 * slot);  // and the scale slot
             }
             if (trace != nullptr) trace[4] = globaltimer_ns();
             tc_commit(bar_acc);  // always: completion of every MMA issued above
@@ -247,6 +249,32 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
         const int row = q * 32 + lane;
         const int m = m0 + row;
         const bool row_ok = m < p.M;
+        // Until the accumulator is ready these warps copy the scale atoms (tcgen05.cp from one
+        // thread complete one after another; from four warps they overlap): warp w copies
+        // k-block w of each stage into the stage's scale slot (of two).
+        if (lane == 0) {
+            const int w = warp - 2;
+            const uint32_t sfa_s0 = sbase + S::kOffSfa, sfb_s0 = sbase + S::kOffSfb;
+            for (int j = 0; j < nkt; ++j) {
+                const int s = j % STAGES, kt = kt_begin + j, slot = j & 1;
+                if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull))
+                    break;
+                if (j >= 2 && !mbar_wait(bar_sff + 8 * slot, ((j >> 1) - 1) & 1, abort_flag, &g_device_status,
+                                         kStatusTimeoutFull))
+                    break;
+                tc_fence_after();
+                const uint32_t t_sf = tmem + C::kColSf + slot * C::kSfSlot;
+                if (w < nkb_of(kt)) {
+                    tc_cp_32x128b_warpx4(t_sf + 4 * w, desc_sf_32x128b(sfa_s0 + s * C::kSfaBytes + w * kSfAtom));
+#pragma unroll
+                    for (int gi = 0; gi < C::kSfbGroups; ++gi)
+                        tc_cp_32x128b_warpx4(t_sf + 16 + 4 * C::kSfbGroups * w + 4 * gi,
+                                             desc_sf_32x128b(sfb_s0 + s * C::kSfbBytes + gi * 4 * kSfAtom + w * kSfAtom));
+                }
+                tc_commit(bar_sfr + 8 * slot);  // arrives when this warp's copies have landed
+            }
+        }
+        __syncwarp();
         const bool done = drain_wait(bar_acc, 0);
         // one decision for all four epilogue warps (tcgen05.ld and the named barriers below
         // must be reached uniformly)
