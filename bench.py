@@ -35,6 +35,34 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_OVER_BF16 = 4.0  # nominal dense ratio, 9 PF / 2.25 PF
 DIT = dict(M=41, H=1536, F=6144)
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels,
+# from the ncu captures summarised in profiles/ (commands there), keyed by a hash of the
+# kernel sources they were taken on: once a source changes the figure is reported as null.
+TRAFFIC = {
+    "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
+                 "sha256": "55a45578f42ae511aca7d35cd22b624830deb6dd0b2ef5f6e15da22c663bc10a",
+                 "bytes": 4211776},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
+    "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
+                        "sha256": "1bc29a87a8bcb6d02ea626072f3435256bd24bbf0f35c7d06f8b5bd2f7fe4476",
+                        "bytes": 38946560},  # profiles/gemm_persistent_prefill_m968_full.md
+}
+
+
+def sources_sha(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "vla_action_head_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic(key):
+    t = TRAFFIC[key]
+    if t["bytes"] is None or t["sha256"] != sources_sha(t["sources"]):
+        return None
+    return t["bytes"]
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -435,7 +463,8 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
             tot_ms += ms
     ach = tot_b / (tot_ms * 1e-3) / 1e9
     out["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                       "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+                       "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic("dit_gemm"),
+                       "algorithmic_bytes_per_launch": tot_b // len(specs),
                        "kernel": "gemm_kernel (4 DiT GEMMs, M=41, L2-cold weights)", "peak_kind": pk_kind,
                        "per_gemm": per}
     # ---- 18-layer action-expert stack (config 3 layers, one CUDA graph) ----
@@ -482,8 +511,10 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     out["prefill_m968"] = {"us_per_layer": round(ms * 1e3, 2), "tflops": round(tf, 1),
                            "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1)}
     out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_peak, 1),
-                            "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4), "traffic": None,
-                            "kernel": "gemm_kernel gate_up 968x32768x2048 GeGLU->FP4",
+                            "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4),
+                            "traffic": traffic("prefill_gate_up"),
+                            "algorithmic_bytes_per_launch": gemm_bytes(968, 32768, 2048, "geglu"),
+                            "kernel": "gemm_persistent_kernel gate_up 968x32768x2048 GeGLU->FP4",
                             "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)"}
     del pre, xp, yp, outs
     # ---- M sweep on the 1536 -> 6144 GEMM (bias, bf16 out), 48 distinct weights ----
