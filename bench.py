@@ -219,8 +219,10 @@ def gemm_ring_time(A, lins, epi, outs, ws, stream, reps=20, res=None):
 
 
 # ---------------------------------------------------------------------------------------
-def cpu_baseline_dit(steps=1):
-    """The oracle (single-threaded C, fp64 GEMM) on one full DiT layer at M = 41."""
+def cpu_baseline_dit(steps=1, threads=1):
+    """The oracle (single-threaded C, fp64 GEMM) on one full DiT layer at M = 41.  threads > 1:
+    the GEMMs' output rows are partitioned over that many host threads (the oracle call
+    releases the interpreter lock), the norms stay on one thread."""
     import numpy as np
     import torch
 
@@ -242,18 +244,36 @@ def cpu_baseline_dit(steps=1):
     def bf16(v):
         return synth.f32_to_bf16_bits(v.astype(np.float32))
 
+    pool = None
+    if threads > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        pool = ThreadPoolExecutor(threads)
+
+    def gemm(*a, **kw):
+        if pool is None:
+            return orc.gemm(*a, **kw)
+        parts = np.array_split(np.arange(M), threads)
+        res = list(pool.map(lambda r: orc.gemm(*a, rows=r, **kw), parts))
+        out = {"v": np.concatenate([r["v"] for r in res])}
+        if res[0]["codes"] is not None:  # each part fills its own rows of zeroed buffers
+            out["codes"] = np.bitwise_or.reduce([r["codes"] for r in res])
+            out["sf"] = np.bitwise_or.reduce([r["sf"] for r in res])
+        return out
+
     t0 = time.perf_counter()
     for _ in range(steps):
         a1, a1s = orc.quantize_norm(x, "adaln", scale=sc, shift=sh, eps=1e-6)
-        orc.gemm(a1, a1s, 1.0, M, W[0][0], W[0][1], W[0][2], 3 * H, H, epi="bias", bias=B[0])
+        gemm(a1, a1s, 1.0, M, W[0][0], W[0][1], W[0][2], 3 * H, H, epi="bias", bias=B[0])
         c, cs = orc.quantize_norm(ctx, "none")
-        h = bf16(orc.gemm(c, cs, 1.0, M, W[1][0], W[1][1], W[1][2], H, H, epi="bias_residual", bias=B[1],
-                          residual=x)["v"])
+        h = bf16(gemm(c, cs, 1.0, M, W[1][0], W[1][1], W[1][2], H, H, epi="bias_residual", bias=B[1],
+                      residual=x)["v"])
         a2, a2s = orc.quantize_norm(h, "layernorm", gamma=ga, beta=be, eps=1e-5)
-        u = orc.gemm(a2, a2s, 1.0, M, W[2][0], W[2][1], W[2][2], F, H, epi="bias_gelu", bias=B[2])
-        orc.gemm(u["codes"], u["sf"], 1.0, M, W[3][0], W[3][1], W[3][2], H, F, epi="bias_residual",
-                 bias=B[3], residual=h)
+        u = gemm(a2, a2s, 1.0, M, W[2][0], W[2][1], W[2][2], F, H, epi="bias_gelu", bias=B[2])
+        gemm(u["codes"], u["sf"], 1.0, M, W[3][0], W[3][1], W[3][2], H, F, epi="bias_residual",
+             bias=B[3], residual=h)
     dt = time.perf_counter() - t0
+    if pool is not None:
+        pool.shutdown()
     return dt / steps * 1e6  # us per layer
 
 
@@ -379,6 +399,18 @@ def main():
     ms_total = max_over_ranks(ws_n, e0.elapsed_time(e1))
     nvfp4.device_status()
     us_layer = ms_total * 1e3 / (args.steps * L * ws_n)
+    # per-step spread (each step timed on its own, after the timed region)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i in range(args.steps):
+            run_steps(1)
+            evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per_step = sorted(evs[i].elapsed_time(evs[i + 1]) * 1e3 / L for i in range(args.steps))
+    spread = {"median": round(statistics.median(per_step), 3),
+              "p95": round(per_step[min(len(per_step) - 1, int(0.95 * len(per_step)))], 3),
+              "unit": UNIT, "steps": args.steps}
     w_bytes = sum(l.weight_bytes() for l in stack[0].linears())
     gbs_weights = w_bytes / (us_layer * 1e-6) / 1e9
 
@@ -409,6 +441,7 @@ def main():
                        "l2": f"inputs larger than L2: {L} x {w_bytes / 1e6:.1f} MB distinct weights per step",
                        "graph": "CUDA graph replay, programmatic dependent launch"},
             "weight_stream_gbs": round(gbs_weights, 1),
+            "per_step_us_per_layer": spread,
             "clocks": clocks,
             "gpu_launches": args.steps * L * layers.DiTLayer.launches,
             "e2e": {"value": round(us_layer_e2e, 3), "unit": UNIT, "h2d_bytes_per_step": M * H * 2,
@@ -428,6 +461,14 @@ def main():
                                               "single-threaded C"}
         except Exception as e:  # the baseline is reported, never required
             line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": str(e)}
+        try:
+            nthr = len(os.sched_getaffinity(0))
+            us_mt = cpu_baseline_dit(1, threads=nthr)
+            line["cpu_baseline_threads"] = {"value": round(us_mt, 1), "unit": UNIT, "cores": nthr,
+                                            "kind": "oracle", "sample": "the same DiT layer, GEMM output rows "
+                                            f"partitioned over {nthr} host threads"}
+        except Exception as e:
+            line["cpu_baseline_threads"] = {"value": None, "sample": str(e)[:200]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:
@@ -531,9 +572,38 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
             outs = [torch.empty((Ms, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
             ms = gemm_ring_time(A, lins, "bias", outs, wsp, stream, reps=10)
         b = gemm_bytes(Ms, 6144, 1536, "bias")
-        sweep.append({"M": Ms, "us": round(ms * 1e3, 3), "gbs": round(b / (ms * 1e-3) / 1e9, 1),
-                      "tflops": round(2.0 * Ms * 6144 * 1536 / (ms * 1e-3) / 1e12, 2)})
+        gbs = b / (ms * 1e-3) / 1e9
+        tf = 2.0 * Ms * 6144 * 1536 / (ms * 1e-3) / 1e12
+        # the bound by arithmetic intensity against the ridge of the two measured peaks
+        hbm_bound = (2.0 * Ms * 6144 * 1536 / b) < fp4_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+        sweep.append({"M": Ms, "us": round(ms * 1e3, 3), "gbs": round(gbs, 1), "tflops": round(tf, 2),
+                      "bound": "hbm" if hbm_bound else "tensor",
+                      "frac": round(gbs / pk["hbm_gbs"] if hbm_bound else tf / fp4_peak, 4)})
     out["m_sweep_1536x6144"] = sweep
+    # ---- tiny config: LayerNorm->NVFP4 of 41 x 256, then 41 x 512 x 256 GEMM + bias ----
+    with torch.cuda.stream(stream):
+        tl = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(1, synth.W0 + 100 * i), (512, 256), 0, 0.02,
+                                                    device=dev),
+                            synth.bf16_normal_torch(synth.seed_of(1, synth.BIAS0 + 100 * i), (512,), 0, 0.01,
+                                                    device=dev)) for i in range(48)]
+        xt = synth.bf16_normal_torch(synth.seed_of(1, synth.X), (41, 256), device=dev)
+        gt = synth.bf16_normal_torch(synth.seed_of(1, synth.GAMMA), (256,), 1.0, 0.1, device=dev)
+        bt = synth.bf16_normal_torch(synth.seed_of(1, synth.BETA), (256,), 0.0, 0.1, device=dev)
+        at = nvfp4.empty_fp4(41, 256, dev)
+        ot = torch.empty((41, 512), dtype=torch.bfloat16, device=dev)
+
+        def tiny():
+            for lin in tl:
+                nvfp4.quantize_norm(xt, "layernorm", gamma=gt, beta=bt, eps=1e-5, out=at)
+                nvfp4.gemm(at, lin.w, "bias", bias=lin.bias, out=ot, workspace=wsp)
+        tiny()
+    torch.cuda.synchronize()
+    g = capture(tiny, stream)
+    ms = time_graph(g, 20, stream) / len(tl)
+    del g
+    out["tiny_41x256_512"] = {"us_per_norm_plus_gemm": round(ms * 1e3, 3),
+                              "gemm_bytes": gemm_bytes(41, 512, 256, "bias"),
+                              "l2": "48 distinct weight copies (L2-warm: 3.6 MB in total)"}
     torch.cuda.synchronize()
     nvfp4.device_status()
     return out
