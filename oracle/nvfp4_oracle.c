@@ -257,6 +257,42 @@ void orc_norm_rows(const void *x, int in_fp32, int rows, int K, int ldx, int kin
     }
 }
 
+/* fp32 -> bf16, round to nearest even at bit 16 (IEEE 754 roundTiesToEven applied to the
+ * 8-bit significand of bfloat16); overflow goes to infinity; NaN stays a quiet NaN.       */
+uint16_t orc_f32_to_bf16(float v) {
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u); /* NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+void orc_f32_to_bf16_array(const float *v, size_t n, uint16_t *out) {
+    for (size_t i = 0; i < n; ++i) out[i] = orc_f32_to_bf16(v[i]);
+}
+
+/* Gated residual update in front of a norm ("Pi0.5 Thor NVFP4 End-to-End Results",
+ * §Implemented Path: gated residual update + Pi0.5 AdaRMSNorm + gate output + NVFP4/SFA in
+ * one launch before Gate+Up and the next layer's QKV):
+ *   h[r, k] = x[r, k] + gate[k] * d[r, k]
+ * x is the residual stream, d the sublayer's output, gate the layer's modulation gate.
+ * READING: one fp32 product, then one fp32 sum (no fused multiply-add), rounded once to
+ * bf16 (the residual stream is bf16).  The norm that follows reads that bf16 h, so the
+ * fused launch is the two-step chain "update, then norm -> FP4".  A NULL gate reads as 1.  */
+void orc_gated_residual(const uint16_t *x, const uint16_t *d, const uint16_t *gate, int rows, int K,
+                        uint16_t *h) {
+    for (int r = 0; r < rows; ++r) {
+        for (int k = 0; k < K; ++k) {
+            size_t i = (size_t)r * K + k;
+            float g = gate ? bf16_to_f32(gate[k]) : 1.0f;
+            float t = g * bf16_to_f32(d[i]);
+            float s = bf16_to_f32(x[i]) + t;
+            h[i] = orc_f32_to_bf16(s);
+        }
+    }
+}
+
 /* Fused norm -> FP4 is, by the pages' contract, identical to the two-step chain
  * ("GROOT N1.7 ...", §What is in the tier: bit-identical to the two-step chain).
  * READING: the intermediate y is not rounded to bf16/fp16 between the steps.           */

@@ -70,6 +70,14 @@ void orc_norm_rows(const void *x, int in_fp32, int rows, int K, int ldx, int kin
                    const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,
                    const uint16_t *mod_shift, float eps, float *y);
 
+/* fp32 -> bf16, round to nearest even (single value and array). */
+uint16_t orc_f32_to_bf16(float v);
+void orc_f32_to_bf16_array(const float *v, size_t n, uint16_t *out);
+
+/* gated residual update: h = bf16(x + gate * d), fp32 product then fp32 sum; gate NULL = 1. */
+void orc_gated_residual(const uint16_t *x, const uint16_t *d, const uint16_t *gate, int rows, int K,
+                        uint16_t *h);
+
 /* fused: norm then quantize, written as the two steps. */
 void orc_quantize_norm(const void *x, int in_fp32, int rows, int K, int ldx, int kind,
                        const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,

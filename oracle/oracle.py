@@ -56,6 +56,10 @@ def lib():
                                C.c_int, P, P, C.c_int, P, C.c_int, P, P, C.c_float, P, P]
         L.orc_gelu_tanh.restype = C.c_double
         L.orc_gelu_tanh.argtypes = [C.c_double]
+        L.orc_f32_to_bf16_array.restype = None
+        L.orc_f32_to_bf16_array.argtypes = [P, C.c_size_t, P]
+        L.orc_gated_residual.restype = None
+        L.orc_gated_residual.argtypes = [P, P, P, C.c_int, C.c_int, P]
         _lib = L
     return _lib
 
@@ -154,6 +158,33 @@ def quantize_norm(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e
                             _p(_c(beta, np.uint16)), _p(_c(scale, np.uint16)),
                             _p(_c(shift, np.uint16)), float(eps), float(g), _p(codes), _p(sf))
     return codes, sf
+
+
+def f32_to_bf16(v):
+    """fp32 values -> bf16 bit patterns (uint16), round to nearest even."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.uint16)
+    lib().orc_f32_to_bf16_array(_p(v), v.size, _p(out))
+    return out
+
+
+def gated_residual(x, d, gate=None):
+    """h = bf16(x + gate * d) for bf16 x, d [rows, K] and gate [K] (None: 1)."""
+    x = _c(x, np.uint16)
+    d = _c(d, np.uint16)
+    rows, K = x.shape
+    h = np.empty((rows, K), np.uint16)
+    lib().orc_gated_residual(_p(x), _p(d), _p(_c(gate, np.uint16)), rows, K, _p(h))
+    return h
+
+
+def residual_quantize_norm(x, d, gate, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
+                           g=1.0):
+    """The fused gated-residual front-end as its two steps: h = gated_residual(x, d, gate),
+    then quantize_norm(h).  Returns (h, codes, sf)."""
+    h = gated_residual(x, d, gate)
+    codes, sf = quantize_norm(h, kind, gamma=gamma, beta=beta, scale=scale, shift=shift, eps=eps, g=g)
+    return h, codes, sf
 
 
 def quantize_weight(w, interleave_gate_up=False):
