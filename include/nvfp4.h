@@ -164,6 +164,22 @@ nvfp4_status nvfp4_norm_f32(const void *x, nvfp4_in_dtype dt, int M, int K, int 
                         const void *mod_scale, const void *mod_shift, float eps, float *y,
                         nvfp4_stream_t stream);
 
+/* Gated residual front-end, one launch ([PI05] §Implemented Path: gated residual update +
+ * Pi0.5 AdaRMSNorm + gate output + NVFP4/SFA in one launch before Gate+Up and the next
+ * layer's QKV).  Per element of the bf16 residual stream x [M, K] (ldx) and the sublayer
+ * output d [M, K] (ldd), with the bf16 gate [K] (NULL reads 1):
+ *   h = bf16_rn(x + gate * d)      (one fp32 product, one fp32 sum, one rounding)
+ * h is stored to h_out [M, K] (ldh, bf16, device) as the new residual stream, and the norm
+ * `kind` + block quantizer of nvfp4_quantize_norm run on that bf16 h, so the result equals
+ * nvfp4_quantize_norm(h, ...) bit for bit.  h_out may alias x (each element is read before
+ * it is written, by the same thread); it must not overlap d.  Same constraints as
+ * nvfp4_quantize_norm, bf16 only; ldd, ldh multiples of 8 and >= K. */
+nvfp4_status nvfp4_residual_quantize_norm(const void *x, const void *d, const void *gate, int M, int K,
+                                          int ldx, int ldd, int ldh, nvfp4_norm kind, const void *gamma,
+                                          const void *beta, const void *mod_scale, const void *mod_shift,
+                                          float eps, float global_scale, void *h_out, uint8_t *codes,
+                                          uint8_t *sf, nvfp4_stream_t stream);
+
 /* ---- offline weight quantize --------------------------------------------------------- */
 
 /* W bf16 [N, K] (ldw) -> codes [N, K/2] + sf (nvfp4_sf_bytes(N, K), pre-zeroed) with the

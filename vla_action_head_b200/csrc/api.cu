@@ -326,9 +326,17 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     return from_cuda(e);
 }
 
+struct Residual {
+    const void *d = nullptr;
+    int ldd = 0;
+    const void *gate = nullptr;
+    void *h = nullptr;
+    int ldh = 0;
+};
+
 nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, nvfp4_norm kind, const void *gamma,
                        const void *beta, const void *mod_scale, const void *mod_shift, float eps, float g,
-                       uint8_t *codes, uint8_t *sf, float *y_out, cudaStream_t stream) {
+                       uint8_t *codes, uint8_t *sf, float *y_out, cudaStream_t stream, const Residual &res = {}) {
     if (M < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32) return NVFP4_ERR_INVALID_ARG;
     if (static_cast<int>(kind) < 0 || static_cast<int>(kind) > 4) return NVFP4_ERR_INVALID_ARG;
@@ -345,9 +353,20 @@ nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, 
     if (!aligned16(x) || ldx % (dt == NVFP4_IN_FP32 ? 4 : 8) != 0) return NVFP4_ERR_MISALIGNED;
     for (const void *pp : {gamma, beta, mod_scale, mod_shift})
         if (pp != nullptr && !aligned16(pp)) return NVFP4_ERR_MISALIGNED;
+    if (res.d != nullptr) {
+        if (dt != NVFP4_IN_BF16 || res.h == nullptr || res.ldd < K || res.ldh < K) return NVFP4_ERR_INVALID_ARG;
+        if (!aligned16(res.d) || !aligned16(res.h) || res.ldd % 8 != 0 || res.ldh % 8 != 0 ||
+            (res.gate != nullptr && !aligned16(res.gate)))
+            return NVFP4_ERR_MISALIGNED;
+    }
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
     NormArgs a = {};
+    a.res_d = static_cast<const uint16_t *>(res.d);
+    a.ldd = res.ldd;
+    a.res_gate = static_cast<const uint16_t *>(res.gate);
+    a.h_out = static_cast<uint16_t *>(res.h);
+    a.ldh = res.ldh;
     a.x = x;
     a.M = M;
     a.K = K;
@@ -449,6 +468,21 @@ nvfp4_status nvfp4_quantize_norm(const void *x, nvfp4_in_dtype dt, int M, int K,
                                  float eps, float global_scale, uint8_t *codes, uint8_t *sf, nvfp4_stream_t stream) {
     return norm_impl(x, dt, M, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, global_scale, codes, sf,
                      nullptr, stream);
+}
+
+nvfp4_status nvfp4_residual_quantize_norm(const void *x, const void *d, const void *gate, int M, int K, int ldx,
+                                          int ldd, int ldh, nvfp4_norm kind, const void *gamma, const void *beta,
+                                          const void *mod_scale, const void *mod_shift, float eps, float global_scale,
+                                          void *h_out, uint8_t *codes, uint8_t *sf, nvfp4_stream_t stream) {
+    if (M > 0 && d == nullptr) return NVFP4_ERR_INVALID_ARG;
+    Residual r;
+    r.d = d;
+    r.ldd = ldd;
+    r.gate = gate;
+    r.h = h_out;
+    r.ldh = ldh;
+    return norm_impl(x, NVFP4_IN_BF16, M, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, global_scale, codes,
+                     sf, nullptr, stream, r);
 }
 
 nvfp4_status nvfp4_norm_f32(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, nvfp4_norm kind, const void *gamma,

@@ -19,6 +19,13 @@ struct NormArgs {
     uint8_t *codes;
     uint8_t *sf;
     float *y_out;  // non-NULL: write the normalized fp32 y instead of quantizing
+    // gated residual front-end (bf16 only): x is replaced by h = bf16(x + gate * d), which
+    // is also stored to h_out; res_d == NULL: none
+    const uint16_t *res_d;
+    int ldd;
+    const uint16_t *res_gate;  // NULL: 1
+    uint16_t *h_out;
+    int ldh;
 };
 
 cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s);

@@ -81,6 +81,10 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
     uint8_t *const codes_out = p.codes;
     uint8_t *const sf_out = p.sf;
     float *const y_out = p.y_out;
+    const uint16_t *const res_d = F32 ? nullptr : p.res_d;
+    const uint16_t *const res_gate = p.res_gate;
+    uint16_t *const h_out = p.h_out;
+    const int ldd = p.ldd, ldh = p.ldh;
     const int nblk = K >> 4;
     const int k_atoms = (K + 63) >> 6;
     const bool row_ok = row < M;
@@ -117,6 +121,32 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
         } else {
 #pragma unroll
             for (int j = 0; j < kWords; ++j) raw[i][j] = 0u;
+        }
+        if constexpr (!F32) {
+            // gated residual front-end ("Pi0.5 Thor NVFP4 End-to-End Results", §Implemented
+            // Path): h = x + gate * d, one fp32 product and one fp32 sum, rounded once to bf16;
+            // h replaces x for the norm and is stored as the new residual stream
+            if (res_d != nullptr && ok) {
+                const uint4 *qd = reinterpret_cast<const uint4 *>(res_d + static_cast<size_t>(src_row) * ldd + b * 16);
+                const uint4 d0 = __ldcg(qd), d1 = __ldcg(qd + 1);
+                uint4 g0 = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u), g1 = g0;
+                if (res_gate != nullptr) {
+                    const uint4 *qg = reinterpret_cast<const uint4 *>(res_gate + b * 16);
+                    g0 = __ldg(qg);
+                    g1 = __ldg(qg + 1);
+                }
+                const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+                const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float lo = __fadd_rn(bf16lo(raw[i][j]), __fmul_rn(bf16lo(gw[j]), bf16lo(dw[j])));
+                    const float hi = __fadd_rn(bf16hi(raw[i][j]), __fmul_rn(bf16hi(gw[j]), bf16hi(dw[j])));
+                    raw[i][j] = pack_bf16x2_rn(lo, hi);
+                }
+                uint4 *qh = reinterpret_cast<uint4 *>(h_out + static_cast<size_t>(row) * ldh + b * 16);
+                qh[0] = make_uint4(raw[i][0], raw[i][1], raw[i][2], raw[i][3]);
+                qh[1] = make_uint4(raw[i][4], raw[i][5], raw[i][6], raw[i][7]);
+            }
         }
         if constexpr (kParamRegs) {
 #pragma unroll

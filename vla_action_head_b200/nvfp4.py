@@ -76,6 +76,7 @@ def lib():
             "nvfp4_get_device_status": (I, [P]),
             "nvfp4_set_gemm_trace": (I, [P, SZ]),
             "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
+            "nvfp4_residual_quantize_norm": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, P, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
             "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
@@ -162,6 +163,25 @@ def quantize_norm(x, kind="none", gamma=None, beta=None, scale=None, shift=None,
     _check("nvfp4_quantize_norm", st)
     out.global_scale = global_scale
     return out
+
+
+def residual_quantize_norm(x, d, gate, kind="adarms", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
+                           global_scale=1.0, h_out=None, out: Optional[NVFP4Tensor] = None):
+    """h = bf16(x + gate * d) (gate None: 1), stored to h_out (may be x itself), then the norm
+    `kind` -> NVFP4 of h.  Returns (h_out, NVFP4Tensor)."""
+    torch = _torch()
+    M, K = x.shape
+    if h_out is None:
+        h_out = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
+    if out is None:
+        out = empty_fp4(M, K, x.device, global_scale)
+    st = lib().nvfp4_residual_quantize_norm(_ptr(x), _ptr(d), _ptr(gate), M, K, x.stride(0), d.stride(0),
+                                            h_out.stride(0), NORM[kind], _ptr(gamma), _ptr(beta), _ptr(scale),
+                                            _ptr(shift), eps, global_scale, _ptr(h_out), _ptr(out.codes),
+                                            _ptr(out.sf), _stream())
+    _check("nvfp4_residual_quantize_norm", st)
+    out.global_scale = global_scale
+    return h_out, out
 
 
 def norm_f32(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, out=None):
