@@ -526,7 +526,28 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     ae_w = sum(l.weight_bytes() for l in ae[0].linears())
     out["action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
                                     "weight_stream_gbs": round(18 * ae_w / (ms * 1e-3) / 1e9, 1)}
-    del ae, xa, ca, ab
+    del ae, xa, ab
+    # ---- the same stack with the gated residual updates fused into the norm front-ends ----
+    with torch.cuda.stream(stream):
+        gae = [layers.GatedActionExpertLayer(layer=i, device=dev, ws=wsp) for i in range(18)]
+        r0 = synth.bf16_normal_torch(synth.seed_of(6, synth.X), (50, 1024), device=dev)
+        rg = r0.clone()
+
+        def gae_fwd():
+            rg.copy_(r0)
+            d, gate = None, None
+            for lay in gae:
+                d, gate = lay.forward(rg, d, gate, ca)
+        gae_fwd()
+    torch.cuda.synchronize()
+    g = capture(gae_fwd, stream)
+    ms = time_graph(g, 50, stream)
+    del g
+    gae_w = sum(l.weight_bytes() for l in gae[0].linears())
+    out["gated_action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
+                                          "weight_stream_gbs": round(18 * gae_w / (ms * 1e-3) / 1e9, 1),
+                                          "front_end": "gated residual + AdaRMSNorm -> NVFP4 in one launch"}
+    del gae, r0, rg, ca
     # ---- prefill layer at M = 968 (tensor-bound): ring of 4 distinct layers ----
     with torch.cuda.stream(stream):
         pre = [layers.PrefillLayer(layer=i, device=dev, ws=wsp) for i in range(4)]

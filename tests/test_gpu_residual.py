@@ -58,3 +58,34 @@ def test_residual_front_end_rejects_bad_args():
     st = L.nvfp4_residual_quantize_norm(x.data_ptr(), None, None, 4, 64, 64, 64, 64, 0, None, None, None, None,
                                         1e-6, 1.0, x.data_ptr(), x.data_ptr(), x.data_ptr(), None)
     assert st == 1  # no d
+
+
+def test_gated_action_expert_layer_against_oracle(orc):
+    """One layer of the gated stack: the attention-output GEMM (no residual epilogue) against
+    the oracle's fp64 GEMM, then the second front-end exactly, given the GPU's GEMM output."""
+    from parity import check_gemm_bf16
+    from vla_action_head_b200 import layers
+    lay = layers.GatedActionExpertLayer(device="cuda")
+    M, H, A = lay.M, lay.H, lay.A
+    x = synth.bf16_normal_torch(synth.seed_of(42, synth.X), (M, H), device="cuda")
+    ctx = synth.bf16_normal_torch(synth.seed_of(42, synth.CONTEXT), (M, A), device="cuda")
+    r = x.clone()
+    lay.forward(r, None, None, ctx)
+    torch.cuda.synchronize()
+    cq, cs = orc.quantize_norm(host(ctx), "none")
+    assert np.array_equal(host(lay.ctx_q.codes), cq) and np.array_equal(host(lay.ctx_q.sf), cs)
+    v = orc.gemm(cq, cs, 1.0, M, host(lay.o.w.codes), host(lay.o.w.sf), lay.o.w.global_scale, H, A, epi="none")["v"]
+    check_gemm_bf16(host(lay.d_o), v, what="gated layer attention-output")
+    rh, rc, rs = orc.residual_quantize_norm(host(x), host(lay.d_o), host(lay.g1), "adarms", scale=host(lay.s2),
+                                            shift=host(lay.t2), eps=1e-6)
+    assert np.array_equal(host(r), rh)
+    assert np.array_equal(host(lay.a2.codes), rc) and np.array_equal(host(lay.a2.sf), rs)
+    # a second layer consumes (d_out, g2) in its first front-end
+    lay2 = layers.GatedActionExpertLayer(layer=1, device="cuda")
+    r_before = host(r).copy()
+    d_out = host(lay.d_out).copy()
+    lay2.forward(r, lay.d_out, lay.g2, ctx)
+    torch.cuda.synchronize()
+    rh1, rc1, rs1 = orc.residual_quantize_norm(r_before, d_out, host(lay.g2), "adarms", scale=host(lay2.s1),
+                                               shift=host(lay2.t1), eps=1e-6)
+    assert np.array_equal(host(lay2.a1.codes), rc1) and np.array_equal(host(lay2.a1.sf), rs1)

@@ -14,6 +14,8 @@ epilogues into preallocated buffers, so a forward can be captured in a CUDA grap
                      AdaRMSNorm->FP4, QKV, attention-output (+residual), AdaRMSNorm->FP4,
                      gate/up with GeGLU -> FP4 (pairwise-interleaved weights), down
                      (+residual).
+  GatedActionExpertLayer  the same layer with the gated residual updates fused into the
+                     norm front-ends (nvfp4_residual_quantize_norm).
   PrefillLayer       backbone-shaped prefill layer at M = 968: RMSNorm->FP4, QKV,
                      RMSNorm->FP4, gate/up GeGLU -> FP4, down (+residual).
 
@@ -137,6 +139,66 @@ class ActionExpertLayer:
             nvfp4.op_gemm(self.a2, self.gate_up.w, "geglu", out=self.u),
             nvfp4.op_gemm(self.u, self.down.w, "residual", residual=self.h, out=y),
         ]
+
+    launches = 7
+
+
+class GatedActionExpertLayer:
+    """Pi0.5 action-expert decoder layer with the gated residual updates moved into the norm
+    front-ends ("Pi0.5 Thor NVFP4 End-to-End Results", §Implemented Path: gated residual update
+    + Pi0.5 AdaRMSNorm + gate output + NVFP4/SFA in one launch before Gate+Up and the next
+    layer's QKV).  The residual stream r is updated in place:
+
+      r = r + g_in * d_in;  a1 = AdaRMS(r)(1 + s1) + t1 -> FP4    (front-end 1; d_in from the
+                                                                    previous layer's down)
+      QKV; context -> FP4; d_o = O(context)                        (bf16, no residual)
+      r = r + g1 * d_o;     a2 = AdaRMS(r)(1 + s2) + t2 -> FP4     (front-end 2)
+      u = GeGLU(gate_up(a2)) -> FP4;  d_out = down(u)              (bf16, no residual)
+
+    forward returns (d_out, g2): the next layer's front-end 1 applies r += g2 * d_out."""
+
+    def __init__(self, M=50, H=1024, A=2048, F=4096, wl=6, layer=0, device="cuda", ws=None):
+        s = lambda tid: synth.seed_of(wl, 100 * layer + tid)  # noqa: E731
+        d = device
+        self.M, self.H, self.A, self.F = M, H, A, F
+        self.s1 = _rand(s(synth.MOD_SCALE), (H,), 0.0, 0.1, d)
+        self.t1 = _rand(s(synth.MOD_SHIFT), (H,), 0.0, 0.1, d)
+        self.s2 = _rand(s(synth.GAMMA), (H,), 0.0, 0.1, d)
+        self.t2 = _rand(s(synth.BETA), (H,), 0.0, 0.1, d)
+        self.g1 = _rand(s(synth.RESIDUAL), (H,), 0.0, 0.5, d)
+        self.g2 = _rand(s(synth.RESIDUAL + 1), (H,), 0.0, 0.5, d)
+        self.qkv = Linear(_rand(s(synth.W0), (2560, H), 0, 0.02, d))
+        self.o = Linear(_rand(s(synth.W0 + 1), (H, A), 0, 0.02, d))
+        self.gate_up = Linear(_rand(s(synth.W0 + 2), (2 * F, H), 0, 0.02, d), interleave_gate_up=True)
+        self.down = Linear(_rand(s(synth.W0 + 3), (H, F), 0, 0.02, d))
+        self.ws = ws or nvfp4.Workspace(d)
+        self.a1 = nvfp4.empty_fp4(M, H, d)
+        self.ctx_q = nvfp4.empty_fp4(M, A, d)
+        self.a2 = nvfp4.empty_fp4(M, H, d)
+        self.u = nvfp4.empty_fp4(M, F, d)
+        self.qkv_out = torch.empty((M, 2560), dtype=torch.bfloat16, device=d)
+        self.d_o = torch.empty((M, H), dtype=torch.bfloat16, device=d)
+        self.d_out = torch.empty((M, H), dtype=torch.bfloat16, device=d)
+
+    def linears(self):
+        return [self.qkv, self.o, self.gate_up, self.down]
+
+    def forward(self, r, d_in, g_in, context):
+        """r: bf16 [M, H] residual stream (updated in place); d_in, g_in: the previous layer's
+        down output and gate (d_in None: a plain AdaRMS front-end for the first layer)."""
+        if d_in is None:
+            nvfp4.quantize_norm(r, "adarms", scale=self.s1, shift=self.t1, eps=1e-6, out=self.a1)
+        else:
+            nvfp4.residual_quantize_norm(r, d_in, g_in, "adarms", scale=self.s1, shift=self.t1, eps=1e-6,
+                                         h_out=r, out=self.a1)
+        nvfp4.gemm(self.a1, self.qkv.w, "none", out=self.qkv_out, workspace=self.ws)
+        nvfp4.quantize_norm(context, "none", out=self.ctx_q)
+        nvfp4.gemm(self.ctx_q, self.o.w, "none", out=self.d_o, workspace=self.ws)
+        nvfp4.residual_quantize_norm(r, self.d_o, self.g1, "adarms", scale=self.s2, shift=self.t2, eps=1e-6,
+                                     h_out=r, out=self.a2)
+        nvfp4.gemm(self.a2, self.gate_up.w, "geglu", out=self.u, workspace=self.ws)
+        nvfp4.gemm(self.u, self.down.w, "none", out=self.d_out, workspace=self.ws)
+        return self.d_out, self.g2
 
     launches = 7
 
