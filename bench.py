@@ -508,6 +508,44 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                        "algorithmic_bytes_per_launch": tot_b // len(specs),
                        "kernel": "gemm_kernel (4 DiT GEMMs, M=41, L2-cold weights)", "peak_kind": pk_kind,
                        "per_gemm": per}
+    # ---- grouped GEMM: 32 cross-attention K/V projections of one M = 41 context in one
+    # launch; a ring of 4 groups with distinct weights (4 x 42.5 MB > L2) ----
+    with torch.cuda.stream(stream):
+        Kc, Nc, G = H, H, 32
+        ctxq = nvfp4.quantize_norm(synth.bf16_normal_torch(synth.seed_of(7, synth.CONTEXT), (M, Kc), device=dev),
+                                   "none")
+        groups, kv_outs = [], [torch.empty((M, Nc), dtype=torch.bfloat16, device=dev) for _ in range(G)]
+        kv_lins = []
+        for r in range(4):
+            ls = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(7, 3000 + 64 * r + g), (Nc, Kc), 0, 0.02,
+                                                        device=dev)) for g in range(G)]
+            kv_lins.append(ls)
+            groups.append(nvfp4.GroupedGemm([(ctxq, l.w, kv_outs[g]) for g, l in enumerate(ls)]))
+
+        def grouped():
+            for grp in groups:
+                grp.run()
+
+        def chained():
+            for ls in kv_lins:
+                for g, l in enumerate(ls):
+                    nvfp4.gemm(ctxq, l.w, "none", out=kv_outs[g], workspace=wsp)
+        grouped()
+        chained()
+    torch.cuda.synchronize()
+    g = capture(grouped, stream)
+    ms_g = time_graph(g, 20, stream) / len(groups)
+    del g
+    g = capture(chained, stream)
+    ms_c = time_graph(g, 20, stream) / len(groups)
+    del g
+    b_grp = G * gemm_bytes(M, Nc, Kc, "none")
+    out["grouped_cross_kv32"] = {"problems": f"{G} x {M}x{Nc}x{Kc}, shared context", "us": round(ms_g * 1e3, 2),
+                                 "gbs": round(b_grp / (ms_g * 1e-3) / 1e9, 1),
+                                 "frac_hbm": round(b_grp / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                                 "us_as_32_launches": round(ms_c * 1e3, 2), "bytes": b_grp,
+                                 "l2": "ring of 4 groups with distinct weights (170 MB > L2)"}
+    del groups, kv_lins, kv_outs, ctxq
     # ---- 18-layer action-expert stack (config 3 layers, one CUDA graph) ----
     with torch.cuda.stream(stream):
         ae = [layers.ActionExpertLayer(layer=i, device=dev, ws=wsp) for i in range(18)]

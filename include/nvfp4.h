@@ -288,7 +288,17 @@ typedef struct {
     /* FP4 output: of the norm op, or of a BIAS_GELU / GEGLU epilogue */
     uint8_t *out_codes, *out_sf;
     float out_global_scale;
+    /* The earlier op whose results this op reads (its input, and a GEMM's residual):
+     *   NVFP4_DEP_PREVIOUS (0, what a zeroed op gets): the op just before it;
+     *   NVFP4_DEP_NONE (-1): none -- its inputs are ready before the run starts;
+     *   j + 1, for 0 <= j < this op's index: op j.
+     * A run of ops with NVFP4_DEP_NONE is a grouped GEMM: one launch streams every op's
+     * weights with no wait between ops. */
+    int dep;
 } nvfp4_op;
+
+#define NVFP4_DEP_PREVIOUS 0
+#define NVFP4_DEP_NONE (-1)
 
 /* Host-side handle of a built program; the device data lives in `buffer`. */
 typedef struct {
@@ -298,21 +308,23 @@ typedef struct {
     int grid;
     int cluster;
     size_t ops_offset, maps_offset, done_offset;
+    int waits;  /* ops that wait for another op (0: the completion counters go unused) */
 } nvfp4_program;
 
 /* Device bytes a program of n_ops ops needs. */
 size_t nvfp4_program_bytes(int n_ops);
 
-/* Validates the ops (the rules of the standalone calls, plus: GEMM M <= 64, N % 64 == 0,
- * K % 32 == 0; norm K <= 4096, bf16 input), chooses each GEMM's schedule, encodes the TMA
+/* Validates the ops (the rules of the standalone calls, plus: at most 4096 ops (else
+ * NVFP4_ERR_UNSUPPORTED_SHAPE); GEMM M <= 64, N % 64 == 0, K % 32 == 0; norm K <= 4096, bf16
+ * input; each dep names an earlier op), chooses each GEMM's schedule, encodes the TMA
  * descriptors and copies the program into `buffer` (device, >= nvfp4_program_bytes(n_ops),
  * 256-byte aligned).  Synchronous (set-up time); the buffers the ops name must stay valid
  * for every later run. */
 nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes,
                                  nvfp4_program *prog);
 
-/* Runs the program on `stream`: zeroes its completion counters (cudaMemsetAsync) and makes
- * one cooperative launch.  Allocates nothing; capturable in a CUDA graph.  Runs of the same
+/* Runs the program on `stream`: zeroes its completion counters (cudaMemsetAsync; skipped
+ * when no op waits for another, as in a grouped GEMM) and makes one cooperative launch.  Allocates nothing; capturable in a CUDA graph.  Runs of the same
  * program must not overlap. */
 nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream);
 

@@ -1,0 +1,132 @@
+"""Grouped NVFP4 GEMM: independent problems in one executor launch ("GROOT N1.7 update: Thor
+NVFP4 + FA4 performance tier", §What is in the tier: the 32 per-frame cross-attention K/V
+projections run as NVFP4 GEMMs).  Every problem meets the GEMM bar against the oracle, the group agrees with the
+standalone calls, and op dependencies other than "the previous op" are honoured."""
+import numpy as np
+import pytest
+
+from parity import bf16_to_f64, check_gemm_bf16, dev_bf16, host, to_gpu_fp4
+from vla_action_head_b200 import nvfp4, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _probe():
+    nvfp4.probe()
+
+
+def _problem(orc, g, M, N, K, with_bias):
+    x = synth.bf16_normal(synth.seed_of(40 + g, synth.CONTEXT), (M, K))
+    w = synth.bf16_normal(synth.seed_of(40 + g, synth.W0), (N, K), 0.0, 0.02)
+    ac, asf = orc.quantize_norm(x, "none")
+    wc, wsf, gw = orc.quantize_weight(w)
+    bias = synth.bf16_normal(synth.seed_of(40 + g, synth.BIAS0), (N,), 0.0, 0.01) if with_bias else None
+    ref = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="bias" if with_bias else "none", bias=bias)
+    return x, (ac, asf), (wc, wsf, gw), bias, ref
+
+
+def _sync():
+    import torch
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_grouped_mixed_shapes_match_oracle(orc, with_bias):
+    """Problems of different M, N and K (tiles of 64 and 128 columns, ragged K) in one group."""
+    import torch
+    shapes = [(41, 1536, 1536), (50, 1024, 2048), (1, 512, 256), (64, 2560, 1024), (17, 256, 96),
+              (41, 3072, 1536), (33, 640, 4096)]
+    probs, refs = [], []
+    for g, (M, N, K) in enumerate(shapes):
+        _, (ac, asf), (wc, wsf, gw), bias, ref = _problem(orc, g, M, N, K, with_bias)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        probs.append((to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K), out,
+                      dev_bf16(bias) if with_bias else None))
+        refs.append(ref["v"])
+    grp = nvfp4.GroupedGemm(probs, epi="bias" if with_bias else "none")
+    grp.run()
+    _sync()
+    for g, (p, ref) in enumerate(zip(probs, refs)):
+        check_gemm_bf16(host(p[2]), ref, what=("grouped", g, shapes[g]))
+
+
+def test_grouped_cross_kv_32_matches_standalone(orc):
+    """32 projections of one shared context, as the K and V of 16 cross-attention layers;
+    checked against the oracle on a sample of problems and against the standalone GEMM on all."""
+    import torch
+    M, N, K, G = 41, 1536, 1536, 32
+    ctx = synth.bf16_normal(synth.seed_of(60, synth.CONTEXT), (M, K))
+    ac, asf = orc.quantize_norm(ctx, "none")
+    A = to_gpu_fp4(ac, asf, 1.0, M, K)
+    probs, refs = [], {}
+    for g in range(G):
+        w = synth.bf16_normal(synth.seed_of(60 + g, synth.W0), (N, K), 0.0, 0.02)
+        wc, wsf, gw = orc.quantize_weight(w)
+        if g in (0, 13, 31):
+            refs[g] = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="none")["v"]
+        probs.append((A, to_gpu_fp4(wc, wsf, gw, N, K), torch.empty((M, N), dtype=torch.bfloat16, device="cuda")))
+    grp = nvfp4.GroupedGemm(probs)
+    grp.run()
+    _sync()
+    for g, ref in refs.items():
+        check_gemm_bf16(host(probs[g][2]), ref, what=("cross-kv", g))
+    for g, (a, w, out) in enumerate(probs):
+        alone = nvfp4.gemm(a, w, "none")
+        _sync()
+        check_gemm_bf16(host(out), bf16_to_f64(host(alone)), what=("vs standalone", g))
+    # replays give the same bytes
+    first = [host(p[2]).copy() for p in probs]
+    for p in probs:
+        p[2].zero_()
+    grp.run()
+    _sync()
+    assert all(np.array_equal(host(p[2]), f) for p, f in zip(probs, first))
+
+
+def test_ops_depend_on_a_named_op(orc):
+    """A norm op, then GEMMs that all read its output (dep = op 0) and so wait for it, with a
+    GEMM reading another's output (dep = that op) at the end."""
+    import torch
+    M, K, N = 41, 1536, 1536
+    x = synth.bf16_normal(synth.seed_of(70, synth.X), (M, K))
+    gamma = synth.bf16_normal(synth.seed_of(70, synth.GAMMA), (K,), 1.0, 0.1)
+    beta = synth.bf16_normal(synth.seed_of(70, synth.BETA), (K,), 0.0, 0.1)
+    ac, asf = orc.quantize_norm(x, "layernorm", gamma=gamma, beta=beta, eps=1e-6)
+    a = nvfp4.empty_fp4(M, K)
+    ops = [nvfp4.op_norm(dev_bf16(x), a, "layernorm", gamma=dev_bf16(gamma), beta=dev_bf16(beta), eps=1e-6)]
+    outs, refs = [], []
+    for g in range(4):
+        w = synth.bf16_normal(synth.seed_of(71 + g, synth.W0), (N, K), 0.0, 0.02)
+        wc, wsf, gw = orc.quantize_weight(w)
+        refs.append(orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="none")["v"])
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        outs.append(out)
+        ops.append(nvfp4.op_gemm(a, to_gpu_fp4(wc, wsf, gw, N, K), "none", out=out, dep=0))
+    # residual read from op 1's output, which is three ops back
+    w = synth.bf16_normal(synth.seed_of(79, synth.W0), (N, K), 0.0, 0.02)
+    wc, wsf, gw = orc.quantize_weight(w)
+    last = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ops.append(nvfp4.op_gemm(a, to_gpu_fp4(wc, wsf, gw, N, K), "residual", residual=outs[0], out=last, dep=1))
+    prog = nvfp4.Program(ops)
+    prog.run()
+    _sync()
+    for g in range(4):
+        check_gemm_bf16(host(outs[g]), refs[g], what=("dep 0", g))
+    res_bits = host(outs[0])
+    ref_last = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="residual", residual=res_bits)["v"]
+    check_gemm_bf16(host(last), ref_last, what="dep 1 residual")
+
+
+def test_forward_dependency_is_rejected(orc):
+    import torch
+    M, N, K = 8, 256, 256
+    _, (ac, asf), (wc, wsf, gw), _, _ = _problem(orc, 0, M, N, K, False)
+    A, W = to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for dep in (0, 1, 5):  # itself, a later op, out of range
+        ops = [nvfp4.op_gemm(A, W, "none", out=out, dep=dep)] if dep == 0 else \
+              [nvfp4.op_gemm(A, W, "none", out=out), nvfp4.op_gemm(A, W, "none", out=out, dep=dep)]
+        with pytest.raises(nvfp4.NVFP4Error):
+            nvfp4.Program(ops)

@@ -584,6 +584,7 @@ size_t nvfp4_program_bytes(int n_ops) {
 
 nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes, nvfp4_program *prog) {
     if (ops == nullptr || n_ops <= 0 || buffer == nullptr || prog == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (n_ops > kExecMaxOps) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (bytes < nvfp4_program_bytes(n_ops)) return NVFP4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
     nvfp4_status st = check_device();
@@ -594,10 +595,35 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
 
     std::vector<CUtensorMap> maps(static_cast<size_t>(n_ops) * 2);
     std::vector<ExecOp> eops(static_cast<size_t>(n_ops));
+    int next_team = 0, waits = 0;
+    // Runs of two or more independent GEMM ops (a grouped GEMM) are scheduled for throughput:
+    // when the run has at least a tile per CTA, no op splits K (a split adds an exchange and
+    // an epilogue pass per unit and buys no parallelism the run does not already have).
+    std::vector<int> run_tiles(static_cast<size_t>(n_ops), 0);
+    for (int i = 0; i < n_ops;) {
+        auto grouped = [&](int k) { return ops[k].type == NVFP4_OP_GEMM && ops[k].dep == NVFP4_DEP_NONE; };
+        if (!grouped(i)) {
+            ++i;
+            continue;
+        }
+        int j = i, tiles = 0;
+        for (; j < n_ops && grouped(j); ++j) tiles += ops[j].N / (ops[j].N % 128 == 0 ? 128 : 64);
+        if (j - i >= 2)
+            for (int k = i; k < j; ++k) run_tiles[k] = tiles;
+        i = j;
+    }
     for (int i = 0; i < n_ops; ++i) {
         const nvfp4_op &o = ops[i];
         ExecOp &e = eops[i];
         std::memset(&e, 0, sizeof e);
+        if (o.dep == NVFP4_DEP_PREVIOUS) e.dep = i - 1;  // op 0 has none
+        else if (o.dep == NVFP4_DEP_NONE) e.dep = -1;
+        else if (o.dep >= 1 && o.dep <= i) e.dep = o.dep - 1;
+        else return NVFP4_ERR_INVALID_ARG;  // a later op, itself, or a bad code
+        if (e.dep >= 0) {
+            eops[static_cast<size_t>(e.dep)].signal = 1;
+            ++waits;
+        }
         if (o.type == NVFP4_OP_QUANTIZE_NORM) {
             if (o.M <= 0 || o.K <= 0 || o.x == nullptr || o.ldx < o.K) return NVFP4_ERR_INVALID_ARG;
             if (static_cast<int>(o.norm) < 0 || static_cast<int>(o.norm) > 4) return NVFP4_ERR_INVALID_ARG;
@@ -635,10 +661,14 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             // op in the fewest rounds with the shortest per-CTA K chain
             double best = 1e30;
             Schedule sc{64, 1, k_tiles, false};
+            if (run_tiles[i] >= grid) {
+                sc = finish(o.N % 128 == 0 ? 128 : 64, 1, o.K, false);
+                best = -1.0;  // fixed: skip the latency model below
+            }
             // Latency model (us) of one round at M <= 64: A load 0.8, MMA 0.7 per k-tile,
             // split exchange 0.8, epilogue 0.6 per pass of 128 threads over 32-column items.
             for (int bn : {128, 64}) {
-                if (o.N % bn != 0) continue;
+                if (o.N % bn != 0 || best < 0.0) continue;
                 for (int s : {1, 2, 4}) {
                     const Schedule c = finish(bn, s, o.K, false);
                     if (kExecCluster % c.splits != 0 || (bn / c.splits) % 32 != 0) continue;
@@ -666,6 +696,14 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             e.splits = sc.splits;
             e.kt_per_split = sc.kt_per_split;
             e.n_tiles = o.N / sc.block_n;
+            {
+                // rotate the op's first tile to the team after the previous GEMM's last one, so
+                // a run of small ops spreads over the whole grid instead of its first teams
+                const int per_team = kExecCluster / e.splits;
+                const int used = std::min(teams, (e.n_tiles + per_team - 1) / per_team);
+                e.team0 = next_team;
+                next_team = (next_team + used) % teams;
+            }
             e.units = static_cast<unsigned>(e.n_tiles * e.splits);  // every CTA of a group signals its slice
             e.a_box_rows = static_cast<uint32_t>((o.M + 7) / 8 * 8);
             e.sfa = o.A.sf;
@@ -706,6 +744,7 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
     prog->maps_offset = 0;
     prog->ops_offset = maps_bytes;
     prog->done_offset = maps_bytes + ops_bytes;
+    prog->waits = waits;
     return NVFP4_OK;
 }
 
@@ -721,7 +760,8 @@ nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream)
     if (device_status_address(&p.status) != cudaSuccess) return NVFP4_ERR_CUDA;
     p.trace = (g_trace != nullptr && g_trace_words >= static_cast<size_t>(prog->n_ops) * prog->grid * 8) ? g_trace
                                                                                                           : nullptr;
-    cudaError_t e = cudaMemsetAsync(p.done, 0, static_cast<size_t>(prog->n_ops) * 4, stream);
+    cudaError_t e = prog->waits > 0 ? cudaMemsetAsync(p.done, 0, static_cast<size_t>(prog->n_ops) * 4, stream)
+                                     : cudaSuccess;
     if (e == cudaSuccess) e = exec_launch(p, prog->grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return from_cuda(e);

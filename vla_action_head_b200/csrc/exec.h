@@ -15,8 +15,13 @@ enum { kOpNorm = 0, kOpGemm = 1 };
 
 // One op of a program, in device memory.  Ops run in program order: op i starts consuming
 // its inputs once done[i - 1] reached ops[i - 1].units (every op depends on the previous one).
+// Most ops a program may hold (the executor keeps one bit per op in shared memory).
+constexpr int kExecMaxOps = 4096;
+
 struct ExecOp {
     int type;
+    int dep;             // index of the op whose completion this op waits for, -1 for none
+    int signal;          // 1 if a later op waits for this one (its units count into done[i])
     unsigned int units;  // done[i] value when the op is complete (norm: rows; GEMM: tiles)
     // ---- norm -> FP4 (one warp per row) ----
     NormArgs norm;
@@ -25,6 +30,7 @@ struct ExecOp {
     int tm_a, tm_b;  // indices into the tensor-map table
     int M, N, K, k_atoms, k_tiles;
     int bn, splits, kt_per_split, n_tiles;
+    int team0;  // the team that takes the op's first tile (ops start where the last left off)
     uint32_t a_box_rows;
     const uint8_t *sfa, *sfb;
     float alpha;

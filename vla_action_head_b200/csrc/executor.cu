@@ -8,19 +8,24 @@
 // the consumers), and the weight tiles of later ops stream into each CTA's shared-memory
 // ring while the current op waits for its input -- weights never depend on activations.
 //
-// Roles (224 threads):
+// Roles (256 threads):
 //   warp 0      weight producer: TMA loads of W code tiles + bulk loads of their scale
 //               atoms, for every GEMM unit of this CTA in program order, as far ahead as the
 //               ring allows.
-//   warp 1      MMA issuer: tcgen05.cp of the scales, tcgen05.mma kind::mxf4nvf4 block16
-//               into one of two TMEM accumulators.
+//   warp 1      MMA issuer: tcgen05.mma kind::mxf4nvf4 block16 into one of two TMEM
+//               accumulators.
+//   warp 7      scale copier: tcgen05.cp of each stage's scale atoms into one of two TMEM
+//               scale slots, a stage ahead of the MMAs (copies issued by the MMA thread itself
+//               would run one after another between its MMAs).
 //   warp 2      activation producer: waits until the op's input is complete, then TMA loads
 //               the A code tiles + scale atoms into the same ring stages.
 //   warps 3..6  epilogue and norm workers: TMEM -> registers -> fused epilogue; split-K
 //               partials are added on the tile's owner CTA over distributed shared memory
 //               in split order (deterministic); norm ops run one row per warp.
 // GEMM work: the grid is a set of clusters of C CTAs; for an op split S ways (S | C), the
-// S CTAs that share a tile are cluster neighbours.
+// S CTAs that share a tile are cluster neighbours.  At start each CTA marks, in a shared-memory
+// bit set, the ops it has work in; the roles walk only those (a grouped GEMM of many small
+// independent ops gives each CTA a few of them).
 // Every wait is bounded (2 s); an expired wait records a device status and unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -36,7 +41,7 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kThreads = 224;
+constexpr int kThreads = 256;
 constexpr int kRing = 6;
 constexpr int kStageA = 8192;   // 64 rows x 128 bytes (M <= 64)
 constexpr int kStageW = 16384;  // 128 rows x 128 bytes (block_n <= 128)
@@ -52,15 +57,17 @@ constexpr int kOffStg = kOffRed + kRedBytes;
 constexpr int kStgBytes = 64 * kStgLd * 2;
 constexpr int kOffStgBias = kOffStg + kStgBytes;
 constexpr int kOffBar = kOffStgBias + 256;
-// barriers: full[R], empty[R], acc_full[2], acc_empty[2]
-constexpr int kOffMisc = kOffBar + (2 * kRing + 4) * 8;
+// barriers: full[R], empty[R], acc_full[2], acc_empty[2], sf_ready[2], sf_free[2]
+constexpr int kOffMisc = kOffBar + (2 * kRing + 8) * 8;
 // misc words: [0] TMEM base, [1] abort flag, [2] red_in (partials received as owner),
 // [3] red_free (frees received as member)
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;
-constexpr int kTmemCols = 512;  // two 128-column accumulators + scale columns
-constexpr int kColSfa = 256;
-constexpr int kColSfb = 272;
+constexpr int kOffMask = kOffMisc + 64;  // one bit per op: this CTA has work in it
+constexpr int kSmemBytes = kOffMask + kExecMaxOps / 8 + 1024;
+constexpr int kTmemCols = 512;  // two 128-column accumulators + two scale slots
+constexpr int kColSf = 256;     // scale slot j: A atoms at kColSf + 32 j, W atoms 16 columns on
+constexpr int kSfSlot = 32;
 constexpr int kSfAtom = 512;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
     unsigned int v;
@@ -136,7 +143,8 @@ __device__ __forceinline__ int op_rounds(const ExecOp &op, int teams, int C) {
 // The GEMM unit of (team, rank) in round r, if any.
 __device__ __forceinline__ bool op_unit(const ExecOp &op, int team, int rank, int teams, int C, int r, Unit &u) {
     const int per_team = C / op.splits;
-    const int tile = (r * teams + team) * per_team + rank / op.splits;
+    const int t = team >= op.team0 ? team - op.team0 : team - op.team0 + teams;  // rotated team index
+    const int tile = (r * teams + t) * per_team + rank / op.splits;
     if (tile >= op.n_tiles) return false;
     u.tile = tile;
     u.split = rank % op.splits;
@@ -144,6 +152,22 @@ __device__ __forceinline__ bool op_unit(const ExecOp &op, int team, int rank, in
     u.kt1 = min(op.k_tiles, u.kt0 + op.kt_per_split);
     u.owner_rank = (rank / op.splits) * op.splits;
     return true;
+}
+
+// Whether CTA (team, rank) has any work in op i: a norm row, or a GEMM unit in round 0
+// (later rounds only add tiles to CTAs that have one in round 0).
+__device__ __forceinline__ bool has_work(const ExecOp &op, int team, int rank, int teams, int C) {
+    if (op.type == kOpNorm) return static_cast<int>(blockIdx.x) * 4 < op.norm.M;
+    Unit u;
+    return op_unit(op, team, rank, teams, C, 0, u);
+}
+// The first op after op i that this CTA has work in (n_ops if none).
+__device__ __forceinline__ int next_op(const uint32_t *mask, int n_ops, int i) {
+    for (int j = i + 1; j < n_ops; j = (j | 31) + 1) {
+        const uint32_t bits = mask[j >> 5] >> (j & 31);
+        if (bits != 0u) return j + __ffs(static_cast<int>(bits)) - 1;
+    }
+    return n_ops;
 }
 
 // Kept out of line: the norm path has its own register allocation, apart from the
@@ -173,6 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     const uint32_t bar_empty = bar_full + 8 * kRing;
     const uint32_t bar_accf = bar_empty + 8 * kRing;
     const uint32_t bar_acce = bar_accf + 16;
+    const uint32_t bar_sfr = bar_acce + 16;  // 2: scale slot copied
+    const uint32_t bar_sff = bar_sfr + 16;   // 2: scale slot read by its MMAs
+    uint32_t *opmask = reinterpret_cast<uint32_t *>(smem + kOffMask);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
     const uint32_t red_in_addr = sbase + kOffMisc + 8;
@@ -192,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
             mbar_init(bar_acce + 8 * b, 1);
+            mbar_init(bar_sfr + 8 * b, 1);
+            mbar_init(bar_sff + 8 * b, 1);
         }
         misc[1] = 0;
         misc[2] = 0;
@@ -201,6 +230,13 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     if (warp == 1) {
         tmem_alloc(smem_u32(const_cast<uint32_t *>(misc)), kTmemCols);
         tmem_relinquish();
+    }
+    // the ops this CTA has work in: one bit per op, 32 ops per warp ballot
+    for (int w = warp; w < (P.n_ops + 31) / 32; w += kThreads / 32) {
+        const int i = 32 * w + lane;
+        const bool mine = i < P.n_ops && has_work(P.ops[i], team, rank, teams, C);
+        const uint32_t bits = __ballot_sync(0xffffffffu, mine);
+        if (lane == 0) opmask[w] = bits;
     }
     tc_fence_before();
     __syncthreads();
@@ -220,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         // ---------------------------- weight producer ----------------------------
         const uint64_t pol = policy_evict_first();
         int step = 0;
-        for (int i = 0; i < P.n_ops; ++i) {
+        for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
             const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmB = P.maps + op.tm_b;
@@ -250,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         // ---------------------------- activation producer ----------------------------
         const uint64_t pol = policy_evict_last();
         int step = 0;
-        for (int i = 0; i < P.n_ops; ++i) {
+        for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
             const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmA = P.maps + op.tm_a;
@@ -260,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 Unit u;
                 if (!op_unit(op, team, rank, teams, C, r, u)) continue;
                 if (!ready) {
-                    if (i > 0 && !wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status)) goto done_a;
+                    if (op.dep >= 0 && !wait_counter(P.done + op.dep, P.ops[op.dep].units, abort_flag, P.status)) goto done_a;
                     fence_proxy_async_global();  // the input was written through the generic proxy
                     ready = true;
                     stamp(i, 1);
@@ -282,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     } else if (warp == 1 && lane == 0) {
         // ---------------------------- MMA issuer ----------------------------
         int step = 0, unit_idx = 0;
-        for (int i = 0; i < P.n_ops; ++i) {
+        for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
             const ExecOp op = P.ops[i];
             if (op.type != kOpGemm) continue;
             const uint32_t idesc = idesc_mxf4nvf4(128, op.bn);
@@ -299,24 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 // a 64-row W tile reads its half of the 128-row scale atom
                 const uint32_t sub = (op.bn == 64) ? static_cast<uint32_t>(((u.tile * op.bn) & 127) >> 5) : 0u;
                 for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
-                    const int slot = step % kRing, use = step / kRing;
-                    if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
+                    const int slot = step % kRing, use = step / kRing, sfs = step & 1;
+                    if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull) ||
+                        !mbar_wait(bar_sfr + 8 * sfs, (step >> 1) & 1, abort_flag, P.status, kStatusTimeoutFull))
                         goto done_m;
                     tc_fence_after();
                     if (kt == u.kt0) stamp(i, 2);
                     const int nkb = nkb_of(op, kt);
                     const uint32_t st = sbase + slot * kStage;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * kb,
-                                             desc_sf_32x128b(st + kStageA + kStageW + kb * kSfAtom));
-                        tc_cp_32x128b_warpx4(tmem + kColSfb + 4 * kb,
-                                             desc_sf_32x128b(st + kStageA + kStageW + kStageSfa + kb * kSfAtom));
-                    }
+                    const uint32_t t_sf = tmem + kColSf + sfs * kSfSlot;
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_mxf4nvf4(t_acc, desc_kmajor_sw128(st + 32 * kb), desc_kmajor_sw128(st + kStageA + 32 * kb),
-                                        idesc, tmem + kColSfa + 4 * kb, tmem + kColSfb + 4 * kb + sub,
-                                        (kt > u.kt0 || kb > 0) ? 1u : 0u);
-                    tc_commit(bar_empty + 8 * slot);
+                                        idesc, t_sf + 4 * kb, t_sf + 16 + 4 * kb + sub, (kt > u.kt0 || kb > 0) ? 1u : 0u);
+                    tc_commit(bar_empty + 8 * slot);  // the stage, once these MMAs have read it
+                    tc_commit(bar_sff + 8 * sfs);     // and the scale slot
                 }
                 stamp(i, 3);
                 tc_commit(bar_accf + 8 * b);
@@ -324,6 +356,41 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
             }
         }
     done_m:;
+    } else if (warp == 7) {
+        if (lane == 0) {
+            // ---------------------------- scale copier ----------------------------
+            // Same walk of k-tile steps as the MMA issuer; step s uses scale slot s & 1, free
+            // again once the MMAs of step s - 2 have completed.
+            int step = 0;
+            for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
+                const ExecOp op = P.ops[i];
+                if (op.type != kOpGemm) continue;
+                const int rounds = op_rounds(op, teams, C);
+                for (int r = 0; r < rounds; ++r) {
+                    Unit u;
+                    if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                    for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
+                        const int slot = step % kRing, use = step / kRing, sfs = step & 1;
+                        if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
+                            goto done_c;
+                        if (step >= 2 && !mbar_wait(bar_sff + 8 * sfs, ((step >> 1) - 1) & 1, abort_flag, P.status,
+                                                    kStatusTimeoutFull))
+                            goto done_c;
+                        tc_fence_after();
+                        const int nkb = nkb_of(op, kt);
+                        const uint32_t st = sbase + slot * kStage;
+                        const uint32_t t_sf = tmem + kColSf + sfs * kSfSlot;
+                        for (int kb = 0; kb < nkb; ++kb) {
+                            tc_cp_32x128b_warpx4(t_sf + 4 * kb, desc_sf_32x128b(st + kStageA + kStageW + kb * kSfAtom));
+                            tc_cp_32x128b_warpx4(t_sf + 16 + 4 * kb,
+                                                 desc_sf_32x128b(st + kStageA + kStageW + kStageSfa + kb * kSfAtom));
+                        }
+                        tc_commit(bar_sfr + 8 * sfs);  // arrives once the copies have landed
+                    }
+                }
+            }
+        done_c:;
+        }
     } else if (warp >= 3) {
         // ---------------------------- epilogue / norm workers ----------------------------
         const int e = threadIdx.x - 96;  // 0..127
@@ -332,18 +399,18 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         const int row = q * 32 + lane;
         int unit_idx = 0;
         unsigned int in_expected = 0, free_expected = 0;  // split-group signals expected so far
-        for (int i = 0; i < P.n_ops; ++i) {
+        for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
             const ExecOp op = P.ops[i];
             if (op.type == kOpNorm) {
                 const int rows_per_round = gridDim.x * 4;
                 if (blockIdx.x * 4 >= op.norm.M) continue;  // no rows for this CTA
-                const bool ok = (e != 0) || i == 0 || wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status);
+                const bool ok = (e != 0) || op.dep < 0 || wait_counter(P.done + op.dep, P.ops[op.dep].units, abort_flag, P.status);
                 if (!bar_epi_and(ok)) goto done_e;
                 if (e == 0) stamp(i, 1);
                 for (int rr = blockIdx.x * 4 + ew; rr < op.norm.M; rr += rows_per_round) {
                     norm_row_any(op.norm, op.bpt, rr, lane);
                     __syncwarp();
-                    if (lane == 0) {
+                    if (lane == 0 && op.signal) {
                         __threadfence();
                         atomicAdd(P.done + i, 1u);
                     }
@@ -372,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 if (!dep_seen) {
                     // the epilogue reads residuals written by earlier ops: acquire here too
                     const bool ok =
-                        (e != 0) || i == 0 || wait_counter(P.done + (i - 1), P.ops[i - 1].units, abort_flag, P.status);
+                        (e != 0) || op.dep < 0 || wait_counter(P.done + op.dep, P.ops[op.dep].units, abort_flag, P.status);
                     if (!bar_epi_and(ok)) goto done_e;
                     dep_seen = true;
                 }
@@ -489,8 +556,10 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                         for (int sp = 0; sp < S; ++sp)
                             red_add_release_cluster(
                                 mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
-                    __threadfence();
-                    atomicAdd(P.done + i, 1u);
+                    if (op.signal) {  // only ops that a later op waits for count completions
+                        __threadfence();
+                        atomicAdd(P.done + i, 1u);
+                    }
                     stamp(i, 6);
                 }
                 if (S > 1) free_expected += static_cast<unsigned>(S);

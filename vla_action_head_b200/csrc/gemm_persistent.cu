@@ -59,14 +59,18 @@ struct PCfg {
     static constexpr int kStage = kOffSfb + kStageSfb;  // 54 KB (BN 256) / 36 KB (BN 128)
     static constexpr int kStages = (216 * 1024) / kStage;
     static constexpr int kOffBar = kStages * kStage;
-    // barriers: full[kStages], empty[kStages], acc_full, acc_empty, sf_ready[2], sf_free[2]
-    static constexpr int kOffMisc = kOffBar + (2 * kStages + 6) * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-    // scale columns: two slots (stage parity) of [A: 4 k-blocks x 4 | W: 4 k-blocks x groups x 4]
+    // scale columns: kSlots slots (step modulo kSlots) of [A: 4 k-blocks x 4 | W: 4 k-blocks x
+    // groups x 4]; the copies of a step may run up to kSlots - 1 steps ahead of its MMAs
+    static constexpr int kSlots = 2;
     static constexpr int kColSf = BN;
     static constexpr int kSfSlot = 16 + 16 * kGroups;
-    static constexpr int kTmemCols = (kColSf + 2 * kSfSlot) <= 256 ? 256 : 512;
+    static constexpr int kTmemCols = (kColSf + kSlots * kSfSlot) <= 256 ? 256 : 512;
+    // barriers: full[kStages], empty[kStages], acc_full, acc_empty, sf_ready[kSlots],
+    // sf_free[kSlots], sf_full[kStages]
+    static constexpr int kOffMisc = kOffBar + (3 * kStages + 2 + 2 * kSlots) * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
+    static_assert(kColSf + kSlots * kSfSlot <= kTmemCols, "tensor memory columns");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using Cf = PCfg<BN>;
     constexpr int kStages = Cf::kStages, kStage = Cf::kStage, kStageA = Cf::kStageA, kStageB = Cf::kStageB;
     constexpr int kOffB = Cf::kOffB, kOffSfa = Cf::kOffSfa, kOffSfb = Cf::kOffSfb, kGroups = Cf::kGroups;
-    constexpr int kColSf = Cf::kColSf, kSfSlot = Cf::kSfSlot, kTmemCols = Cf::kTmemCols;
+    constexpr int kColSf = Cf::kColSf, kSfSlot = Cf::kSfSlot, kTmemCols = Cf::kTmemCols, kSlots = Cf::kSlots;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -105,8 +109,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_empty = bar_full + 8 * kStages;
     const uint32_t bar_accf = bar_empty + 8 * kStages;
     const uint32_t bar_acce = bar_accf + 8;
-    const uint32_t bar_sfr = bar_acce + 8;  // 2: scale slot copied (one arrival per copier warp)
-    const uint32_t bar_sff = bar_sfr + 16;  // 2: scale slot read by its MMAs
+    const uint32_t bar_sfr = bar_acce + 8;            // kSlots: slot copied (an arrival per copier)
+    const uint32_t bar_sff = bar_sfr + 8 * kSlots;    // kSlots: slot read by its MMAs
+    const uint32_t bar_sfl = bar_sff + 8 * kSlots;    // kStages: the stage's scale atoms have landed
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + Cf::kOffMisc);  // [0] TMEM base, [1] abort
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
@@ -123,10 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_sfl + 8 * s, 1);
         }
         mbar_init(bar_accf, 1);
         mbar_init(bar_acce, 1);
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < kSlots; ++j) {
             mbar_init(bar_sfr + 8 * j, kCopiers);
             mbar_init(bar_sff + 8 * j, 1);
         }
@@ -151,31 +157,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------ producer (whole warp) ------------------------------
         const uint64_t pol = policy_evict_last();  // A and W both fit in L2 and are re-read
+        // The scale atoms complete on their own barrier (sf_full) and are issued before the code
+        // tiles: the copiers move them into tensor memory while the 48 KB of codes still land.
         auto expect = [&](int st) {
             const int nkb = nkb_of(st % k_tiles);
-            const uint32_t bytes = kStageA + kStageB + static_cast<uint32_t>(nkb) * (1u + kGroups) * kSfAtom;
-            if (lane == 0) mbar_arrive_expect_tx(bar_full + 8 * (st % kStages), bytes);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar_sfl + 8 * (st % kStages), static_cast<uint32_t>(nkb) * (1u + kGroups) * kSfAtom);
+                mbar_arrive_expect_tx(bar_full + 8 * (st % kStages), kStageA + kStageB);
+            }
             __syncwarp();
         };
         auto issue_w = [&](int st) {
             const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
             const int n_tile = t / m_tiles, nkb = nkb_of(kt);
-            const uint32_t full = bar_full + 8 * s, base = sbase + s * kStage;
-            if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * BN, full, pol);
+            const uint32_t full = bar_full + 8 * s, sfl = bar_sfl + 8 * s, base = sbase + s * kStage;
             if (lane < kGroups) {  // the k-blocks' atoms of each 128-row group are contiguous
                 const size_t grp = static_cast<size_t>(n_tile) * kGroups + lane;
                 bulk_load(base + kOffSfb + lane * 4 * kSfAtom, p.sfb + (grp * p.k_atoms + 4 * kt) * kSfAtom,
-                          static_cast<uint32_t>(nkb) * kSfAtom, full, pol);
+                          static_cast<uint32_t>(nkb) * kSfAtom, sfl, pol);
             }
+            __syncwarp();
+            if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * BN, full, pol);
         };
         auto issue_a = [&](int st) {
             const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
             const int m_tile = t % m_tiles, nkb = nkb_of(kt);
-            const uint32_t full = bar_full + 8 * s, base = sbase + s * kStage;
+            const uint32_t full = bar_full + 8 * s, sfl = bar_sfl + 8 * s, base = sbase + s * kStage;
             if (lane == 0) {
-                tma_load_2d(base, &tmA, kt * 128, m_tile * 128, full, pol);
                 bulk_load(base + kOffSfa, p.sfa + (static_cast<size_t>(m_tile) * p.k_atoms + 4 * kt) * kSfAtom,
-                          static_cast<uint32_t>(nkb) * kSfAtom, full, pol);
+                          static_cast<uint32_t>(nkb) * kSfAtom, sfl, pol);
+                tma_load_2d(base, &tmA, kt * 128, m_tile * 128, full, pol);
             }
         };
         const int pre = min(kStages, steps);
@@ -199,8 +210,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // every issued stage must have landed before the CTA may exit
         if (lane == 0)
-            for (int st = max(0, issued - kStages); st < issued; ++st)
+            for (int st = max(0, issued - kStages); st < issued; ++st) {
                 drain_wait(bar_full + 8 * (st % kStages), (st / kStages) & 1, p.status);
+                drain_wait(bar_sfl + 8 * (st % kStages), (st / kStages) & 1, p.status);
+            }
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------ MMA issuer ------------------------------
@@ -212,9 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < k_tiles; ++kt, ++st) {
-                    const int s = st % kStages, slot = st & 1;
+                    const int s = st % kStages, slot = st % kSlots;
                     if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull) ||
-                        !mbar_wait(bar_sfr + 8 * slot, (st >> 1) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
+                        !mbar_wait(bar_sfr + 8 * slot, (st / kSlots) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
                         ok = false;
                         break;
                     }
@@ -241,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Copier c takes k-blocks 2c and 2c + 1 of every stage.
             const int c = warp - 10;
             for (int st = 0; st < steps; ++st) {
-                const int s = st % kStages, slot = st & 1, kt = st % k_tiles;
-                if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull))
+                const int s = st % kStages, slot = st % kSlots, kt = st % k_tiles;
+                if (!mbar_wait(bar_sfl + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull))
                     break;
-                if (st >= 2 && !mbar_wait(bar_sff + 8 * slot, ((st >> 1) - 1) & 1, abort_flag, p.status,
+                if (st >= kSlots && !mbar_wait(bar_sff + 8 * slot, (st / kSlots - 1) & 1, abort_flag, p.status,
                                           kStatusTimeoutFull))
                     break;
                 tc_fence_after();

@@ -43,13 +43,14 @@ class _Op(C.Structure):
                 ("mod_shift", C.c_void_p), ("eps", C.c_float),
                 ("A", _Tensor), ("W", _Tensor), ("epi", C.c_int), ("bias", C.c_void_p),
                 ("residual", C.c_void_p), ("ldr", C.c_int), ("out_bf16", C.c_void_p), ("ldo", C.c_int),
-                ("out_codes", C.c_void_p), ("out_sf", C.c_void_p), ("out_global_scale", C.c_float)]
+                ("out_codes", C.c_void_p), ("out_sf", C.c_void_p), ("out_global_scale", C.c_float),
+                ("dep", C.c_int)]
 
 
 class _Program(C.Structure):
     _fields_ = [("buffer", C.c_void_p), ("bytes", C.c_size_t), ("n_ops", C.c_int), ("grid", C.c_int),
                 ("cluster", C.c_int), ("ops_offset", C.c_size_t), ("maps_offset", C.c_size_t),
-                ("done_offset", C.c_size_t)]
+                ("done_offset", C.c_size_t), ("waits", C.c_int)]
 
 
 _lib = None
@@ -276,21 +277,36 @@ def device_status():
 
 
 # ---- layer executor ----------------------------------------------------------------------
-def op_norm(x, out: NVFP4Tensor, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6):
-    """A norm -> FP4 op of a program (bf16 x [M, K] -> out)."""
+def _dep(dep):
+    """"previous" (the op before), None (no wait) or the index of an earlier op."""
+    if dep == "previous":
+        return 0
+    if dep is None:
+        return -1
+    if isinstance(dep, int) and dep >= 0:
+        return dep + 1
+    raise ValueError(f"dep must be 'previous', None or an op index, got {dep!r}")
+
+
+def op_norm(x, out: NVFP4Tensor, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
+            dep="previous"):
+    """A norm -> FP4 op of a program (bf16 x [M, K] -> out); `dep` names the op it waits for."""
     M, K = x.shape
     op = _Op(type=0, M=M, N=0, K=K, x=x.data_ptr(), ldx=x.stride(0), norm=NORM[kind],
              gamma=_ptr(gamma), beta=_ptr(beta), mod_scale=_ptr(scale), mod_shift=_ptr(shift), eps=eps,
-             out_codes=out.codes.data_ptr(), out_sf=out.sf.data_ptr(), out_global_scale=out.global_scale)
+             out_codes=out.codes.data_ptr(), out_sf=out.sf.data_ptr(), out_global_scale=out.global_scale,
+             dep=_dep(dep))
     op.keep = (x, out, gamma, beta, scale, shift)  # the program only holds raw pointers
     return op
 
 
-def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None, out_global_scale=1.0):
-    """A GEMM op of a program; `out` is bf16 [M, N] or, for FP4 epilogues, an NVFP4Tensor."""
+def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None, out_global_scale=1.0,
+            dep="previous"):
+    """A GEMM op of a program; `out` is bf16 [M, N] or, for FP4 epilogues, an NVFP4Tensor;
+    `dep` names the op whose results it reads ("previous", None or an op index)."""
     e = EPI[epi]
     op = _Op(type=1, M=a.rows, N=w.rows, K=a.K, A=a.c(), W=w.c(), epi=e, bias=_ptr(bias),
-             residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0)
+             residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0, dep=_dep(dep))
     if e in (4, 5):
         op.out_codes, op.out_sf, op.out_global_scale = out.codes.data_ptr(), out.sf.data_ptr(), out_global_scale
     else:
@@ -317,3 +333,17 @@ class Program:
 
     def run(self):
         _check("nvfp4_program_run", lib().nvfp4_program_run(C.byref(self.prog), _stream()))
+
+
+class GroupedGemm(Program):
+    """A grouped NVFP4 GEMM: independent problems (a_g, w_g, out_g[, bias_g]) of M <= 64 rows,
+    all run by one launch that streams every problem's weights back to back with no wait
+    between problems.  Problems may differ in N and K; each takes the same epilogue kind."""
+
+    def __init__(self, problems, epi="none", device="cuda"):
+        ops = []
+        for pr in problems:
+            a, w, out = pr[0], pr[1], pr[2]
+            bias = pr[3] if len(pr) > 3 else None
+            ops.append(op_gemm(a, w, epi, bias=bias, out=out, dep=None))
+        super().__init__(ops, device=device)
