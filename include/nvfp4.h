@@ -135,6 +135,14 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * rows done (norm ops) or accumulator drained to shared memory (GEMM ops). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
+/* Schedule option for the default (block_n = 0, splits = 0) schedule at M > 128: whether the
+ * CTA-pair kernel (256 x 256 tiles on 2-CTA clusters, tcgen05 cta_group::2; N % 256 == 0)
+ * may run.  -1: where its cost model prefers it; 0: never (the initial value, unless the
+ * environment variable NVFP4_GEMM_PAIR is 1); 1: wherever N % 256 == 0.  Results are the
+ * same either way (the same per-element fp32 sums).  Host-side state, not thread safe.
+ * NVFP4_ERR_INVALID_ARG for other values. */
+nvfp4_status nvfp4_set_pair_mode(int mode);
+
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
 
 /* Per row of x [M, K] (leading dimension ldx, bf16 or fp32): the norm `kind`, then the

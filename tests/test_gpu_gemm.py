@@ -124,20 +124,51 @@ def test_device_status_clean():
     nvfp4.device_status()
 
 
-# The default schedule for many rows with N % 256 == 0 runs the persistent kernel (one CTA
-# per SM walks the tiles; the scale factors go to TMEM through 128x256b copies of
-# replicated images); explicit (256, 1) runs the one-tile-per-CTA kernel.
+# The default schedule for many rows runs a persistent kernel: one CTA per SM walking
+# 128 x 256 or 128 x 128 tiles, or (N % 256 == 0) CTA pairs walking 256 x 256 tiles with
+# tcgen05 cta_group::2.  pair_mode pins which one; explicit (block_n, splits) runs the
+# one-tile-per-CTA kernel.
+@pytest.fixture(params=[0, 1], ids=["one_cta", "cta_pair"])
+def pair_mode(request):
+    nvfp4.set_pair_mode(request.param)
+    yield request.param
+    nvfp4.set_pair_mode(0)
+
+
 @pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
 @pytest.mark.parametrize("N,rows", [(512, None), (10240, [0, 5, 127, 128, 255, 256, 299])])
-def test_persistent_epilogues(orc, epi, N, rows):
-    """N = 512 runs 128-wide tiles (12 of them); N = 10240 runs 256-wide ones (120)."""
+def test_persistent_epilogues(orc, pair_mode, epi, N, rows):
+    """One CTA per tile: N = 512 runs 128-wide tiles (12 of them), N = 10240 256-wide ones
+    (120).  CTA pairs: 4 and 80 tiles of 256 x 256; the last pair's second CTA holds no
+    valid row (M = 300)."""
     _run(orc, 300, N, 768, epi, rows=rows)
 
 
-def test_persistent_multi_tile_and_tails(orc):
-    """More tiles than SMs (each CTA walks several), the M tail of 968 = 7 * 128 + 72, and
-    a last K tile with an odd number of 64-wide blocks (K = 4160)."""
+def test_persistent_multi_tile_and_tails(orc, pair_mode):
+    """More tiles than SMs (each CTA or pair walks several), the M tail of 968 = 7 * 128 + 72,
+    and a last K tile with an odd number of 64-wide blocks (K = 4160)."""
     rows = [0, 1, 63, 127, 128, 500, 767, 895, 896, 900, 960, 967]
     _run(orc, 968, 5120, 1024, "none", rows=rows)
     _run(orc, 968, 2048, 4160, "residual", rows=rows)
     _run(orc, 968, 4096, 512, "geglu", rows=rows)
+
+
+def test_pair_and_one_cta_agree(orc):
+    """The two many-row kernels give the same bytes (same per-element fp32 sums)."""
+    import torch
+    M, N, K = 700, 1024, 1536
+    x = synth.bf16_normal(synth.seed_of(35, synth.X), (M, K))
+    w = synth.bf16_normal(synth.seed_of(35, synth.W0), (N, K), 0.0, 0.02)
+    ac, asf = orc.quantize_norm(x, "none")
+    wc, wsf, gw = orc.quantize_weight(w)
+    A, W = to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+    outs = []
+    for mode in (0, 1):
+        nvfp4.set_pair_mode(mode)
+        try:
+            outs.append(host(nvfp4.gemm(A, W, "none")))
+            torch.cuda.synchronize()
+            nvfp4.device_status()
+        finally:
+            nvfp4.set_pair_mode(0)
+    assert np.array_equal(outs[0], outs[1])

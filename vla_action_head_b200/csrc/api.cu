@@ -76,6 +76,21 @@ bool make_code_map(CUtensorMap *m, const void *ptr, int rows, int row_bytes, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scale atoms (512 bytes each: 128 rows x 4 k-blocks) as a 2-D array of 16-bit words,
+// `atoms` rows of 256; the box is 4 consecutive atoms (a 256-wide K tile of one 128-row
+// group).  Rows past the array read as zeros.
+bool make_sf_map(CUtensorMap *m, const void *ptr, int atoms) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {256u, static_cast<cuuint64_t>(atoms)};
+    cuuint64_t strides[1] = {512u};
+    cuuint32_t box[2] = {256u, 4u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 unsigned long long *g_trace = nullptr;  // diagnostics: per-CTA GEMM timestamps
 size_t g_trace_words = 0;
 size_t g_trace_cursor = 0;
@@ -155,7 +170,20 @@ Schedule choose(int M, int N, int K) {
 // Tile width of the persistent kernel for many rows (0: not applicable).  A 128-wide tile
 // costs about 0.72 of a 256-wide one (more scale copies per FLOP), so 128 wins when 256-wide
 // tiles would leave SMs idle, e.g. N = 2048 at M = 968 (64 tiles on 148 SMs).
+// The many-row schedule: 256 or 128 = the one-CTA persistent kernel with that tile width,
+// kPairTiles = 256 x 256 tiles on CTA pairs.  Cost: waves x the relative time of a wave
+// (a 128-wide tile does half the work of a 256-wide one for 0.72 of its time: the wider
+// tile is bound by shared-memory traffic, which the pair kernel halves for W).
+// nvfp4_set_pair_mode (or NVFP4_GEMM_PAIR=0 / 1 in the environment) turns the pair kernel
+// off / on wherever it applies.  Off by default: on B200 its copies of the scale atoms into
+// both CTAs' tensor memory cost about twice those of one CTA, and the 256 x 256 tiles ran
+// slower than the one-CTA 128 x 256 tiles (prefill gate/up 55 us against 45 us).
+int g_pair_mode = [] {
+    const char *v = getenv("NVFP4_GEMM_PAIR");
+    return v == nullptr ? 0 : (v[0] == '0' ? 0 : 1);
+}();
 int choose_persistent(int M, int N) {
+    const int pair_mode = g_pair_mode;
     const int sms = sm_count_cached();
     const int m_tiles = (M + 127) / 128;
     int best = 0;
@@ -168,6 +196,11 @@ int choose_persistent(int M, int N) {
             best_cost = cost;
             best = bn;
         }
+    }
+    if (N % 256 == 0 && pair_mode != 0) {
+        const int tiles = ((M + 255) / 256) * (N / 256), units = gemm_pair_clusters();
+        const double cost = ((tiles + units - 1) / units) * 0.7;
+        if (cost < best_cost || pair_mode == 1) best = kPairTiles;
     }
     return best;
 }
@@ -261,7 +294,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     Schedule sc;
     int persistent_bn = 0;  // > 0: the persistent kernel with this tile width
     if (block_n == 0 && splits == 0 && M > 128 && (persistent_bn = choose_persistent(M, N)) > 0) {
-        sc = finish(persistent_bn, 1, K, false);
+        sc = finish(persistent_bn == kPairTiles ? 256 : persistent_bn, 1, K, false);
     } else if (block_n == 0 && splits == 0) {
         sc = choose(M, N, K);
     } else if (block_n == 0 && splits == -1) {
@@ -307,21 +340,27 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
         p.tickets = static_cast<uint32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + (tiles * 4 + 255) / 256 * 256);
     }
-    const size_t ctas = static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
+    const size_t ctas = persistent_bn == kPairTiles ? static_cast<size_t>(p.n_tiles) * ((M + 255) / 256) * 2
+                                                    : static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
     if (g_trace != nullptr && g_trace_cursor + 8 * ctas <= g_trace_words) {
         p.trace = g_trace + g_trace_cursor;
         g_trace_cursor += 8 * ctas;
     }
-    CUtensorMap ta, tb;
+    const bool pair = persistent_bn == kPairTiles;
+    CUtensorMap ta, tb, tsa, tsb;
     if (!make_code_map(&ta, A->codes, M, K / 2, static_cast<int>(p.a_box_rows)) ||
-        !make_code_map(&tb, W->codes, N, K / 2, sc.block_n))
+        !make_code_map(&tb, W->codes, N, K / 2, pair ? 128 : sc.block_n))
+        return NVFP4_ERR_CUDA;
+    if (pair && (!make_sf_map(&tsa, A->sf, (M + 127) / 128 * p.k_atoms) ||
+                 !make_sf_map(&tsb, W->sf, (N + 127) / 128 * p.k_atoms)))
         return NVFP4_ERR_CUDA;
     // default schedule for many rows: the persistent kernel; an explicit (block_n, splits)
     // request runs the one-tile-per-CTA kernel
     const bool persistent = persistent_bn > 0;
     if (persistent && (p.status = status_word()) == nullptr) return NVFP4_ERR_CUDA;
-    cudaError_t e = persistent ? launch_gemm_persistent(ta, tb, p, persistent_bn, stream)
-                               : launch_gemm(ta, tb, p, sc.block_n, stream);
+    cudaError_t e = pair         ? launch_gemm_pair(ta, tb, tsa, tsb, p, stream)
+                    : persistent ? launch_gemm_persistent(ta, tb, p, persistent_bn, stream)
+                                 : launch_gemm(ta, tb, p, sc.block_n, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return from_cuda(e);
 }
@@ -395,7 +434,7 @@ nvfp4_status nvfp4_probe(void) {
     if (st != NVFP4_OK) return st;
     // the kernels of this library must load on the device
     if (probe_norm_kernels() != cudaSuccess || probe_gemm_kernels() != cudaSuccess ||
-        probe_gemm_persistent() != cudaSuccess) {
+        probe_gemm_persistent() != cudaSuccess || probe_gemm_pair() != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
     }
@@ -448,6 +487,12 @@ size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int split
     Schedule sc = finish(block_n, splits < 0 ? -splits : splits, K, splits > 0);
     if (sc.cluster && M > 128) sc = finish(block_n, sc.splits, K, false);
     return workspace_for(M, N, sc);
+}
+
+nvfp4_status nvfp4_set_pair_mode(int mode) {
+    if (mode < -1 || mode > 1) return NVFP4_ERR_INVALID_ARG;
+    g_pair_mode = mode;
+    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
