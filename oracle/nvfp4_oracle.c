@@ -357,6 +357,80 @@ float orc_quantize_weight(const uint16_t *w, int N, int K, int ldw, int interlea
     return g;
 }
 
+/* ------------------------------------------------------------------------------------ */
+/* MSE-searched block scales for weights ("Pi0.5 Thor NVFP4 End-to-End Results",
+ * §E0M3 Uniform-INT4 Decoder Weights: the default decoder weights are NVFP4 "(MSE)";
+ * §Fused GeGLU FFN in the Decoder: the gate/up weight is MSE-quantized like the other
+ * decoder projections).  The pages name the criterion, not the search.
+ * READING: per 16-element block every UE4M3 scale byte s = 0x00 .. 0x7E is a candidate.
+ * The codes for s are those the amax quantizer writes once its scale is s: q_i =
+ * E2M1_RNE(y_i * (1 / (dec(s) * g))) in fp32, all +0 when dec(s) = 0.  The block error
+ *   E(s) = sum_i (y_i - val(q_i) * dec(s) * g)^2
+ * is formed in fp64 (the product is exact; one rounded difference and one rounded
+ * square-add per term, terms in index order).  The byte with the smallest E is kept, the
+ * smaller byte on ties (so a zero block keeps s = 0).  g stays amax(|W|) / 2688.          */
+double orc_block_sse(const float *y, float g, uint8_t s, uint8_t *codes8) {
+    float ds = orc_e4m3_decode(s);
+    uint8_t q[16];
+    if (ds == 0.0f) {
+        memset(q, 0, sizeof q);
+    } else {
+        float S = ds * g;
+        float r = 1.0f / S;
+        for (int i = 0; i < 16; ++i) q[i] = orc_e2m1_encode(y[i] * r);
+    }
+    if (codes8 != NULL)
+        for (int j = 0; j < 8; ++j) codes8[j] = (uint8_t)(q[2 * j] | (q[2 * j + 1] << 4));
+    double e = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        double rec = (double)orc_e2m1_decode(q[i]) * (double)ds * (double)g;
+        double d = (double)y[i] - rec;
+        e = e + d * d;
+    }
+    return e;
+}
+
+uint8_t orc_quantize_block16_mse(const float *y, float g, uint8_t *codes8) {
+    uint8_t best = 0;
+    double best_e = orc_block_sse(y, g, 0, NULL);
+    for (int s = 1; s <= 0x7E; ++s) {
+        double e = orc_block_sse(y, g, (uint8_t)s, NULL);
+        if (e < best_e) {
+            best_e = e;
+            best = (uint8_t)s;
+        }
+    }
+    orc_block_sse(y, g, best, codes8);
+    return best;
+}
+
+/* As orc_quantize_weight, with the block scales of orc_quantize_block16_mse. */
+float orc_quantize_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up,
+                              uint8_t *codes, uint8_t *sf) {
+    float amax = 0.0f;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            float m = fabsf(bf16_to_f32(w[(size_t)n * ldw + k]));
+            if (m > amax) amax = m;
+        }
+    float g = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    int nblk = (K + 15) / 16;
+    float blk[16];
+    for (int r = 0; r < N; ++r) {
+        int src = r;
+        if (interleave_gate_up) src = (r % 2 == 0) ? r / 2 : N / 2 + r / 2;
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? bf16_to_f32(w[(size_t)src * ldw + k]) : 0.0f;
+            }
+            uint8_t s = orc_quantize_block16_mse(blk, g, codes + (size_t)r * nblk * 8 + (size_t)b * 8);
+            sf[orc_sf_offset(r, b, K)] = s;
+        }
+    }
+    return g;
+}
+
 /* Dequantized value of element k of row `row`: val(code) * dec(scale) * g, exact in fp64. */
 static double deq_elem(const uint8_t *codes, const uint8_t *sf, float g, int row, int k, int K) {
     int nblk = (K + 15) / 16;

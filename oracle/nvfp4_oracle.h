@@ -88,6 +88,13 @@ void orc_quantize_norm(const void *x, int in_fp32, int rows, int K, int ldx, int
 float orc_quantize_weight(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up,
                           uint8_t *codes, uint8_t *sf);
 
+/* MSE-searched block scales (weights): E(s) of one block with scale byte s (codes8 may be
+ * NULL), the block quantizer that keeps the byte of least E, and the weight quantizer. */
+double orc_block_sse(const float *y, float g, uint8_t s, uint8_t *codes8);
+uint8_t orc_quantize_block16_mse(const float *y, float g, uint8_t *codes8);
+float orc_quantize_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up,
+                              uint8_t *codes, uint8_t *sf);
+
 /* dequantize rows -> fp64 [rows, K] */
 void orc_dequantize(const uint8_t *codes, const uint8_t *sf, float g, int rows, int K,
                     double *out);

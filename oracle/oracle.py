@@ -49,6 +49,12 @@ def lib():
                                         P, C.c_float, C.c_float, P, P]
         L.orc_quantize_weight.restype = C.c_float
         L.orc_quantize_weight.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int, P, P]
+        L.orc_block_sse.restype = C.c_double
+        L.orc_block_sse.argtypes = [P, C.c_float, C.c_uint8, P]
+        L.orc_quantize_block16_mse.restype = C.c_uint8
+        L.orc_quantize_block16_mse.argtypes = [P, C.c_float, P]
+        L.orc_quantize_weight_mse.restype = C.c_float
+        L.orc_quantize_weight_mse.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int, P, P]
         L.orc_dequantize.restype = None
         L.orc_dequantize.argtypes = [P, P, C.c_float, C.c_int, C.c_int, P]
         L.orc_gemm.restype = None
@@ -194,6 +200,31 @@ def quantize_weight(w, interleave_gate_up=False):
     sf = np.zeros(sf_bytes(N, K), np.uint8)
     g = lib().orc_quantize_weight(_p(w), N, K, K, int(bool(interleave_gate_up)), _p(codes), _p(sf))
     return codes, sf, float(np.float32(g))
+
+
+def quantize_weight_mse(w, interleave_gate_up=False):
+    """quantize_weight with MSE-searched block scales (the byte of least block error)."""
+    w = _c(w, np.uint16)
+    N, K = w.shape
+    codes = np.zeros((N, (K + 15) // 16 * 8), np.uint8)
+    sf = np.zeros(sf_bytes(N, K), np.uint8)
+    g = lib().orc_quantize_weight_mse(_p(w), N, K, K, int(bool(interleave_gate_up)), _p(codes), _p(sf))
+    return codes, sf, float(np.float32(g))
+
+
+def block_sse(y, g, s):
+    """(E(s), 8 code bytes) of one 16-value fp32 block at scale byte s."""
+    y = _c(y, np.float32)
+    codes = np.zeros(8, np.uint8)
+    e = lib().orc_block_sse(_p(y), float(g), int(s), _p(codes))
+    return float(e), codes
+
+
+def quantize_block16_mse(y, g):
+    y = _c(y, np.float32)
+    codes = np.zeros(8, np.uint8)
+    s = lib().orc_quantize_block16_mse(_p(y), float(g), _p(codes))
+    return int(s), codes
 
 
 def dequantize(codes, sf, g, rows, K):
