@@ -201,6 +201,18 @@ nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw,
                                    float *global_scale_out, void *scratch,
                                    nvfp4_stream_t stream);
 
+/* As nvfp4_quantize_weight, with MSE-searched block scales ([PI05] §E0M3 Uniform-INT4
+ * Decoder Weights: the default decoder weights are NVFP4 "(MSE)"; §Fused GeGLU FFN in the
+ * Decoder: the interleaved gate/up weight is MSE-quantized too).  Per 16-element block,
+ * every UE4M3 scale byte 0x00..0x7E is tried with the codes the amax quantizer would write
+ * at that scale; the byte whose block squared error (fp64, terms in index order) is least
+ * is kept, the smaller byte on ties.  The global scale is the same amax / 2688.  Same
+ * arguments and constraints as nvfp4_quantize_weight. */
+nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw,
+                                       int interleave_gate_up, uint8_t *codes, uint8_t *sf,
+                                       float *global_scale_out, void *scratch,
+                                       nvfp4_stream_t stream);
+
 /* ---- block-scaled NVFP4 GEMM with fused epilogue ------------------------------------ */
 
 /* acc[m, n] = sum_k dec(A)[m, k] * dec(W)[n, k] over the E2M1 codes and UE4M3 block scales

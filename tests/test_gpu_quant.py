@@ -159,3 +159,50 @@ def test_weight_quantizer_matches_oracle(orc, N, K, inter):
     assert np.float32(q.global_scale) == np.float32(rg)
     assert np.array_equal(host(q.codes), rc)
     assert np.array_equal(host(q.sf), rs)
+
+
+def _weights(kind, seed, N, K):
+    """bf16 weights: Gaussian, heavy-tailed (a few large values per row), or Gaussian rows
+    of very different magnitudes (small blocks take subnormal E4M3 scales)."""
+    w = synth.bf16_normal(synth.seed_of(seed, synth.W0), (N, K), 0.0, 0.02)
+    f = synth.bf16_bits_to_f32(w)
+    if kind == "outliers":
+        f[:, ::37] *= 25.0
+    elif kind == "row_scales":
+        f *= np.logspace(-6, 0, N, dtype=np.float32)[:, None]
+    return synth.f32_to_bf16_bits(f) if kind != "gauss" else w
+
+
+@pytest.mark.parametrize("N,K,inter,kind", [(64, 256, False, "gauss"), (130, 1024, True, "gauss"),
+                                            (48, 2048, False, "outliers"), (96, 512, False, "row_scales"),
+                                            (256, 4096, True, "gauss"), (16, 48, False, "gauss")])
+def test_weight_mse_scales_match_oracle(orc, N, K, inter, kind):
+    """MSE-searched block scales: codes, scale bytes and global scale bit for bit."""
+    w = _weights(kind, 6, N, K)
+    q = nvfp4.quantize_weight(dev_bf16(w), interleave_gate_up=inter, scales="mse")
+    rc, rs, rg = orc.quantize_weight_mse(w, interleave_gate_up=inter)
+    assert np.float32(q.global_scale) == np.float32(rg)
+    assert np.array_equal(host(q.sf), rs)
+    assert np.array_equal(host(q.codes), rc)
+
+
+def test_weight_mse_never_worse_than_amax(orc):
+    """On the device results: per block, dequantized squared error of the MSE scales is at
+    most that of the amax scales; the two differ on most blocks of Gaussian weights."""
+    N, K = 128, 1024
+    w = _weights("gauss", 7, N, K)
+    wd = dev_bf16(w)
+    qa = nvfp4.quantize_weight(wd)
+    qm = nvfp4.quantize_weight(wd, scales="mse")
+    wf = synth.bf16_bits_to_f32(w).astype(np.float64)
+    da = orc.dequantize(host(qa.codes), host(qa.sf), qa.global_scale, N, K)
+    dm = orc.dequantize(host(qm.codes), host(qm.sf), qm.global_scale, N, K)
+    ea = ((wf - da) ** 2).reshape(N, K // 16, 16).sum(-1)
+    em = ((wf - dm) ** 2).reshape(N, K // 16, 16).sum(-1)
+    assert np.all(em <= ea * (1 + 1e-12) + 1e-300)
+    assert (em < ea).mean() > 0.3
+
+
+def test_weight_mse_rejects_bad_scales_argument():
+    with pytest.raises(ValueError):
+        nvfp4.quantize_weight(dev_bf16(synth.bf16_normal(1, (16, 64))), scales="max")

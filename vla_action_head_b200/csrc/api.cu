@@ -538,8 +538,9 @@ nvfp4_status nvfp4_norm_f32(const void *x, nvfp4_in_dtype dt, int M, int K, int 
                      stream);
 }
 
-nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up, uint8_t *codes,
-                                   uint8_t *sf, float *global_scale_out, void *scratch, nvfp4_stream_t stream) {
+static nvfp4_status quantize_weight_impl(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up,
+                                         uint8_t *codes, uint8_t *sf, float *global_scale_out, void *scratch,
+                                         bool mse, cudaStream_t stream) {
     if (w_bf16 == nullptr || codes == nullptr || sf == nullptr || global_scale_out == nullptr || scratch == nullptr)
         return NVFP4_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0 || ldw < K) return NVFP4_ERR_INVALID_ARG;
@@ -552,6 +553,11 @@ nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, in
     uint32_t *amax = static_cast<uint32_t *>(scratch);
     cudaError_t e = launch_weight_amax(static_cast<const uint16_t *>(w_bf16), N, K, ldw, amax, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (mse) {
+        e = launch_weight_mse(static_cast<const uint16_t *>(w_bf16), N, K, ldw, interleave_gate_up ? 1 : 0, amax,
+                              codes, sf, stream);
+        if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
     NormArgs a = {};
     a.x = w_bf16;
     a.M = N;
@@ -564,9 +570,11 @@ nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, in
     a.interleave = interleave_gate_up ? 1 : 0;
     a.codes = codes;
     a.sf = sf;
-    e = launch_norm_quant(a, false, stream);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (!mse) {
+        e = launch_norm_quant(a, false, stream);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
     uint32_t bits = 0;
     e = cudaMemcpyAsync(&bits, amax, sizeof(bits), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
@@ -575,6 +583,19 @@ nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, in
     std::memcpy(&am, &bits, sizeof am);
     *global_scale_out = (am == 0.0f) ? 1.0f : am / 2688.0f;
     return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up, uint8_t *codes,
+                                   uint8_t *sf, float *global_scale_out, void *scratch, nvfp4_stream_t stream) {
+    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, false,
+                                stream);
+}
+
+nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up,
+                                       uint8_t *codes, uint8_t *sf, float *global_scale_out, void *scratch,
+                                       nvfp4_stream_t stream) {
+    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, true,
+                                stream);
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,

@@ -30,6 +30,9 @@ struct NormArgs {
 
 cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s);
 cudaError_t launch_weight_amax(const uint16_t *w, int N, int K, int ldw, uint32_t *amax_bits, cudaStream_t s);
+// MSE-searched block scales for an N x K bf16 weight (global scale from *amax_bits).
+cudaError_t launch_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave, const uint32_t *amax_bits,
+                              uint8_t *codes, uint8_t *sf, cudaStream_t s);
 cudaError_t probe_norm_kernels();
 cudaError_t probe_gemm_kernels();
 

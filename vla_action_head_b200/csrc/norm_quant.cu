@@ -48,6 +48,90 @@ __global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t *w, int
     }
 }
 
+// MSE-searched weight block scales ("Pi0.5 Thor NVFP4 End-to-End Results", §E0M3
+// Uniform-INT4 Decoder Weights: the default decoder weights are NVFP4 "(MSE)"; §Fused GeGLU
+// FFN in the Decoder).  Per 16-element block every UE4M3 scale byte s = 0x00 .. 0x7E is
+// tried with the codes the amax quantizer writes at that scale (q_i = E2M1(y_i * rcp(dec(s)
+// g)), all +0 when dec(s) = 0); the block error E(s) = sum_i (y_i - val(q_i) dec(s) g)^2 is
+// formed in fp64 with one rounding per operation, terms in index order; the byte of least E
+// wins, the smaller byte on ties.  g = amax(|W|) / 2688, as for the amax scales.
+// E2M1 code -> value: magnitudes 0, 0.5, 1, 1.5 (m / 2), 2, 3, 4 (m - 2) and 6.
+__device__ __forceinline__ float e2m1_value(uint32_t q) {
+    const uint32_t m = q & 7u;
+    const float v = m < 4u ? 0.5f * static_cast<float>(m) : (m == 7u ? 6.0f : static_cast<float>(m - 2u));
+    return (q & 8u) ? -v : v;
+}
+__device__ __forceinline__ double block_sse(const float (&y)[16], float g, uint32_t s, uint2 &codes) {
+    const float ds = e4m3_to_f32(s);
+    if (ds == 0.0f) {
+        codes = make_uint2(0u, 0u);
+    } else {
+        const float r = __frcp_rn(__fmul_rn(ds, g));
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(y[i], r);
+        codes.x = cvt_e2m1x8(v);
+        codes.y = cvt_e2m1x8(v + 8);
+    }
+    const double dsg_ds = static_cast<double>(ds), dg = static_cast<double>(g);
+    double e = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t q = ((i < 8 ? codes.x : codes.y) >> (4 * (i & 7))) & 0xFu;
+        const double rec = __dmul_rn(__dmul_rn(static_cast<double>(e2m1_value(q)), dsg_ds), dg);
+        const double d = __dsub_rn(static_cast<double>(y[i]), rec);
+        e = __dadd_rn(e, __dmul_rn(d, d));
+    }
+    return e;
+}
+
+// One warp per block; lane L tries bytes L, L + 32, L + 64, L + 96 (< 127).
+__global__ void __launch_bounds__(256) weight_mse_kernel(const uint16_t *w, int N, int K, int ldw, int interleave,
+                                                         const uint32_t *amax_bits, uint8_t *codes, uint8_t *sf) {
+    const int lane = threadIdx.x & 31;
+    const int nblk = K >> 4;
+    const long long blk = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (blk >= static_cast<long long>(N) * nblk) return;  // whole warps only
+    const int r = static_cast<int>(blk / nblk), b = static_cast<int>(blk % nblk);
+    const int src = interleave ? ((r & 1) == 0 ? r / 2 : N / 2 + r / 2) : r;
+    const uint4 *p = reinterpret_cast<const uint4 *>(w + static_cast<size_t>(src) * ldw + b * 16);
+    const uint4 u0 = __ldg(p), u1 = __ldg(p + 1);
+    const uint32_t ws[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        y[2 * j] = bf16lo(ws[j]);
+        y[2 * j + 1] = bf16hi(ws[j]);
+    }
+    const float amax = __uint_as_float(*amax_bits);
+    const float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    double best_e = 0.0;
+    uint32_t best_s = 0xFFu;
+    for (uint32_t s = static_cast<uint32_t>(lane); s < 127u; s += 32u) {
+        uint2 c;
+        const double e = block_sse(y, g, s, c);
+        if (best_s == 0xFFu || e < best_e) {
+            best_e = e;
+            best_s = s;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double oe = __shfl_xor_sync(0xffffffffu, best_e, o);
+        const uint32_t os = __shfl_xor_sync(0xffffffffu, best_s, o);
+        if (os != 0xFFu && (best_s == 0xFFu || oe < best_e || (oe == best_e && os < best_s))) {
+            best_e = oe;
+            best_s = os;
+        }
+    }
+    if (lane == 0) {
+        uint2 c;
+        block_sse(y, g, best_s, c);
+        *reinterpret_cast<uint2 *>(codes + static_cast<size_t>(r) * nblk * 8 + b * 8) = c;
+        sf[sf_offset(r, b, (K + 63) / 64)] = static_cast<uint8_t>(best_s);
+    }
+}
+
 // ---- launchers (host) ---------------------------------------------------------------------
 template <int TPR, bool F32>
 static cudaError_t launch_tpr(const NormArgs &a, int bpt, cudaStream_t s) {
@@ -91,6 +175,15 @@ cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s) {
     }
     const int bpt = (nblk + 127) / 128;
     return f32_in ? launch_tpr<128, true>(a, bpt, s) : launch_tpr<128, false>(a, bpt, s);
+}
+
+cudaError_t launch_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave, const uint32_t *amax_bits,
+                              uint8_t *codes, uint8_t *sf, cudaStream_t s) {
+    const long long blocks = static_cast<long long>(N) * (K >> 4);
+    const long long ctas = (blocks + 7) / 8;
+    if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    weight_mse_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(w, N, K, ldw, interleave, amax_bits, codes, sf);
+    return cudaGetLastError();
 }
 
 cudaError_t probe_norm_kernels() {

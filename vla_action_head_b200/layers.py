@@ -29,11 +29,12 @@ from . import nvfp4, synth
 
 
 class Linear:
-    """NVFP4 weight [N, K] (+ optional bf16 bias), quantized once from bf16."""
+    """NVFP4 weight [N, K] (+ optional bf16 bias), quantized once from bf16 with amax or
+    MSE-searched block scales."""
 
-    def __init__(self, w_bf16, bias=None, interleave_gate_up=False):
+    def __init__(self, w_bf16, bias=None, interleave_gate_up=False, scales="amax"):
         self.N, self.K = w_bf16.shape
-        self.w = nvfp4.quantize_weight(w_bf16.contiguous(), interleave_gate_up=interleave_gate_up)
+        self.w = nvfp4.quantize_weight(w_bf16.contiguous(), interleave_gate_up=interleave_gate_up, scales=scales)
         self.bias = bias
 
     def weight_bytes(self):
@@ -97,16 +98,19 @@ class DiTLayer:
 
 
 class ActionExpertLayer:
-    def __init__(self, M=50, H=1024, A=2048, F=4096, wl=3, layer=0, device="cuda", ws=None):
+    # The decoder projections take MSE-searched block scales by default ("Pi0.5 Thor NVFP4
+    # End-to-End Results", §E0M3 Uniform-INT4 Decoder Weights: NVFP4 "(MSE, default)").
+    def __init__(self, M=50, H=1024, A=2048, F=4096, wl=3, layer=0, device="cuda", ws=None, weight_scales="mse"):
         s = lambda tid: synth.seed_of(wl, 100 * layer + tid)  # noqa: E731
         d = device
         self.M, self.H, self.A, self.F = M, H, A, F
         self.scale1 = _rand(s(synth.MOD_SCALE), (H,), 0.0, 0.1, d)
         self.scale2 = _rand(s(synth.MOD_SHIFT), (H,), 0.0, 0.1, d)
-        self.qkv = Linear(_rand(s(synth.W0), (2560, H), 0, 0.02, d))
-        self.o = Linear(_rand(s(synth.W0 + 1), (H, A), 0, 0.02, d))
-        self.gate_up = Linear(_rand(s(synth.W0 + 2), (2 * F, H), 0, 0.02, d), interleave_gate_up=True)
-        self.down = Linear(_rand(s(synth.W0 + 3), (H, F), 0, 0.02, d))
+        self.qkv = Linear(_rand(s(synth.W0), (2560, H), 0, 0.02, d), scales=weight_scales)
+        self.o = Linear(_rand(s(synth.W0 + 1), (H, A), 0, 0.02, d), scales=weight_scales)
+        self.gate_up = Linear(_rand(s(synth.W0 + 2), (2 * F, H), 0, 0.02, d), interleave_gate_up=True,
+                              scales=weight_scales)
+        self.down = Linear(_rand(s(synth.W0 + 3), (H, F), 0, 0.02, d), scales=weight_scales)
         self.ws = ws or nvfp4.Workspace(d)
         self.a1 = nvfp4.empty_fp4(M, H, d)
         self.ctx_q = nvfp4.empty_fp4(M, A, d)
@@ -157,7 +161,7 @@ class GatedActionExpertLayer:
 
     forward returns (d_out, g2): the next layer's front-end 1 applies r += g2 * d_out."""
 
-    def __init__(self, M=50, H=1024, A=2048, F=4096, wl=6, layer=0, device="cuda", ws=None):
+    def __init__(self, M=50, H=1024, A=2048, F=4096, wl=6, layer=0, device="cuda", ws=None, weight_scales="mse"):
         s = lambda tid: synth.seed_of(wl, 100 * layer + tid)  # noqa: E731
         d = device
         self.M, self.H, self.A, self.F = M, H, A, F
@@ -167,10 +171,11 @@ class GatedActionExpertLayer:
         self.t2 = _rand(s(synth.BETA), (H,), 0.0, 0.1, d)
         self.g1 = _rand(s(synth.RESIDUAL), (H,), 0.0, 0.5, d)
         self.g2 = _rand(s(synth.RESIDUAL + 1), (H,), 0.0, 0.5, d)
-        self.qkv = Linear(_rand(s(synth.W0), (2560, H), 0, 0.02, d))
-        self.o = Linear(_rand(s(synth.W0 + 1), (H, A), 0, 0.02, d))
-        self.gate_up = Linear(_rand(s(synth.W0 + 2), (2 * F, H), 0, 0.02, d), interleave_gate_up=True)
-        self.down = Linear(_rand(s(synth.W0 + 3), (H, F), 0, 0.02, d))
+        self.qkv = Linear(_rand(s(synth.W0), (2560, H), 0, 0.02, d), scales=weight_scales)
+        self.o = Linear(_rand(s(synth.W0 + 1), (H, A), 0, 0.02, d), scales=weight_scales)
+        self.gate_up = Linear(_rand(s(synth.W0 + 2), (2 * F, H), 0, 0.02, d), interleave_gate_up=True,
+                              scales=weight_scales)
+        self.down = Linear(_rand(s(synth.W0 + 3), (H, F), 0, 0.02, d), scales=weight_scales)
         self.ws = ws or nvfp4.Workspace(d)
         self.a1 = nvfp4.empty_fp4(M, H, d)
         self.ctx_q = nvfp4.empty_fp4(M, A, d)

@@ -81,6 +81,7 @@ def lib():
             "nvfp4_residual_quantize_norm": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, P, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
+            "nvfp4_quantize_weight_mse": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
             "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
                                F, P, SZ, P]),
             "nvfp4_program_bytes": (SZ, [I]),
@@ -201,7 +202,11 @@ def norm_f32(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, o
 _scratch = {}
 
 
-def quantize_weight(w, interleave_gate_up=False) -> NVFP4Tensor:
+def quantize_weight(w, interleave_gate_up=False, scales="amax") -> NVFP4Tensor:
+    """bf16 W [N, K] -> NVFP4; scales "amax" (block amax / 6) or "mse" (the scale byte of
+    least block squared error)."""
+    if scales not in ("amax", "mse"):
+        raise ValueError(f"scales must be 'amax' or 'mse', got {scales!r}")
     torch = _torch()
     N, K = w.shape
     out = empty_fp4(N, K, w.device)
@@ -209,10 +214,10 @@ def quantize_weight(w, interleave_gate_up=False) -> NVFP4Tensor:
     if dev not in _scratch:
         _scratch[dev] = torch.zeros(256, dtype=torch.uint8, device=w.device)
     g = C.c_float(0.0)
-    st = lib().nvfp4_quantize_weight(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)),
-                                     _ptr(out.codes), _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]),
-                                     _stream())
-    _check("nvfp4_quantize_weight", st)
+    name = "nvfp4_quantize_weight" if scales == "amax" else "nvfp4_quantize_weight_mse"
+    st = getattr(lib(), name)(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)), _ptr(out.codes),
+                              _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]), _stream())
+    _check(name, st)
     out.global_scale = g.value
     return out
 
