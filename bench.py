@@ -153,14 +153,22 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(ws, v):
+def max_over_ranks(ws, v, device="cuda"):
+    """The largest v over the ranks (every rank gets it); `device` is where the collective
+    runs ("cuda" under NCCL, "cpu" under gloo)."""
     if ws == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def us_per_layer(ms_max, steps, layers_per_step, ws):
+    """Whole-job time per layer: every rank runs `steps` x `layers_per_step` layers of its own
+    (replicas), the job ends with the slowest rank."""
+    return ms_max * 1e3 / (steps * layers_per_step * ws)
 
 
 # ---------------------------------------------------------------------------------------
@@ -398,7 +406,7 @@ def main():
     clocks = clk.stop()
     ms_total = max_over_ranks(ws_n, e0.elapsed_time(e1))
     nvfp4.device_status()
-    us_layer = ms_total * 1e3 / (args.steps * L * ws_n)
+    us_layer = us_per_layer(ms_total, args.steps, L, ws_n)
     # per-step spread (each step timed on its own, after the timed region)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with torch.cuda.stream(stream):
@@ -429,7 +437,7 @@ def main():
     torch.cuda.synchronize()
     barrier(ws_n)
     ms_e2e = max_over_ranks(ws_n, e0.elapsed_time(e1))
-    us_layer_e2e = ms_e2e * 1e3 / (args.steps * L * ws_n)
+    us_layer_e2e = us_per_layer(ms_e2e, args.steps, L, ws_n)
 
     line = {"metric": METRIC, "value": round(us_layer, 3), "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4), "higher_is_better": False,
