@@ -139,7 +139,11 @@ Schedule finish(int block_n, int splits, int K, bool use_cluster = true) {
 // Default schedule.  Small M streams the weights: pick the tile width and split factor
 // (<= 8, reduced in a cluster) that put about one CTA on every SM, preferring wider tiles
 // and fewer splits.  Large M is compute-bound: widest tile, no split.
-Schedule choose(int M, int N, int K) {
+// fp4_out: the epilogue re-quantizes (bias+GELU or GeGLU -> FP4), which costs far more per
+// output element than a bf16 store, so the owner CTAs' share of the epilogue enters the cost
+// (measured at M = 41, N = 6144, K = 1536: 64-wide tiles split 2 ways take 6.6 us where
+// 128-wide ones split 3 ways take 7.8 us).
+Schedule choose(int M, int N, int K, bool fp4_out) {
     const int sms = sm_count_cached();
     const int k_tiles = (K + 255) / 256;
     const int m_tiles = (M + 127) / 128;
@@ -153,8 +157,10 @@ Schedule choose(int M, int N, int K) {
                 const Schedule c = finish(bn, s, K);
                 const int ctas = n_tiles * c.splits;
                 if (ctas > 2 * sms) continue;
+                if (fp4_out && 2 * ctas > 3 * sms) continue;  // two heavy epilogues per SM (measured slow)
+                const int owner_rows = (std::min(M, 128) + c.splits - 1) / c.splits;
                 const double cost = std::fabs(static_cast<double>(ctas - sms)) / sms + 0.03 * c.splits +
-                                    (bn == 64 ? 0.05 : 0.0);
+                                    (bn == 64 ? 0.05 : 0.0) + (fp4_out ? 1e-3 * owner_rows * bn : 0.0);
                 if (cost < best_cost) {
                     best_cost = cost;
                     best = c;
@@ -167,9 +173,6 @@ Schedule choose(int M, int N, int K) {
     return finish(bn, 1, K);
 }
 
-// Tile width of the persistent kernel for many rows (0: not applicable).  A 128-wide tile
-// costs about 0.72 of a 256-wide one (more scale copies per FLOP), so 128 wins when 256-wide
-// tiles would leave SMs idle, e.g. N = 2048 at M = 968 (64 tiles on 148 SMs).
 // The many-row schedule: 256 or 128 = the one-CTA persistent kernel with that tile width,
 // kPairTiles = 256 x 256 tiles on CTA pairs.  Cost: waves x the relative time of a wave
 // (a 128-wide tile does half the work of a 256-wide one for 0.72 of its time: the wider
@@ -217,7 +220,7 @@ Schedule choose_workspace(int M, int N, int K) {
         if (splits > k_tiles) splits = k_tiles;
         return finish(bn, splits, K, false);
     }
-    return choose(M, N, K);
+    return choose(M, N, K, false);
 }
 
 size_t workspace_for(int M, int N, const Schedule &s) {
@@ -296,7 +299,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if (block_n == 0 && splits == 0 && M > 128 && (persistent_bn = choose_persistent(M, N)) > 0) {
         sc = finish(persistent_bn == kPairTiles ? 256 : persistent_bn, 1, K, false);
     } else if (block_n == 0 && splits == 0) {
-        sc = choose(M, N, K);
+        sc = choose(M, N, K, epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
     } else if (block_n == 0 && splits == -1) {
         sc = choose_workspace(M, N, K);
     } else {
@@ -476,7 +479,7 @@ nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream) 
 
 size_t nvfp4_gemm_workspace_bytes(int M, int N, int K) {
     if (M <= 0 || N <= 0 || K <= 0 || N % 64 != 0) return 0;
-    return workspace_for(M, N, choose(M, N, K));
+    return workspace_for(M, N, choose(M, N, K, false));
 }
 
 size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int splits) {

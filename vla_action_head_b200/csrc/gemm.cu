@@ -57,11 +57,16 @@ struct Cfg {
     static constexpr int kBBytes = BN * 128;
     static constexpr int kSfaBytes = 4 * kSfAtom;
     static constexpr int kSfbBytes = kSfbGroups * 4 * kSfAtom;
-    // tensor-memory columns: accumulator, then 16 columns of A scales, then B scales
-    // scale columns: two slots (stage parity) of [A: 4 k-blocks x 4 | W: 4 k-blocks x groups x 4]
+    // tensor-memory columns: the accumulator, then kSlots scale slots of [A: 4 k-blocks x 4 |
+    // W: 4 k-blocks x groups x 4]; K tile j uses slot j % kSlots.  Up to 128 columns wide, as
+    // many slots as fit in 256 columns (6 at BN 64, 4 at BN 128): a CTA with that many K
+    // tiles or fewer never waits for a slot, so the copies of every tile start as soon as it
+    // lands.  (256 columns keep two CTAs per SM: the next kernel's CTAs allocate while this
+    // one runs.)
     static constexpr int kColSf = BN;
     static constexpr int kSfSlot = 16 + 16 * kSfbGroups;
-    static constexpr int kColsUsed = BN + 2 * kSfSlot;
+    static constexpr int kSlots = BN <= 128 ? (256 - BN) / kSfSlot : 2;
+    static constexpr int kColsUsed = BN + kSlots * kSfSlot;
     static constexpr int kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64 : kColsUsed <= 128 ? 128
                                      : kColsUsed <= 256 ? 256 : 512;
 };
@@ -78,7 +83,8 @@ struct Smem {
     static constexpr int kOffSfa = kOffB + STAGES * Cfg<BN>::kBBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * Cfg<BN>::kSfaBytes;
     static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes;
-    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 5) * 8;
+    // barriers: full[STAGES], empty[STAGES], acc, sf_ready[kSlots], sf_free[kSlots]
+    static constexpr int kOffMisc = kOffBar + (2 * STAGES + 1 + 2 * Cfg<BN>::kSlots) * 8;
     static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
     // split-K partial tile for the cluster reduction, reusing the stage buffers
     static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
@@ -110,8 +116,8 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     const uint32_t bar_full = sbase + S::kOffBar;             // STAGES barriers
     const uint32_t bar_empty = bar_full + STAGES * 8;         // STAGES barriers
     const uint32_t bar_acc = bar_empty + STAGES * 8;          // 1 barrier
-    const uint32_t bar_sfr = bar_acc + 8;                     // 2: scale slot copied (4 arrivals)
-    const uint32_t bar_sff = bar_sfr + 16;                    // 2: scale slot read by its MMAs
+    const uint32_t bar_sfr = bar_acc + 8;                     // kSlots: scale slot copied (4 arrivals)
+    const uint32_t bar_sff = bar_sfr + 8 * C::kSlots;         // kSlots: scale slot read by its MMAs
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + S::kOffMisc);
     // misc[0] = tensor-memory base, misc[1] = abort flag, misc[2] = split-K ticket,
     // misc[3] = accumulator-valid decision of the epilogue warps
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             mbar_init(bar_empty + 8 * s, 1);
         }
         mbar_init(bar_acc, 1);
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < C::kSlots; ++j) {
             mbar_init(bar_sfr + 8 * j, 4);
             mbar_init(bar_sff + 8 * j, 1);
         }
@@ -222,9 +228,10 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             const uint32_t t_acc = tmem;
             const uint32_t sfb_sub = (BN == 64) ? static_cast<uint32_t>((n0 & 127) >> 5) : 0u;
             for (int j = 0; j < nkt; ++j) {
-                const int s = j % STAGES, kt = kt_begin + j, slot = j & 1;
+                const int s = j % STAGES, kt = kt_begin + j, slot = j % C::kSlots;
                 if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull) ||
-                    !mbar_wait(bar_sfr + 8 * slot, (j >> 1) & 1, abort_flag, &g_device_status, kStatusTimeoutFull))
+                    !mbar_wait(bar_sfr + 8 * slot, (j / C::kSlots) & 1, abort_flag, &g_device_status,
+                               kStatusTimeoutFull))
                     break;
                 tc_fence_after();
                 if (trace != nullptr && j == 0) trace[3] = globaltimer_ns();
@@ -251,16 +258,16 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
         const bool row_ok = m < p.M;
         // Until the accumulator is ready these warps copy the scale atoms (tcgen05.cp from one
         // thread complete one after another; from four warps they overlap): warp w copies
-        // k-block w of each stage into the stage's scale slot (of two).
+        // k-block w of each stage into the stage's scale slot.
         if (lane == 0) {
             const int w = warp - 2;
             const uint32_t sfa_s0 = sbase + S::kOffSfa, sfb_s0 = sbase + S::kOffSfb;
             for (int j = 0; j < nkt; ++j) {
-                const int s = j % STAGES, kt = kt_begin + j, slot = j & 1;
+                const int s = j % STAGES, kt = kt_begin + j, slot = j % C::kSlots;
                 if (!mbar_wait(bar_full + 8 * s, (j / STAGES) & 1, abort_flag, &g_device_status, kStatusTimeoutFull))
                     break;
-                if (j >= 2 && !mbar_wait(bar_sff + 8 * slot, ((j >> 1) - 1) & 1, abort_flag, &g_device_status,
-                                         kStatusTimeoutFull))
+                if (j >= C::kSlots && !mbar_wait(bar_sff + 8 * slot, (j / C::kSlots - 1) & 1, abort_flag,
+                                                 &g_device_status, kStatusTimeoutFull))
                     break;
                 tc_fence_after();
                 const uint32_t t_sf = tmem + C::kColSf + slot * C::kSfSlot;
