@@ -136,13 +136,14 @@ Schedule finish(int block_n, int splits, int K, bool use_cluster = true) {
     return Schedule{block_n, eff, per, use_cluster && eff > 1 && eff <= kMaxClusterSplits};
 }
 
-// Default schedule.  Small M streams the weights: pick the tile width and split factor
-// (<= 8, reduced in a cluster) that put about one CTA on every SM, preferring wider tiles
-// and fewer splits.  Large M is compute-bound: widest tile, no split.
-// fp4_out: the epilogue re-quantizes (bias+GELU or GeGLU -> FP4), which costs far more per
-// output element than a bf16 store, so the owner CTAs' share of the epilogue enters the cost
-// (measured at M = 41, N = 6144, K = 1536: 64-wide tiles split 2 ways take 6.6 us where
-// 128-wide ones split 3 ways take 7.8 us).
+// Default schedule: the tile width and split factor (<= 8, reduced in a cluster) of least
+// modelled time.  Small M is a chain of latencies; the cost is a latency model (us) fitted to schedule
+// sweeps of the DiT (M = 41) and action-expert (M = 50) GEMMs on B200:
+//   0.3 per K tile a CTA walks, + 0.3 + 0.004 * block_n for a split-K exchange (two cluster
+//   barriers and the partial rows pushed to their owners), + the operand bytes streamed at
+//   30 GB/s per CTA (up to one CTA per SM), + 2e-4 per element of a re-quantizing epilogue
+//   (bias+GELU or GeGLU -> FP4) on the owner CTA.  Grids above 1.35 CTAs per SM (1.5 for a
+//   re-quantizing epilogue) measured slow and are not used.
 Schedule choose(int M, int N, int K, bool fp4_out) {
     const int sms = sm_count_cached();
     const int k_tiles = (K + 255) / 256;
@@ -150,17 +151,19 @@ Schedule choose(int M, int N, int K, bool fp4_out) {
     if (M <= 128) {
         Schedule best{64, 1, k_tiles, false};
         double best_cost = 1e30;
+        const double bytes = static_cast<double>(N) * K * (0.5 + 1.0 / 16) + static_cast<double>(M) * K * 0.5;
         for (int bn : {128, 64}) {
             if (N % bn != 0) continue;
             const int n_tiles = N / bn * m_tiles;
             for (int s = 1; s <= kMaxClusterSplits && s <= k_tiles; ++s) {
                 const Schedule c = finish(bn, s, K);
                 const int ctas = n_tiles * c.splits;
-                if (ctas > 2 * sms) continue;
-                if (fp4_out && 2 * ctas > 3 * sms) continue;  // two heavy epilogues per SM (measured slow)
+                if (20 * ctas > 27 * sms) continue;
+                if (fp4_out && 2 * ctas > 3 * sms) continue;
                 const int owner_rows = (std::min(M, 128) + c.splits - 1) / c.splits;
-                const double cost = std::fabs(static_cast<double>(ctas - sms)) / sms + 0.03 * c.splits +
-                                    (bn == 64 ? 0.05 : 0.0) + (fp4_out ? 1e-3 * owner_rows * bn : 0.0);
+                const double cost = 0.3 * c.kt_per_split + (c.splits > 1 ? 0.3 + 0.004 * bn : 0.0) +
+                                    bytes / (std::min(ctas, sms) * 30e3) +
+                                    (fp4_out ? 2e-4 * owner_rows * bn : 0.0);
                 if (cost < best_cost) {
                     best_cost = cost;
                     best = c;
