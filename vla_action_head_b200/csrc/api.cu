@@ -143,7 +143,8 @@ Schedule finish(int block_n, int splits, int K, bool use_cluster = true) {
 //   barriers and the partial rows pushed to their owners), + the operand bytes streamed at
 //   30 GB/s per CTA (up to one CTA per SM), + 2e-4 per element of a re-quantizing epilogue
 //   (bias+GELU or GeGLU -> FP4) on the owner CTA.  Grids above 1.35 CTAs per SM (1.5 for a
-//   re-quantizing epilogue) measured slow and are not used.
+//   re-quantizing epilogue), or above what one wave of the kernel holds, measured slow and
+//   are not used.
 Schedule choose(int M, int N, int K, bool fp4_out) {
     const int sms = sm_count_cached();
     const int k_tiles = (K + 255) / 256;
@@ -159,6 +160,11 @@ Schedule choose(int M, int N, int K, bool fp4_out) {
                 const Schedule c = finish(bn, s, K);
                 const int ctas = n_tiles * c.splits;
                 if (20 * ctas > 27 * sms) continue;
+                // M > 64 runs one CTA per SM: more CTAs than one wave holds (clusters must fit in
+                // a GPC) run as two waves.  (At M <= 64, two CTAs share an SM; the occupancy API
+                // under-counts those waves, and the measured grids fit.)
+                const int wave = M > 64 ? gemm_wave_ctas(false, bn, c.splits) : 0;
+                if (wave > 0 && ctas > wave) continue;
                 if (fp4_out && 2 * ctas > 3 * sms) continue;
                 const int owner_rows = (std::min(M, 128) + c.splits - 1) / c.splits;
                 const double cost = 0.3 * c.kt_per_split + (c.splits > 1 ? 0.3 + 0.004 * bn : 0.0) +

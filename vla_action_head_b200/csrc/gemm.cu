@@ -539,6 +539,56 @@ cudaError_t read_and_clear_device_status(cudaStream_t s, uint32_t *out) {
     return cudaMemcpyToSymbol(g_device_status, &zero, sizeof(uint32_t));
 }
 
+template <int BN, int STAGES, bool SMALL_A>
+static int wave_ctas_of(int cluster) {
+    using S = Smem<BN, STAGES, SMALL_A>;
+    if (cudaFuncSetAttribute(gemm_kernel<BN, STAGES, SMALL_A>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S::kBytes) != cudaSuccess)
+        return 0;
+    if (cluster <= 1) {
+        int per_sm = 0, dev = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm_kernel<BN, STAGES, SMALL_A>, kThreads,
+                                                          S::kBytes) != cudaSuccess ||
+            cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 0;
+        return per_sm * sms;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cluster));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = S::kBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<BN, STAGES, SMALL_A>, &cfg) != cudaSuccess) return 0;
+    return n * cluster;
+}
+
+int gemm_wave_ctas(bool small, int block_n, int cluster) {
+    if (cluster < 1 || cluster > 8) return 0;
+    static int cache[2][3][9] = {};  // [small][64, 128, 256][cluster]; 0 = not yet asked
+    const int w = block_n == 64 ? 0 : block_n == 128 ? 1 : block_n == 256 ? 2 : -1;
+    if (w < 0) return 0;
+    int &c = cache[small ? 1 : 0][w][cluster];
+    if (c == 0) {
+        int v = 0;
+        switch (block_n) {
+        case 64: v = small ? wave_ctas_of<64, 5, true>(cluster) : wave_ctas_of<64, 6, false>(cluster); break;
+        case 128: v = small ? wave_ctas_of<128, 3, true>(cluster) : wave_ctas_of<128, 5, false>(cluster); break;
+        default: v = small ? wave_ctas_of<256, 2, true>(cluster) : wave_ctas_of<256, 3, false>(cluster); break;
+        }
+        cudaGetLastError();
+        c = v > 0 ? v : -1;
+    }
+    return c > 0 ? c : 0;
+}
+
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s) {
     const bool small = p.a_box_rows <= 64;

@@ -40,6 +40,9 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                         cudaStream_t s);
+// CTAs that one wave of the one-tile kernel holds for the given A rows class (small: M <= 64),
+// tile width and cluster size (1: no cluster), from the occupancy API; 0 if unknown.
+int gemm_wave_ctas(bool small, int block_n, int cluster);
 
 // Persistent 128 x block_n tile kernel for many rows (gemm_persistent.cu): block_n 256 or
 // 128, one split.  Grid: min(tiles, SMs) CTAs.
