@@ -329,12 +329,19 @@ typedef struct {
     int cluster;
     size_t ops_offset, maps_offset, done_offset;
     int waits;  /* ops that wait for another op (0: the completion counters go unused) */
+    int kind;   /* 0: the layer executor; 1: the grouped GEMM kernel (see nvfp4_program_build) */
+    int epi;    /* kind 1: the epilogue of every op */
+    int tiles;  /* kind 1: output tiles over all ops */
 } nvfp4_program;
 
 /* Device bytes a program of n_ops ops needs. */
 size_t nvfp4_program_bytes(int n_ops);
 
-/* Validates the ops (the rules of the standalone calls, plus: at most 4096 ops (else
+/* A program of 2..256 GEMM ops that all have dep = NVFP4_DEP_NONE, the same epilogue and
+ * N % 128 == 0 is a grouped GEMM and runs on the grouped kernel: one CTA per SM walks all the
+ * problems' 128 x 128 output tiles through one TMA / tensor-core pipeline, so the weight
+ * stream does not stop at problem boundaries (kind 1).  Other programs run on the executor.
+ * Validates the ops (the rules of the standalone calls, plus: at most 4096 ops (else
  * NVFP4_ERR_UNSUPPORTED_SHAPE); GEMM M <= 64, N % 64 == 0, K % 32 == 0; norm K <= 4096, bf16
  * input; each dep names an earlier op), chooses each GEMM's schedule, encodes the TMA
  * descriptors and copies the program into `buffer` (device, >= nvfp4_program_bytes(n_ops),

@@ -5,7 +5,7 @@ standalone calls, and op dependencies other than "the previous op" are honoured.
 import numpy as np
 import pytest
 
-from parity import bf16_to_f64, check_gemm_bf16, dev_bf16, host, to_gpu_fp4
+from parity import bf16_to_f64, check_fp4_output, check_gemm_bf16, dev_bf16, host, to_gpu_fp4
 from vla_action_head_b200 import nvfp4, synth
 
 pytestmark = pytest.mark.gpu
@@ -46,10 +46,63 @@ def test_grouped_mixed_shapes_match_oracle(orc, with_bias):
                       dev_bf16(bias) if with_bias else None))
         refs.append(ref["v"])
     grp = nvfp4.GroupedGemm(probs, epi="bias" if with_bias else "none")
+    assert grp.prog.kind == 1  # the grouped kernel
     grp.run()
     _sync()
     for g, (p, ref) in enumerate(zip(probs, refs)):
         check_gemm_bf16(host(p[2]), ref, what=("grouped", g, shapes[g]))
+
+
+@pytest.mark.parametrize("epi", ["residual", "bias_gelu", "geglu"])
+def test_grouped_kernel_epilogues(orc, epi):
+    """The grouped kernel's other epilogue kinds, including FP4 outputs, on problems of
+    different M (one above 128 rows: two m-tiles) and K."""
+    import torch
+    shapes = [(41, 1024, 1536), (150, 512, 512), (8, 256, 2048)]
+    probs, refs = [], []
+    for g, (M, N, K) in enumerate(shapes):
+        x = synth.bf16_normal(synth.seed_of(90 + g, synth.CONTEXT), (M, K))
+        w = synth.bf16_normal(synth.seed_of(90 + g, synth.W0), (N, K), 0.0, 0.02)
+        ac, asf = orc.quantize_norm(x, "none")
+        wc, wsf, gw = orc.quantize_weight(w, interleave_gate_up=(epi == "geglu"))
+        bias = synth.bf16_normal(synth.seed_of(90 + g, synth.BIAS0), (N,), 0.0, 0.01) if epi == "bias_gelu" else None
+        res = synth.bf16_normal(synth.seed_of(90 + g, synth.RESIDUAL), (M, N)) if epi == "residual" else None
+        ref = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res)
+        A, W = to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+        if epi in ("bias_gelu", "geglu"):
+            out = nvfp4.empty_fp4(M, N // 2 if epi == "geglu" else N)
+        else:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        probs.append(nvfp4.op_gemm(A, W, epi, bias=dev_bf16(bias) if bias is not None else None,
+                                   residual=dev_bf16(res) if res is not None else None, out=out, dep=None))
+        refs.append((ref, out, M, N, K))
+    prog = nvfp4.Program(probs)
+    assert prog.prog.kind == 1
+    prog.run()
+    _sync()
+    for ref, out, M, N, K in refs:
+        if epi in ("bias_gelu", "geglu"):
+            check_fp4_output(orc, host(out.codes), host(out.sf), ref["codes"], ref["sf"], ref["h"], 1.0, M, out.K,
+                             what=(M, N, K, epi))
+        else:
+            check_gemm_bf16(host(out), ref["v"], what=(M, N, K, epi))
+
+
+def test_groups_the_kernel_does_not_take_run_on_the_executor(orc):
+    """A problem with N % 128 != 0, or mixed epilogues, keeps the group on the executor."""
+    import torch
+    probs, refs = [], []
+    for g, (M, N, K) in enumerate([(41, 192, 512), (41, 256, 512)]):
+        _, (ac, asf), (wc, wsf, gw), _, ref = _problem(orc, 30 + g, M, N, K, False)
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        probs.append((to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K), out))
+        refs.append(ref["v"])
+    grp = nvfp4.GroupedGemm(probs)
+    assert grp.prog.kind == 0
+    grp.run()
+    _sync()
+    for p, ref in zip(probs, refs):
+        check_gemm_bf16(host(p[2]), ref, what="executor group")
 
 
 def test_grouped_cross_kv_32_matches_standalone(orc):
@@ -68,6 +121,7 @@ def test_grouped_cross_kv_32_matches_standalone(orc):
             refs[g] = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="none")["v"]
         probs.append((A, to_gpu_fp4(wc, wsf, gw, N, K), torch.empty((M, N), dtype=torch.bfloat16, device="cuda")))
     grp = nvfp4.GroupedGemm(probs)
+    assert grp.prog.kind == 1
     grp.run()
     _sync()
     for g, ref in refs.items():

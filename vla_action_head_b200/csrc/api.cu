@@ -446,7 +446,8 @@ nvfp4_status nvfp4_probe(void) {
     if (st != NVFP4_OK) return st;
     // the kernels of this library must load on the device
     if (probe_norm_kernels() != cudaSuccess || probe_gemm_kernels() != cudaSuccess ||
-        probe_gemm_persistent() != cudaSuccess || probe_gemm_pair() != cudaSuccess) {
+        probe_gemm_persistent() != cudaSuccess || probe_gemm_pair() != cudaSuccess ||
+        probe_gemm_grouped() != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
     }
@@ -656,9 +657,13 @@ size_t nvfp4_program_bytes(int n_ops) {
     if (n_ops <= 0) return 0;
     const size_t maps = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
     const size_t ops = (static_cast<size_t>(n_ops) * sizeof(ExecOp) + 255) / 256 * 256;
-    const size_t done = (static_cast<size_t>(n_ops) * 4 + 255) / 256 * 256;
+    // completion counters (executor) or the grouped kernel's tile table (4 n + 1 words)
+    const size_t done = (static_cast<size_t>(n_ops) * 16 + 4 + 255) / 256 * 256;
     return maps + ops + done;
 }
+
+static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t maps_off, size_t ops_off,
+                          size_t tab_off, nvfp4_program *prog, nvfp4_status *st);
 
 nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes, nvfp4_program *prog) {
     if (ops == nullptr || n_ops <= 0 || buffer == nullptr || prog == nullptr) return NVFP4_ERR_INVALID_ARG;
@@ -667,6 +672,24 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
     if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
+    {
+        // a grouped GEMM (independent GEMM ops, one epilogue, N % 128 == 0) takes the grouped
+        // kernel; its ops follow the rules of the standalone GEMM (any M)
+        const size_t maps_b = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
+        const size_t ops_b = (static_cast<size_t>(n_ops) * sizeof(ExecOp) + 255) / 256 * 256;
+        nvfp4_status gst = NVFP4_OK;
+        if (build_grouped(ops, n_ops, static_cast<uint8_t *>(buffer), 0, maps_b, maps_b + ops_b, prog, &gst)) {
+            if (gst != NVFP4_OK) return gst;
+            prog->buffer = buffer;
+            prog->bytes = bytes;
+            prog->n_ops = n_ops;
+            prog->cluster = 1;
+            prog->maps_offset = 0;
+            prog->ops_offset = maps_b;
+            prog->done_offset = maps_b + ops_b;
+            return NVFP4_OK;
+        }
+    }
     int grid = 0;
     if (exec_grid(kExecCluster, &grid) != cudaSuccess || grid < kExecCluster) return NVFP4_ERR_CUDA;
     const int teams = grid / kExecCluster;
@@ -823,12 +846,116 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
     prog->ops_offset = maps_bytes;
     prog->done_offset = maps_bytes + ops_bytes;
     prog->waits = waits;
+    prog->kind = 0;
+    prog->epi = 0;
+    prog->tiles = 0;
     return NVFP4_OK;
+}
+
+// A program of independent GEMM ops with one epilogue kind and N % 128 == 0 (a grouped GEMM)
+// runs on the grouped persistent kernel instead of the executor: the same results (one split
+// per tile, as the executor's grouped schedule), with the weight stream kept running across
+// problem boundaries.  Writes the problems' GemmArgs over the op area, their tensor maps and
+// the tile table; returns false if the program is not such a group.
+static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t maps_off, size_t ops_off,
+                          size_t tab_off, nvfp4_program *prog, nvfp4_status *st) {
+    if (n_ops < 2 || n_ops > kGroupedMaxProblems) return false;
+    for (int i = 0; i < n_ops; ++i) {
+        const nvfp4_op &o = ops[i];
+        if (o.type != NVFP4_OP_GEMM || o.dep != NVFP4_DEP_NONE || o.epi != ops[0].epi || o.N % 128 != 0)
+            return false;
+    }
+    static_assert(sizeof(GemmArgs) <= sizeof(ExecOp), "the op area holds the grouped problems");
+    for (int i = 0; i < n_ops; ++i) {
+        const nvfp4_op &o = ops[i];
+        *st = validate_gemm(&o.A, &o.W, o.M, o.N, o.K, o.epi, o.bias, o.residual, o.ldr, o.out_bf16, o.ldo,
+                            o.out_codes, o.out_sf, o.out_global_scale);
+        if (*st == NVFP4_OK && o.M <= 0) *st = NVFP4_ERR_UNSUPPORTED_SHAPE;
+        if (*st != NVFP4_OK) return true;
+    }
+    uint32_t *status = status_word();
+    if (status == nullptr) {
+        *st = NVFP4_ERR_CUDA;
+        return true;
+    }
+    std::vector<GemmArgs> probs(static_cast<size_t>(n_ops));
+    std::vector<CUtensorMap> maps(static_cast<size_t>(n_ops) * 2);
+    std::vector<int> tab(static_cast<size_t>(4 * n_ops + 1));
+    int total = 0;
+    for (int i = 0; i < n_ops; ++i) {
+        const nvfp4_op &o = ops[i];
+        GemmArgs &p = probs[i];
+        p = GemmArgs{};
+        p.M = o.M;
+        p.N = o.N;
+        p.K = o.K;
+        p.k_atoms = (o.K + 63) / 64;
+        p.k_tiles = (o.K + 255) / 256;
+        p.kt_per_split = p.k_tiles;
+        p.splits = 1;
+        p.n_tiles = o.N / 128;
+        p.a_box_rows = static_cast<uint32_t>(o.M >= 128 ? 128 : (o.M + 7) / 8 * 8);
+        p.sfa = o.A.sf;
+        p.sfb = o.W.sf;
+        p.alpha = o.A.global_scale * o.W.global_scale;
+        p.epi = static_cast<int>(o.epi);
+        p.bias = static_cast<const uint16_t *>(o.bias);
+        p.residual = static_cast<const uint16_t *>(o.residual);
+        p.ldr = o.ldr;
+        p.out = static_cast<uint16_t *>(o.out_bf16);
+        p.ldo = o.ldo;
+        p.out_codes = o.out_codes;
+        p.out_sf = o.out_sf;
+        p.g_out = o.out_global_scale;
+        p.status = status;
+        if (!make_code_map(&maps[2 * i], o.A.codes, o.M, o.K / 2, static_cast<int>(p.a_box_rows)) ||
+            !make_code_map(&maps[2 * i + 1], o.W.codes, o.N, o.K / 2, 128)) {
+            *st = NVFP4_ERR_CUDA;
+            return true;
+        }
+        const int m_tiles = (o.M + 127) / 128;
+        tab[i] = total;
+        tab[n_ops + 1 + i] = m_tiles;
+        tab[2 * n_ops + 1 + i] = p.k_tiles;
+        tab[3 * n_ops + 1 + i] = p.k_atoms;
+        total += m_tiles * p.n_tiles;
+    }
+    tab[n_ops] = total;
+    if (cudaMemcpy(base + maps_off, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) !=
+            cudaSuccess ||
+        cudaMemcpy(base + ops_off, probs.data(), probs.size() * sizeof(GemmArgs), cudaMemcpyHostToDevice) !=
+            cudaSuccess ||
+        cudaMemcpy(base + tab_off, tab.data(), tab.size() * sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+        *st = NVFP4_ERR_CUDA;
+        return true;
+    }
+    const int sms = sm_count_cached();
+    prog->grid = total < sms ? total : sms;
+    prog->kind = 1;
+    prog->epi = static_cast<int>(ops[0].epi);
+    prog->tiles = total;
+    prog->waits = 0;
+    *st = NVFP4_OK;
+    return true;
 }
 
 nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream) {
     if (prog == nullptr || prog->buffer == nullptr || prog->n_ops <= 0) return NVFP4_ERR_INVALID_ARG;
     uint8_t *base = static_cast<uint8_t *>(prog->buffer);
+    if (prog->kind == 1) {
+        GroupedParams g;
+        g.probs = reinterpret_cast<const GemmArgs *>(base + prog->ops_offset);
+        g.maps = reinterpret_cast<const CUtensorMap *>(base + prog->maps_offset);
+        g.tab = reinterpret_cast<const int *>(base + prog->done_offset);
+        g.n_probs = prog->n_ops;
+        g.total_tiles = prog->tiles;
+        g.status = status_word();
+        if (g.status == nullptr) return NVFP4_ERR_CUDA;
+        g.trace = (g_trace != nullptr && g_trace_words >= static_cast<size_t>(prog->grid) * 8) ? g_trace : nullptr;
+        cudaError_t e = launch_gemm_grouped(g, prog->epi, prog->grid, stream);
+        if (e == cudaSuccess) e = cudaGetLastError();
+        return from_cuda(e);
+    }
     ExecParams p;
     p.ops = reinterpret_cast<const ExecOp *>(base + prog->ops_offset);
     p.maps = reinterpret_cast<const CUtensorMap *>(base + prog->maps_offset);

@@ -61,6 +61,23 @@ cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const
                              const CUtensorMap &tsb, const GemmArgs &p, cudaStream_t s);
 cudaError_t probe_gemm_pair();
 
+// Grouped kernel (gemm_grouped.cu): independent problems, one epilogue kind, 128 x 128 tiles
+// numbered problem by problem, one CTA per SM.  probs[n] and maps[2n] (A with a_box_rows-row
+// boxes, W with 128-row boxes) and tab[4n + 1] (first tile of each problem and the total,
+// then m_tiles, k_tiles, k_atoms of each) in device memory.
+constexpr int kGroupedMaxProblems = 256;
+struct GroupedParams {
+    const GemmArgs *probs;
+    const CUtensorMap *maps;
+    const int *tab;
+    int n_probs;
+    int total_tiles;
+    uint32_t *status;
+    unsigned long long *trace;
+};
+cudaError_t launch_gemm_grouped(const GroupedParams &p, int epi, int grid, cudaStream_t s);
+cudaError_t probe_gemm_grouped();
+
 // Device address and size of the library-owned split-K workspace used by
 // nvfp4_gemm_noalloc (looked up once per device; allocation-free).
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes);

@@ -50,7 +50,8 @@ class _Op(C.Structure):
 class _Program(C.Structure):
     _fields_ = [("buffer", C.c_void_p), ("bytes", C.c_size_t), ("n_ops", C.c_int), ("grid", C.c_int),
                 ("cluster", C.c_int), ("ops_offset", C.c_size_t), ("maps_offset", C.c_size_t),
-                ("done_offset", C.c_size_t), ("waits", C.c_int)]
+                ("done_offset", C.c_size_t), ("waits", C.c_int), ("kind", C.c_int), ("epi", C.c_int),
+                ("tiles", C.c_int)]
 
 
 _lib = None
