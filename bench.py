@@ -40,11 +40,11 @@ DIT = dict(M=41, H=1536, F=6144)
 # kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                 "sha256": "2be4db985612d63018ff52978875ca1e296bb5c4fac37f912a37b44e8e6651b2",
-                 "bytes": 4213312},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
+                 "sha256": "c02d86ea06f0bf39cd6616bf51453ef05dae1f37baccc3bc2a3552679e148ff5",
+                 "bytes": 4213504},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "b06a56937a13895ef6280ab4d01b8b746d48ed61c2e0da1c79dfa7716130afbe",
-                        "bytes": 38945280},  # profiles/gemm_persistent_prefill_m968_full.md
+                        "sha256": "d6145caab9fe16acf1c1d1dff391d0982d8c2032b529bc85ff7e8eb0e52ab62e",
+                        "bytes": 38958080},  # profiles/gemm_persistent_prefill_m968_full.md
 }
 
 
@@ -75,7 +75,7 @@ def parse():
     ap.add_argument("--soak-steps", type=int, default=200,
                     help="untimed steps while the clock sampler starts (0 for profiling runs)")
     ap.add_argument("--profile-case", default=None,
-                    help="run one small case for ncu (dit-gemms | prefill-gemms | norm) and exit")
+                    help="run one small case for ncu (dit-gemms | prefill-gemms | grouped | norm) and exit")
     return ap.parse_args()
 
 
@@ -332,6 +332,14 @@ def profile_case(name):
         y = torch.empty_like(x)
         for _ in range(3):
             lay.forward(x, x, y)
+    elif name == "grouped":
+        M, H, G = DIT["M"], DIT["H"], 32
+        ctxq = nvfp4.quantize_norm(torch.randn(M, H, device="cuda").to(torch.bfloat16), "none")
+        outs = [torch.empty((M, H), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+        lins = [layers.Linear(0.02 * torch.randn(H, H, device="cuda").to(torch.bfloat16)) for _ in range(G)]
+        grp = nvfp4.GroupedGemm([(ctxq, l.w, outs[g]) for g, l in enumerate(lins)])
+        for _ in range(3):
+            grp.run()
     elif name == "norm":
         x = torch.randn(968, 2048, device="cuda").to(torch.bfloat16)
         g = torch.ones(2048, device="cuda").to(torch.bfloat16)
