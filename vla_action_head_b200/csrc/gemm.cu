@@ -82,14 +82,19 @@ struct Smem {
     static constexpr int kOffB = kOffA + STAGES * kA;
     static constexpr int kOffSfa = kOffB + STAGES * Cfg<BN>::kBBytes;
     static constexpr int kOffSfb = kOffSfa + STAGES * Cfg<BN>::kSfaBytes;
-    static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes;
+    // split-K partial rows for the cluster reduction (owner slots: S x ceil(rows / S) rows,
+    // S <= 8).  At SMALL_A and BN 64 they have a region of their own, so a CTA may push its
+    // partials while its peers' MMAs still read their stages; otherwise they reuse the stages.
+    static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
+    static constexpr bool kSepRed = SMALL_A && BN == 64;
+    static constexpr int kRedBytes = ((SMALL_A ? 64 : 128) + 8) * kRedLd * 4;
+    static constexpr int kOffRed = kSepRed ? kOffSfb + STAGES * Cfg<BN>::kSfbBytes : 0;
+    static constexpr int kOffBar = kOffSfb + STAGES * Cfg<BN>::kSfbBytes + (kSepRed ? kRedBytes : 0);
     // barriers: full[STAGES], empty[STAGES], acc, sf_ready[kSlots], sf_free[kSlots]
     static constexpr int kOffMisc = kOffBar + (2 * STAGES + 1 + 2 * Cfg<BN>::kSlots) * 8;
     static constexpr int kBytes = kOffMisc + 16 + 1024;  // + alignment slack
-    // split-K partial tile for the cluster reduction, reusing the stage buffers
-    static constexpr int kRedLd = BN + 4;  // floats per row (padded against bank conflicts)
-    // owner slots of the cluster split-K reduction: S x ceil(rows / S) rows, S <= 8
-    static_assert(((SMALL_A ? 64 : 128) + 8) * kRedLd * 4 <= kOffBar, "reduction slots must fit the stages");
+    static_assert(kSepRed || kRedBytes <= kOffBar, "reduction slots must fit the stages");
+    static_assert(!SMALL_A || kBytes <= 113 * 1024, "two CTAs per SM");
     static_assert(Cfg<BN>::kBBytes >= 8192, "SMALL_A window overlaps the W tile");
 };
 
@@ -163,6 +168,12 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    // With a separate reduction region the only cluster-wide requirement before the partial
+    // rows are pushed is that every peer has started (its shared memory exists): a cluster
+    // barrier here, while the previous kernel still runs (programmatic launch), covers it.
+    if constexpr (S::kSepRed) {
+        if (p.cluster) cluster_sync_all();
+    }
     if (trace != nullptr && threadIdx.x == 0) {
         trace[0] = t_entry;
         trace[2] = globaltimer_ns();
@@ -359,8 +370,9 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
 
     if (p.cluster) {
         // Deterministic split-K reduction over distributed shared memory.  CTA `rank` of the
-        // cluster (= its split) owns local rows rank, rank + S, ...  (1) a cluster barrier:
-        // every CTA's MMAs are done with its stage buffers, which now hold partials; (2) every
+        // cluster (= its split) owns local rows rank, rank + S, ...  (1) a cluster barrier
+        // (only where the partial slots reuse the stages): every CTA's MMAs are done with its
+        // stage buffers, which now hold partials; (2) every
         // CTA pushes each of its accumulator rows into slot [split][row / S] of the row's
         // owner (remote stores, nothing waits on them); (3) a cluster barrier: all partials
         // landed; (4) all threads of each owner add its rows' S partials from its own shared
@@ -371,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
         const int rank = static_cast<int>(cluster_ctarank());
         const int rows_valid = min(SMALL_A ? 64 : 128, p.M - m0);
         const int R = (rows_valid + S_ - 1) / S_;  // rows per owner
-        float *part = reinterpret_cast<float *>(smem);
+        float *part = reinterpret_cast<float *>(smem + S::kOffRed);
         if (warp < 2) pdl_wait();  // the residual may come from the previous kernel
         auto reduce = [&](auto width) {
             constexpr int W = decltype(width)::value;
@@ -385,7 +397,10 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
                 if (has_res) load_bf16<W>(p.residual + static_cast<size_t>(m0 + i0) * p.ldr + n0 + ch0 * W, rw0);
             }
             __syncwarp();
-            cluster_sync_all();  // (1)
+            // (1): the stages become partial slots; with a region of their own only this CTA's
+            // threads need to meet (every one reads the accumulator-valid word below)
+            if constexpr (!S::kSepRed) cluster_sync_all();
+            else __syncthreads();
             if (trace != nullptr && threadIdx.x == 64) trace[7] = globaltimer_ns();
             const bool acc_ok = misc[3] != 0u;
             if (warp >= 2 && acc_ok) {
@@ -579,7 +594,7 @@ int gemm_wave_ctas(bool small, int block_n, int cluster) {
     if (c == 0) {
         int v = 0;
         switch (block_n) {
-        case 64: v = small ? wave_ctas_of<64, 5, true>(cluster) : wave_ctas_of<64, 6, false>(cluster); break;
+        case 64: v = small ? wave_ctas_of<64, 4, true>(cluster) : wave_ctas_of<64, 6, false>(cluster); break;
         case 128: v = small ? wave_ctas_of<128, 3, true>(cluster) : wave_ctas_of<128, 5, false>(cluster); break;
         default: v = small ? wave_ctas_of<256, 2, true>(cluster) : wave_ctas_of<256, 3, false>(cluster); break;
         }
@@ -595,7 +610,7 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
     // M <= 64: ~100 KB of shared memory and <= 256 TMEM columns, so two CTAs share an SM and
     // the next GEMM prefetches its weights while this one finishes.  Larger M: deep pipelines.
     switch (block_n) {
-    case 64: return small ? launch_bn<64, 5, true>(ta, tb, p, s) : launch_bn<64, 6, false>(ta, tb, p, s);
+    case 64: return small ? launch_bn<64, 4, true>(ta, tb, p, s) : launch_bn<64, 6, false>(ta, tb, p, s);
     case 128: return small ? launch_bn<128, 3, true>(ta, tb, p, s) : launch_bn<128, 5, false>(ta, tb, p, s);
     case 256: return small ? launch_bn<256, 2, true>(ta, tb, p, s) : launch_bn<256, 3, false>(ta, tb, p, s);
     default: return cudaErrorInvalidValue;
