@@ -285,6 +285,17 @@ def cpu_baseline_dit(steps=1, threads=1):
     return dt / steps * 1e6  # us per layer
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def reference_arm(args):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -474,7 +485,7 @@ def main():
             us_cpu = cpu_baseline_dit(1)
             line["cpu_baseline"] = {"value": round(us_cpu, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
                                     "sample": "one full DiT layer (M=41, hidden 1536, FFN 6144), fp64 GEMM, "
-                                              "single-threaded C"}
+                                              "single-threaded C", "cpu_model": cpu_model()}
         except Exception as e:  # the baseline is reported, never required
             line["cpu_baseline"] = {"value": None, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": str(e)}
         try:
@@ -580,6 +591,23 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     ae_w = sum(l.weight_bytes() for l in ae[0].linears())
     out["action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
                                     "weight_stream_gbs": round(18 * ae_w / (ms * 1e-3) / 1e9, 1)}
+    # its four GEMMs alone, each over the 18 layers' weights (L2-cold)
+    a0 = ae[0]
+    ae_per = {}
+    res50 = torch.zeros((50, 1024), dtype=torch.bfloat16, device=dev)
+    with torch.cuda.stream(stream):
+        for name, A, attr, epi, N, K in [("qkv", a0.a1, "qkv", "none", 2560, 1024),
+                                         ("o", a0.ctx_q, "o", "residual", 1024, 2048),
+                                         ("gate_up", a0.a2, "gate_up", "geglu", 8192, 1024),
+                                         ("down", a0.u, "down", "residual", 1024, 4096)]:
+            outs = ([nvfp4.empty_fp4(50, N // 2, dev) for _ in range(2)] if epi == "geglu" else
+                    [torch.empty((50, N), dtype=torch.bfloat16, device=dev) for _ in range(2)])
+            ms_g = gemm_ring_time(A, [getattr(l, attr) for l in ae], epi, outs, wsp, stream,
+                                  res=res50 if epi == "residual" else None)
+            b = gemm_bytes(50, N, K, epi)
+            ae_per[name] = {"us": round(ms_g * 1e3, 3), "gbs": round(b / (ms_g * 1e-3) / 1e9, 1), "bytes": b,
+                            "frac_hbm": round(b / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    out["action_expert_stack18"]["per_gemm"] = ae_per
     del ae, xa, ab
     # ---- the same stack with the gated residual updates fused into the norm front-ends ----
     with torch.cuda.stream(stream):
@@ -655,6 +683,33 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                       "bound": "hbm" if hbm_bound else "tensor",
                       "frac": round(gbs / pk["hbm_gbs"] if hbm_bound else tf / fp4_peak, 4)})
     out["m_sweep_1536x6144"] = sweep
+    # ---- norm -> NVFP4 alone at the configs' shapes, over 48 distinct inputs per replay ----
+    norm_res = {}
+    for label, Mn, Kn, kind in [("adaln_41x1536", 41, 1536, "adaln"), ("layernorm_41x1536", 41, 1536, "layernorm"),
+                                ("adarms_50x1024", 50, 1024, "adarms"), ("rmsnorm_968x2048", 968, 2048, "rmsnorm")]:
+        with torch.cuda.stream(stream):
+            xs = [synth.bf16_normal_torch(synth.seed_of(8, 500 + i), (Mn, Kn), device=dev) for i in range(48)]
+            gam = synth.bf16_normal_torch(synth.seed_of(8, synth.GAMMA), (Kn,), 1.0, 0.1, device=dev)
+            bet = synth.bf16_normal_torch(synth.seed_of(8, synth.BETA), (Kn,), 0.0, 0.1, device=dev)
+            sc = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SCALE), (Kn,), 0.0, 0.1, device=dev)
+            sh = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SHIFT), (Kn,), 0.0, 0.1, device=dev)
+            prm = {"layernorm": dict(gamma=gam, beta=bet, eps=1e-5), "rmsnorm": dict(gamma=gam, eps=1e-6),
+                   "adaln": dict(scale=sc, shift=sh, eps=1e-6), "adarms": dict(scale=sc, eps=1e-6)}[kind]
+            qo = nvfp4.empty_fp4(Mn, Kn, dev)
+
+            def norms(xs=xs, kind=kind, prm=prm, qo=qo):
+                for xi in xs:
+                    nvfp4.quantize_norm(xi, kind, out=qo, **prm)
+            norms()
+        torch.cuda.synchronize()
+        g = capture(norms, stream)
+        ms_n = time_graph(g, 10, stream) / len(xs)
+        del g
+        nb = 2 * Mn * Kn + Mn * Kn // 2 + Mn * Kn // 16 + 2 * Kn * (2 if kind in ("layernorm", "adaln") else 1)
+        norm_res[label] = {"us": round(ms_n * 1e3, 3), "gbs": round(nb / (ms_n * 1e-3) / 1e9, 1), "bytes": nb,
+                           "frac_hbm": round(nb / (ms_n * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del xs
+    out["norm_quant"] = norm_res
     # ---- tiny config: LayerNorm->NVFP4 of 41 x 256, then 41 x 512 x 256 GEMM + bias ----
     with torch.cuda.stream(stream):
         tl = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(1, synth.W0 + 100 * i), (512, 256), 0, 0.02,
