@@ -651,16 +651,25 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     with torch.cuda.stream(stream):
         outs = [nvfp4.empty_fp4(968, 16384, dev) for _ in range(2)]
         ms_gu = gemm_ring_time(pre[0].a2, [p.gate_up for p in pre], "geglu", outs, wsp, stream, reps=10)
+        outs_q = [torch.empty((968, 2560), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        ms_q = gemm_ring_time(pre[0].a1, [p.qkv for p in pre], "none", outs_q, wsp, stream, reps=10)
+        # down: 64 tiles of 128 x 256 with K = 16384 split in two through the workspace
+        outs_d = [torch.empty((968, 2048), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        ms_dn = gemm_ring_time(pre[0].u, [p.down for p in pre], "residual", outs_d, wsp, stream, reps=10, res=xp)
     tf_gu = 2.0 * 968 * 32768 * 2048 / (ms_gu * 1e-3) / 1e12
     out["prefill_m968"] = {"us_per_layer": round(ms * 1e3, 2), "tflops": round(tf, 1),
-                           "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1)}
+                           "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1),
+                           "qkv_us": round(ms_q * 1e3, 2),
+                           "qkv_tflops": round(2.0 * 968 * 2560 * 2048 / (ms_q * 1e-3) / 1e12, 1),
+                           "down_us": round(ms_dn * 1e3, 2),
+                           "down_tflops": round(2.0 * 968 * 2048 * 16384 / (ms_dn * 1e-3) / 1e12, 1)}
     out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_peak, 1),
                             "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4),
                             "traffic": traffic("prefill_gate_up"),
                             "algorithmic_bytes_per_launch": gemm_bytes(968, 32768, 2048, "geglu"),
                             "kernel": "gemm_persistent_kernel gate_up 968x32768x2048 GeGLU->FP4",
                             "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)"}
-    del pre, xp, yp, outs
+    del pre, xp, yp, outs, outs_q, outs_d
     # ---- M sweep on the 1536 -> 6144 GEMM (bias, bf16 out), 48 distinct weights ----
     with torch.cuda.stream(stream):
         lins = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(5, 1000 + i), (6144, 1536), 0, 0.02,

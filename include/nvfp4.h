@@ -109,10 +109,13 @@ size_t nvfp4_sf_offset(int row, int kblk, int K);
 /* Zeroes a scale-factor buffer (cudaMemsetAsync); once per allocation is enough. */
 nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream);
 
-/* Workspace bytes nvfp4_gemm needs for this shape; 0 if none.  The default schedule reduces
- * split-K partials inside a thread-block cluster (distributed shared memory) and needs no
- * workspace; schedules that reduce through global memory (more than 8 splits, or the ones
- * selected by negative `splits` in nvfp4_gemm_ex) need tile tickets + fp32 partials.  A
+/* Workspace bytes nvfp4_gemm needs for this shape; 0 if none.  For M <= 128 the default
+ * schedule reduces split-K partials inside a thread-block cluster (distributed shared
+ * memory) and needs no workspace; schedules that reduce through global memory (more than 8
+ * splits, the ones selected by negative `splits` in nvfp4_gemm_ex, and the many-row (M > 128)
+ * schedule when it splits K in two because the shape has fewer output tiles than SMs, e.g.
+ * 968 x 2048 x 16384) need tile counters + fp32 partials (splits x M x N x 4 bytes; the
+ * many-row schedule rounds M up to whole 128-row tiles).  A
  * workspace must be zeroed once at allocation; every call leaves its ticket words zero
  * again (after NVFP4_ERR_TIMEOUT, zero it again). */
 size_t nvfp4_gemm_workspace_bytes(int M, int N, int K);

@@ -42,6 +42,12 @@ def test_workspace_sizes(L):
     assert ws >= 4 * 41 * 1536 * 4
     assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 0, -1) > 0
     assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 96, 1) == 0  # N % 96 != 0
+    # many rows: 64 tiles of 128 x 256 on 148 SMs, K = 16384 split in two through the
+    # workspace (two counters per tile, 512 bytes + two fp32 partials of 8 whole 128-row
+    # tiles x N)
+    assert L.nvfp4_gemm_workspace_bytes(968, 2048, 16384) == 512 + 2 * 1024 * 2048 * 4
+    assert L.nvfp4_gemm_workspace_bytes(968, 32768, 2048) == 0  # 1024 tiles: no split
+    assert L.nvfp4_gemm_workspace_bytes(968, 2560, 2048) == 0  # 80 tiles, 8 K tiles: no split
 
 
 def _t(codes=0x1000, sf=0x2000, g=1.0, rows=4, K=64):

@@ -153,6 +153,41 @@ def test_persistent_multi_tile_and_tails(orc, pair_mode):
     _run(orc, 968, 4096, 512, "geglu", rows=rows)
 
 
+@pytest.mark.parametrize("epi", ["none", "bias_residual", "bias_gelu", "geglu"])
+def test_persistent_split_k(orc, epi):
+    """Fewer output tiles than SMs and a long K: the many-row kernel splits K in two through
+    the workspace (M = 256, N = 512, K = 8192: 8 tiles of 128 x 128, 16 units of 16 K
+    tiles).  The second split of a tile to arrive adds the other's partial to its own."""
+    assert nvfp4.lib().nvfp4_gemm_workspace_bytes(256, 512, 8192) > 0  # the split schedule
+    _run(orc, 256, 512, 8192, epi, rows=[0, 1, 77, 127, 128, 200, 255])
+
+
+def test_persistent_split_k_prefill_down(orc):
+    """The prefill down projection: 968 x 2048 x 16384 + residual, 64 tiles of 128 x 256,
+    K split in two (128 units), the M tail of 72 rows."""
+    assert nvfp4.lib().nvfp4_gemm_workspace_bytes(968, 2048, 16384) > 0
+    _run(orc, 968, 2048, 16384, "residual", rows=[0, 127, 128, 500, 895, 896, 967])
+
+
+def test_persistent_split_k_deterministic_and_tickets_reset(orc):
+    """Two runs give the same bytes whichever split arrives last, and every ticket word is
+    zero again afterwards (the workspace is reusable without clearing)."""
+    import torch
+    M, N, K = 968, 2048, 16384
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 36, M, N, K)
+    A, W = to_gpu_fp4(ac, asf, ga, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+    ws = nvfp4.Workspace(torch.device("cuda"))
+    o1 = host(nvfp4.gemm(A, W, "none", workspace=ws))
+    o2 = host(nvfp4.gemm(A, W, "none", workspace=ws))
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    assert np.array_equal(o1, o2)
+    need = nvfp4.lib().nvfp4_gemm_workspace_bytes(M, N, K)
+    buf, _ = ws.get(need)
+    tickets = host(buf[:256].view(torch.int32))
+    assert not tickets.any()
+
+
 def test_pair_and_one_cta_agree(orc):
     """The two many-row kernels give the same bytes (same per-element fp32 sums)."""
     import torch

@@ -182,37 +182,48 @@ Schedule choose(int M, int N, int K, bool fp4_out) {
     return finish(bn, 1, K);
 }
 
-// The many-row schedule: 256 or 128 = the one-CTA persistent kernel with that tile width,
-// kPairTiles = 256 x 256 tiles on CTA pairs.  Cost: waves x the relative time of a wave
-// (a 128-wide tile does half the work of a 256-wide one for 0.72 of its time: the wider
-// tile is bound by shared-memory traffic, which the pair kernel halves for W).
-// nvfp4_set_pair_mode (or NVFP4_GEMM_PAIR=0 / 1 in the environment) turns the pair kernel
-// off / on wherever it applies.  Off by default: on B200 its copies of the scale atoms into
-// both CTAs' tensor memory cost about twice those of one CTA, and the 256 x 256 tiles ran
-// slower than the one-CTA 128 x 256 tiles (prefill gate/up 55 us against 45 us).
+// The many-row schedule: block_n 256 or 128 = the one-CTA persistent kernel with that tile
+// width and `splits` (1 or 2) K splits (through the workspace), or kPairTiles = 256 x 256
+// tiles on CTA pairs.  Cost (us): waves x K tiles per unit x the measured time of a K tile
+// (0.82 at 256 columns, 0.70 at 128: the wider tile does twice the work for 1.17x the time),
+// + 2.5 for the partial's round trip; splits must divide the K tiles.  (Four splits of the
+// 968 x 2048 x 16384 down projection measured slower than two: 41.5 against 36.6 us.)  The pair kernel is off unless
+// nvfp4_set_pair_mode (or NVFP4_GEMM_PAIR=1) turns it on: on B200 its copies of the scale
+// atoms into both CTAs' tensor memory cost about twice those of one CTA, and the 256 x 256
+// tiles ran slower than the one-CTA 128 x 256 tiles (prefill gate/up 55 us against 45 us).
 int g_pair_mode = [] {
     const char *v = getenv("NVFP4_GEMM_PAIR");
     return v == nullptr ? 0 : (v[0] == '0' ? 0 : 1);
 }();
-int choose_persistent(int M, int N) {
+struct ManyRows {
+    int block_n;  // 0: not applicable
+    int splits;
+};
+ManyRows choose_persistent(int M, int N, int K) {
     const int pair_mode = g_pair_mode;
     const int sms = sm_count_cached();
     const int m_tiles = (M + 127) / 128;
-    int best = 0;
+    const int k_tiles = (K + 255) / 256;
+    ManyRows best{0, 1};
     double best_cost = 1e30;
     for (int bn : {256, 128}) {
         if (N % bn != 0) continue;
         const int tiles = m_tiles * (N / bn);
-        const double cost = ((tiles + sms - 1) / sms) * (bn == 256 ? 1.0 : 0.72);
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = bn;
+        for (int s : {1, 2}) {
+            if (k_tiles % s != 0) continue;
+            const int units = tiles * s;
+            const double cost = ((units + sms - 1) / sms) * (k_tiles / s) * (bn == 256 ? 0.82 : 0.70) +
+                                (s > 1 ? 2.5 : 0.0);
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = ManyRows{bn, s};
+            }
         }
     }
     if (N % 256 == 0 && pair_mode != 0) {
         const int tiles = ((M + 255) / 256) * (N / 256), units = gemm_pair_clusters();
-        const double cost = ((tiles + units - 1) / units) * 0.7;
-        if (cost < best_cost || pair_mode == 1) best = kPairTiles;
+        const double cost = ((tiles + units - 1) / units) * k_tiles * 0.82 * 0.7;
+        if (cost < best_cost || pair_mode == 1) best = ManyRows{kPairTiles, 1};
     }
     return best;
 }
@@ -232,11 +243,16 @@ Schedule choose_workspace(int M, int N, int K) {
     return choose(M, N, K, false);
 }
 
-size_t workspace_for(int M, int N, const Schedule &s) {
+// Tile counters (padded to 256 bytes) + the fp32 partials.  One-tile kernel: one ticket per
+// tile, splits x M x N partials.  Persistent kernel (`persistent`): an arrival ticket and a
+// published count per tile, splits x whole 128-row tiles x N partials.
+size_t ticket_bytes(size_t tiles, bool persistent) { return (tiles * (persistent ? 8 : 4) + 255) / 256 * 256; }
+
+size_t workspace_for(int M, int N, const Schedule &s, bool persistent = false) {
     if (s.splits <= 1 || s.cluster) return 0;
     const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / s.block_n);
-    const size_t tickets = (tiles * 4 + 255) / 256 * 256;
-    return tickets + static_cast<size_t>(s.splits) * M * N * sizeof(float);
+    const size_t rows = persistent ? static_cast<size_t>((M + 127) / 128) * 128 : static_cast<size_t>(M);
+    return ticket_bytes(tiles, persistent) + static_cast<size_t>(s.splits) * rows * N * sizeof(float);
 }
 
 // Argument checks shared by nvfp4_gemm* and the GEMM op of a program (no device access).
@@ -305,8 +321,10 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
 
     Schedule sc;
     int persistent_bn = 0;  // > 0: the persistent kernel with this tile width
-    if (block_n == 0 && splits == 0 && M > 128 && (persistent_bn = choose_persistent(M, N)) > 0) {
-        sc = finish(persistent_bn == kPairTiles ? 256 : persistent_bn, 1, K, false);
+    ManyRows many{0, 1};
+    if (block_n == 0 && splits == 0 && M > 128 && (many = choose_persistent(M, N, K)).block_n > 0) {
+        persistent_bn = many.block_n;
+        sc = finish(persistent_bn == kPairTiles ? 256 : persistent_bn, many.splits, K, false);
     } else if (block_n == 0 && splits == 0) {
         sc = choose(M, N, K, epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
     } else if (block_n == 0 && splits == -1) {
@@ -318,7 +336,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
         sc = finish(block_n, splits < 0 ? -splits : splits, K, splits > 0);
         if (sc.cluster && M > 128) sc = finish(block_n, sc.splits, K, false);
     }
-    const size_t need = workspace_for(M, N, sc);
+    const size_t need = workspace_for(M, N, sc, persistent_bn > 0);
     if (need > 0) {
         if (workspace == nullptr || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
         if (!aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
@@ -350,7 +368,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if (need > 0) {
         const size_t tiles = static_cast<size_t>((M + 127) / 128) * p.n_tiles;
         p.tickets = static_cast<uint32_t *>(workspace);
-        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + (tiles * 4 + 255) / 256 * 256);
+        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + ticket_bytes(tiles, persistent_bn > 0));
     }
     const size_t ctas = persistent_bn == kPairTiles ? static_cast<size_t>(p.n_tiles) * ((M + 255) / 256) * 2
                                                     : static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
@@ -489,6 +507,12 @@ nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream) 
 
 size_t nvfp4_gemm_workspace_bytes(int M, int N, int K) {
     if (M <= 0 || N <= 0 || K <= 0 || N % 64 != 0) return 0;
+    if (M > 128) {
+        const ManyRows many = choose_persistent(M, N, K);
+        if (many.block_n > 0 && many.block_n != kPairTiles)
+            return workspace_for(M, N, finish(many.block_n, many.splits, K, false), true);
+        if (many.block_n == kPairTiles) return 0;
+    }
     return workspace_for(M, N, choose(M, N, K, false));
 }
 
@@ -770,7 +794,7 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             // split exchange 0.8, epilogue 0.6 per pass of 128 threads over 32-column items.
             for (int bn : {128, 64}) {
                 if (o.N % bn != 0 || best < 0.0) continue;
-                for (int s : {1, 2, 4}) {
+                for (int s : {1, 2}) {
                     const Schedule c = finish(bn, s, o.K, false);
                     if (kExecCluster % c.splits != 0 || (bn / c.splits) % 32 != 0) continue;
                     const int n_tiles = o.N / bn;

@@ -69,11 +69,6 @@ constexpr int kSfSlot = 32;
 constexpr int kSfAtom = 512;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 __device__ __forceinline__ unsigned int ld_acquire_cluster_smem(uint32_t addr) {
     unsigned int v;
     asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");

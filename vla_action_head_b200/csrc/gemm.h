@@ -46,7 +46,7 @@ int gemm_wave_ctas(bool small, int block_n, int cluster);
 
 // Persistent 128 x block_n tile kernel for many rows (gemm_persistent.cu): block_n 256 or
 // 128, one split.  Grid: min(tiles, SMs) CTAs.
-int gemm_persistent_grid(int M, int n_tiles);
+int gemm_persistent_grid(int M, int n_tiles, int splits);
 cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                                    cudaStream_t s);
 cudaError_t probe_gemm_persistent();

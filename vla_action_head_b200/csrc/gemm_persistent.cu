@@ -27,6 +27,12 @@
 // From separate warps they overlap (48 copies: 4490 cycles from one thread, 1011 from eight
 // warps), so two copier warps issue them and the MMA warp only issues MMAs.
 //
+// Split K in two (when a GEMM has fewer 128 x BN tiles than SMs, e.g. the prefill down
+// projection: 64 tiles of K = 16384): the CTAs walk (tile, split) units.  Each split of a
+// tile takes an arrival ticket when its accumulator is complete; the second to arrive
+// reduces, the first publishes its fp32 partial through the workspace (2 counters per tile
+// + tiles x 128 x BN floats per split).
+//
 // Every wait is bounded (sm100.cuh); an expired wait records a status and the CTA unwinds.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -76,6 +82,24 @@ struct PCfg {
 
 // Barrier of the 256 epilogue threads that also ANDs a flag across them (every decision to
 // abandon the work is taken by all eight warps together).
+// Bounded wait until the published count at p reaches target (split K: the reducer of a tile
+// waits for the splits that arrived before it; they wait on nothing, so this ends unless one
+// of them aborted).
+__device__ bool wait_published(const unsigned int *p, unsigned int target, volatile int *abort_flag, uint32_t *status) {
+    if (ld_acquire_gpu(p) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(32);
+        if (ld_acquire_gpu(p) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(status, static_cast<uint32_t>(kStatusOk), static_cast<uint32_t>(kStatusTimeoutPeer));
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ bool bar_epi_and(bool v) {
     uint32_t r;
     asm volatile(
@@ -112,15 +136,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_sfr = bar_acce + 8;            // kSlots: slot copied (an arrival per copier)
     const uint32_t bar_sff = bar_sfr + 8 * kSlots;    // kSlots: slot read by its MMAs
     const uint32_t bar_sfl = bar_sff + 8 * kSlots;    // kStages: the stage's scale atoms have landed
-    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + Cf::kOffMisc);  // [0] TMEM base, [1] abort
+    // misc: [0] TMEM base, [1] abort flag, [2] split-K arrival ticket of the current unit
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + Cf::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = (p.M + 127) / 128;
     const int tiles = m_tiles * p.n_tiles;
-    const int k_tiles = p.k_tiles;
-    const int my_tiles = static_cast<int>(blockIdx.x) < tiles ? (tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-    const int steps = my_tiles * k_tiles;
+    // work units: (tile, split); split s (0 or 1) covers K tiles [s * kps, (s + 1) * kps) (kps
+    // divides the K tiles); unit u is tile u % tiles, split u / tiles
+    const int n_splits = p.splits, kps = p.kt_per_split;
+    const int units = tiles * n_splits;
+    const int my_tiles = static_cast<int>(blockIdx.x) < units ? (units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+    const int steps = my_tiles * kps;
     unsigned long long *trace = p.trace != nullptr ? p.trace + 8ull * blockIdx.x : nullptr;
     if (trace != nullptr && threadIdx.x == 0) trace[0] = globaltimer_ns();
 
@@ -152,23 +180,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
 
     auto nkb_of = [&](int kt) { return min(4, p.k_atoms - 4 * kt); };
-    auto tile_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
+    auto unit_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
+    auto tile_of = [&](int i) { return unit_of(i) % tiles; };
+    // A walk over this CTA's steps: unit i, its tile t, step j of the unit = global K tile
+    // kt0 + j.  Advancing costs an increment; the divisions run once per unit.
+    struct Walk {
+        int i, j, t, kt0;
+    };
+    auto walk_unit = [&](Walk &w) {
+        const int u = unit_of(w.i);
+        w.t = u % tiles;
+        w.kt0 = (u / tiles) * kps;
+    };
+    auto walk_next = [&](Walk &w) {
+        if (++w.j == kps) {
+            w.j = 0;
+            ++w.i;
+            walk_unit(w);
+        }
+    };
+    auto walk_start = [&]() {
+        Walk w{0, 0, 0, 0};
+        walk_unit(w);
+        return w;
+    };
 
     if (warp == 0) {
         // ------------------------------ producer (whole warp) ------------------------------
         const uint64_t pol = policy_evict_last();  // A and W both fit in L2 and are re-read
         // The scale atoms complete on their own barrier (sf_full) and are issued before the code
         // tiles: the copiers move them into tensor memory while the 48 KB of codes still land.
-        auto expect = [&](int st) {
-            const int nkb = nkb_of(st % k_tiles);
+        auto expect = [&](int st, const Walk &w) {
+            const int nkb = nkb_of(w.kt0 + w.j);
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar_sfl + 8 * (st % kStages), static_cast<uint32_t>(nkb) * (1u + kGroups) * kSfAtom);
                 mbar_arrive_expect_tx(bar_full + 8 * (st % kStages), kStageA + kStageB);
             }
             __syncwarp();
         };
-        auto issue_w = [&](int st) {
-            const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
+        auto issue_w = [&](int st, const Walk &w) {
+            const int s = st % kStages, t = w.t, kt = w.kt0 + w.j;
             const int n_tile = t / m_tiles, nkb = nkb_of(kt);
             const uint32_t full = bar_full + 8 * s, sfl = bar_sfl + 8 * s, base = sbase + s * kStage;
             if (lane < kGroups) {  // the k-blocks' atoms of each 128-row group are contiguous
@@ -179,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) tma_load_2d(base + kOffB, &tmB, kt * 128, n_tile * BN, full, pol);
         };
-        auto issue_a = [&](int st) {
-            const int s = st % kStages, t = tile_of(st / k_tiles), kt = st % k_tiles;
+        auto issue_a = [&](int st, const Walk &w) {
+            const int s = st % kStages, t = w.t, kt = w.kt0 + w.j;
             const int m_tile = t % m_tiles, nkb = nkb_of(kt);
             const uint32_t full = bar_full + 8 * s, sfl = bar_sfl + 8 * s, base = sbase + s * kStage;
             if (lane == 0) {
@@ -190,12 +241,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         const int pre = min(kStages, steps);
-        for (int st = 0; st < pre; ++st) {
-            expect(st);
-            issue_w(st);
+        Walk wk = walk_start();
+        for (int st = 0; st < pre; ++st, walk_next(wk)) {
+            expect(st, wk);
+            issue_w(st, wk);
         }
         pdl_wait();  // A and its scales come from the previous kernel
-        for (int st = 0; st < pre; ++st) issue_a(st);
+        {
+            Walk wa = walk_start();
+            for (int st = 0; st < pre; ++st, walk_next(wa)) issue_a(st, wa);
+        }
         int issued = pre;
         for (int st = pre; st < steps; ++st) {
             const int s = st % kStages, use = st / kStages;
@@ -203,10 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0)
                 ok = mbar_wait(bar_empty + 8 * s, (use - 1) & 1, abort_flag, p.status, kStatusTimeoutEmpty);
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-            expect(st);
-            issue_w(st);
-            issue_a(st);
+            expect(st, wk);
+            issue_w(st, wk);
+            issue_a(st, wk);
             issued = st + 1;
+            walk_next(wk);
         }
         // every issued stage must have landed before the CTA may exit
         if (lane == 0)
@@ -224,8 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 tc_fence_after();
                 bool ok = true;
-                for (int kt = 0; kt < k_tiles; ++kt, ++st) {
-                    const int s = st % kStages, slot = st % kSlots;
+                const int kt0 = (unit_of(i) / tiles) * kps;
+                for (int j = 0; j < kps; ++j, ++st) {
+                    const int s = st % kStages, slot = st % kSlots, kt = kt0 + j;
                     if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull) ||
                         !mbar_wait(bar_sfr + 8 * slot, (st / kSlots) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
                         ok = false;
@@ -238,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_mxf4nvf4(tmem, desc_kmajor_sw128(base + 32 * kb), desc_kmajor_sw128(base + kOffB + 32 * kb),
                                         idesc, t_sf + 4 * kb, t_sf + 16 + 4 * kGroups * kb,
-                                        (kt > 0 || kb > 0) ? 1u : 0u);
+                                        (j > 0 || kb > 0) ? 1u : 0u);
                     tc_commit(bar_empty + 8 * s);     // frees the stage once these MMAs have read it
                     tc_commit(bar_sff + 8 * slot);    // and the scale slot
                 }
@@ -253,8 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // overlap, and with two scale slots they overlap the MMAs of the previous stage too.
             // Copier c takes k-blocks 2c and 2c + 1 of every stage.
             const int c = warp - 10;
-            for (int st = 0; st < steps; ++st) {
-                const int s = st % kStages, slot = st % kSlots, kt = st % k_tiles;
+            Walk wk = walk_start();
+            for (int st = 0; st < steps; ++st, walk_next(wk)) {
+                const int s = st % kStages, slot = st % kSlots, kt = wk.kt0 + wk.j;
                 if (!mbar_wait(bar_sfl + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull))
                     break;
                 if (st >= kSlots && !mbar_wait(bar_sff + 8 * slot, (st / kSlots - 1) & 1, abort_flag, p.status,
@@ -289,25 +347,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                 e != 0 || mbar_wait(bar_accf, i & 1, abort_flag, p.status, kStatusTimeoutAccum);
             if (!bar_epi_and(got && *abort_flag == 0)) break;
             tc_fence_after();
-            uint32_t r[kChunks][32];
             const uint32_t t_row =
                 tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * (BN / 2));
+            const int m = m_tile * 128 + row;
+            const int n = n_tile * BN + half * (BN / 2);
+            // Split K, arrive then publish: a split takes the tile's arrival ticket first.  The
+            // last to arrive reduces; every other one copies its fp32 partial to the workspace in
+            // the threads' own order (float4 (c, j) of epilogue thread e at ((split * tiles + t) *
+            // 8 kChunks + 8 c + j) * 256 + e: a warp's store covers 512 contiguous bytes) and
+            // counts itself published.  The reducer waits (bounded) for the S - 1 others, which
+            // arrived before it and wait on nothing, then adds the partials in split order 0..S-1,
+            // its own straight from tensor memory (the same sum whichever split arrives last).
+            const int split = unit_of(i) / tiles;
+            constexpr int kVec = kChunks * 8;  // float4 per thread
+            float4 *part = n_splits > 1 ? reinterpret_cast<float4 *>(p.partials) + static_cast<size_t>(t) * kVec * 256 + e
+                                        : nullptr;
+            const size_t split_stride = static_cast<size_t>(tiles) * kVec * 256;
+            bool reducer = n_splits == 1;
+            if (n_splits > 1) {
+                if (e == 0) misc[2] = atomicAdd(p.tickets + 2 * t, 1u);
+                bar_epi_and(true);
+                reducer = misc[2] == static_cast<uint32_t>(n_splits - 1);
+            }
+            if (!reducer) {
+                uint32_t r[kChunks][32];
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
-            tmem_ld_wait();
+                for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
+                tmem_ld_wait();
+                tc_fence_before();
+                bar_epi_and(true);
+                if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
+                if (m < p.M) {
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            __stcg(part + split * split_stride + (8 * c + j) * 256,
+                                   make_float4(__uint_as_float(r[c][4 * j]), __uint_as_float(r[c][4 * j + 1]),
+                                               __uint_as_float(r[c][4 * j + 2]), __uint_as_float(r[c][4 * j + 3])));
+                }
+                __threadfence();
+                bar_epi_and(true);
+                if (e == 0) atomicAdd(p.tickets + 2 * t + 1, 1u);  // published
+                continue;
+            }
+            if (n_splits == 1) {
+                uint32_t r[kChunks][32];
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
+                tmem_ld_wait();
+                tc_fence_before();
+                bar_epi_and(true);
+                if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
+                if (m < p.M) {
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) {
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
+                        epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
+                    }
+                }
+                continue;
+            }
+            // the reducer
+            const bool pub = e != 0 || wait_published(p.tickets + 2 * t + 1, static_cast<unsigned>(n_splits - 1),
+                                                       abort_flag, p.status);
+            if (!bar_epi_and(pub && *abort_flag == 0)) break;
+            __threadfence();
+            {
+                // S = 2.  Every line this thread will read (the other split's partial, the
+                // residual row) is prefetched into L1 first, so the chunks' loads do not each
+                // wait a round trip to L2.  The prefetches follow the acquire of the publish
+                // count, and no older copy of a partial line can sit in L1: L1 does not keep
+                // global data across launches, and within a launch each line is read once, here.
+                const float4 *oth = part + (1 - split) * split_stride;
+                if (m < p.M) {
+#pragma unroll
+                    for (int j = 0; j < kVec; ++j) prefetch_l1(oth + j * 256);
+                    if constexpr (EPI == kEpiResidual || EPI == kEpiBiasResidual) {
+                        const uint16_t *rr = p.residual + static_cast<size_t>(m) * p.ldr + n;
+#pragma unroll
+                        for (int k = 0; k < BN / 2; k += 64) prefetch_l1(rr + k);
+                        prefetch_l1(rr + BN / 2 - 1);
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < kChunks; ++c) {
+                    uint32_t own[32];
+                    tmem_ld_32x32b_x32(t_row + 32 * c, own);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        float v[32];  // p0 + p1 (IEEE addition commutes: the same bits either way)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 w = oth[(8 * c + j) * 256];
+                            v[4 * j] = __fadd_rn(__uint_as_float(own[4 * j]), w.x);
+                            v[4 * j + 1] = __fadd_rn(__uint_as_float(own[4 * j + 1]), w.y);
+                            v[4 * j + 2] = __fadd_rn(__uint_as_float(own[4 * j + 2]), w.z);
+                            v[4 * j + 3] = __fadd_rn(__uint_as_float(own[4 * j + 3]), w.w);
+                        }
+                        epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
+                    }
+                }
+            }
             tc_fence_before();
             bar_epi_and(true);
-            if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
-            const int m = m_tile * 128 + row;
-            if (m < p.M) {
-                const int n = n_tile * BN + half * (BN / 2);
-#pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
-                    epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
-                }
+            if (e == 0) {
+                mbar_arrive(bar_acce);  // the MMA warp may start the next tile
+                p.tickets[2 * t] = 0u;  // ready for the next call
+                p.tickets[2 * t + 1] = 0u;
             }
         }
     }
@@ -332,12 +481,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-int gemm_persistent_grid(int M, int n_tiles) {
+int gemm_persistent_grid(int M, int n_tiles, int splits) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         sms = 148;
-    const int tiles = ((M + 127) / 128) * n_tiles;
-    return tiles < sms ? tiles : sms;
+    const int units = ((M + 127) / 128) * n_tiles * (splits > 1 ? splits : 1);
+    return units < sms ? units : sms;
 }
 
 template <int BN, int EPI>
@@ -350,7 +499,7 @@ static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, cons
         attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(gemm_persistent_grid(p.M, p.n_tiles));
+    cfg.gridDim = dim3(gemm_persistent_grid(p.M, p.n_tiles, p.splits));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = PCfg<BN>::kSmemBytes;
     cfg.stream = s;
@@ -377,6 +526,9 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
 
 cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                                    cudaStream_t s) {
+    // 1 or 2 splits that tile the K tiles exactly; a split run needs its tickets and partials
+    if (p.splits < 1 || p.splits > 2 || p.kt_per_split * p.splits != p.k_tiles) return cudaErrorInvalidValue;
+    if (p.splits > 1 && (p.tickets == nullptr || p.partials == nullptr)) return cudaErrorInvalidValue;
     if (block_n == 256) return launch_bn<256>(ta, tb, p, s);
     if (block_n == 128) return launch_bn<128>(ta, tb, p, s);
     return cudaErrorInvalidValue;
