@@ -64,7 +64,9 @@ struct PCfg {
     static constexpr int kOffSfb = kOffSfa + kStageSfa;
     static constexpr int kStage = kOffSfb + kStageSfb;  // 54 KB (BN 256) / 36 KB (BN 128)
     static constexpr int kStages = (216 * 1024) / kStage;
-    static constexpr int kOffBar = kStages * kStage;
+    // per epilogue warp, 1 KB to stage 16 rows x 64 bytes of bf16 output / residual
+    static constexpr int kOffStaging = kStages * kStage;
+    static constexpr int kOffBar = kOffStaging + 8 * 1024;
     // scale columns: kSlots slots (step modulo kSlots) of [A: 4 k-blocks x 4 | W: 4 k-blocks x
     // groups x 4]; the copies of a step may run up to kSlots - 1 steps ahead of its MMAs
     static constexpr int kSlots = 2;
@@ -100,6 +102,88 @@ __device__ bool wait_published(const unsigned int *p, unsigned int target, volat
     }
 }
 
+// bf16 epilogue of one 32-column chunk of a warp's 32 rows (lane l holds row m0 + l, values
+// v of columns n .. n + 31): v * alpha (+ bias) (+ residual), rounded to bf16, the same
+// arithmetic as epilogue_chunk.  The residual is read and the output written through a 1 KB
+// shared-memory buffer, 16 rows at a time, so that 4 lanes move the 64 bytes of one row
+// (8 rows per warp access) instead of 32 lanes each touching a different row.  16-byte piece
+// q of staged row r sits at r * 64 + 16 * (q ^ ((r >> 1) & 3)): both access patterns are
+// free of bank conflicts.  Every lane of the warp must call it (rows >= M are not touched).
+template <int EPI>
+__device__ __forceinline__ void bf16_chunk_staged(const GemmArgs &p, int m0, int lane, int n, float *v,
+                                                  uint8_t *stage) {
+    const float alpha = p.alpha;
+    const int M = p.M;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], alpha);
+    if constexpr (EPI == kEpiBias || EPI == kEpiBiasResidual) {
+        uint32_t bw[16];
+        load_bf16<32>(p.bias + n, bw);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            v[2 * t] = __fadd_rn(v[2 * t], bf16lo(bw[t]));
+            v[2 * t + 1] = __fadd_rn(v[2 * t + 1], bf16hi(bw[t]));
+        }
+    }
+    auto slot = [&](int r, int q) { return reinterpret_cast<uint4 *>(stage + r * 64 + 16 * (q ^ ((r >> 1) & 3))); };
+    const int q = lane & 3;
+    if constexpr (EPI == kEpiResidual || EPI == kEpiBiasResidual) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int r = (lane >> 2) + 8 * k, row = m0 + 16 * h + r;
+                uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                if (row < M) u = *reinterpret_cast<const uint4 *>(p.residual + static_cast<size_t>(row) * p.ldr + n + 8 * q);
+                *slot(r, q) = u;
+            }
+            __syncwarp();
+            if ((lane >> 4) == h) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 u = *slot(lane & 15, j);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        v[8 * j + 2 * t] = __fadd_rn(v[8 * j + 2 * t], bf16lo(w[t]));
+                        v[8 * j + 2 * t + 1] = __fadd_rn(v[8 * j + 2 * t + 1], bf16hi(w[t]));
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if ((lane >> 4) == h) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *slot(lane & 15, j) = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                                 pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                                 pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int r = (lane >> 2) + 8 * k, row = m0 + 16 * h + r;
+            const uint4 u = *slot(r, q);
+            if (row < M) *reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(row) * p.ldo + n + 8 * q) = u;
+        }
+        __syncwarp();
+    }
+}
+
+// One 32-column chunk of the epilogue: bf16 kinds through the staging buffer (every lane),
+// FP4 kinds per row.
+template <int EPI>
+__device__ __forceinline__ void chunk_out(const GemmArgs &p, int m0, int lane, int n, float *v, uint8_t *stage) {
+    if constexpr (EPI == kEpiBiasGelu || EPI == kEpiGeglu) {
+        if (m0 + lane < p.M) epilogue_chunk<32, EPI>(p, m0 + lane, n, v);
+    } else {
+        bf16_chunk_staged<EPI>(p, m0, lane, n, v, stage);
+    }
+}
+
 __device__ __forceinline__ bool bar_epi_and(bool v) {
     uint32_t r;
     asm volatile(
@@ -118,7 +202,9 @@ __device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint32
     return mbar_wait(bar, parity, &dummy, status, kStatusTimeoutDrain);
 }
 
-template <int BN, int EPI>
+// SPLIT: K split in two (p.splits == 2); a separate instance, so the unsplit kernel carries
+// none of the split epilogue.
+template <int BN, int EPI, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const GemmArgs p) {
@@ -145,7 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tiles = m_tiles * p.n_tiles;
     // work units: (tile, split); split s (0 or 1) covers K tiles [s * kps, (s + 1) * kps) (kps
     // divides the K tiles); unit u is tile u % tiles, split u / tiles
-    const int n_splits = p.splits, kps = p.kt_per_split;
+    constexpr int n_splits = SPLIT ? 2 : 1;
+    const int kps = p.kt_per_split;
     const int units = tiles * n_splits;
     const int my_tiles = static_cast<int>(blockIdx.x) < units ? (units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
     const int steps = my_tiles * kps;
@@ -339,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kChunks = BN / 64;   // 32-column chunks per thread
         const int row = q * 32 + lane;
         const int e = threadIdx.x - 64;
+        uint8_t *const stage = smem + Cf::kOffStaging + (warp - 2) * 1024;
         pdl_wait();  // residuals may come from the previous kernel
         for (int i = 0; i < my_tiles; ++i) {
             const int t = tile_of(i);
@@ -351,6 +439,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(half * (BN / 2));
             const int m = m_tile * 128 + row;
             const int n = n_tile * BN + half * (BN / 2);
+            if constexpr (!SPLIT) {
+                if (i + 1 < my_tiles) {
+                    // another tile follows: drain the accumulator at once and hand it back, so
+                    // this epilogue runs under the next tile's MMAs
+                    uint32_t r[kChunks][32];
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    bar_epi_and(true);
+                    if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
+                    if (m < p.M) {
+#pragma unroll
+                        for (int c = 0; c < kChunks; ++c) {
+                            float v[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
+                            epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
+                        }
+                    }
+                } else {
+                    // the CTA's last tile: nothing runs under its epilogue, which is the launch's
+                    // tail; read the accumulator a chunk at a time (few registers live) and
+                    // store through the staging buffer
+#pragma unroll 1
+                    for (int c = 0; c < kChunks; ++c) {
+                        uint32_t a[32];
+                        tmem_ld_32x32b_x32(t_row + 32 * c, a);
+                        tmem_ld_wait();
+                        float v[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]);
+                        chunk_out<EPI>(p, m - lane, lane, n + 32 * c, v, stage);
+                    }
+                    tc_fence_before();
+                    bar_epi_and(true);
+                    if (e == 0) mbar_arrive(bar_acce);
+                }
+                continue;
+            }
             // Split K, arrive then publish: a split takes the tile's arrival ticket first.  The
             // last to arrive reduces; every other one copies its fp32 partial to the workspace in
             // the threads' own order (float4 (c, j) of epilogue thread e at ((split * tiles + t) *
@@ -360,16 +488,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // its own straight from tensor memory (the same sum whichever split arrives last).
             const int split = unit_of(i) / tiles;
             constexpr int kVec = kChunks * 8;  // float4 per thread
-            float4 *part = n_splits > 1 ? reinterpret_cast<float4 *>(p.partials) + static_cast<size_t>(t) * kVec * 256 + e
-                                        : nullptr;
+            float4 *part = reinterpret_cast<float4 *>(p.partials) + static_cast<size_t>(t) * kVec * 256 + e;
             const size_t split_stride = static_cast<size_t>(tiles) * kVec * 256;
-            bool reducer = n_splits == 1;
-            if (n_splits > 1) {
-                if (e == 0) misc[2] = atomicAdd(p.tickets + 2 * t, 1u);
-                bar_epi_and(true);
-                reducer = misc[2] == static_cast<uint32_t>(n_splits - 1);
-            }
-            if (!reducer) {
+            if (e == 0) misc[2] = atomicAdd(p.tickets + 2 * t, 1u);
+            bar_epi_and(true);
+            if (misc[2] == 0u) {  // first to arrive: publish
                 uint32_t r[kChunks][32];
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
@@ -391,64 +514,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (e == 0) atomicAdd(p.tickets + 2 * t + 1, 1u);  // published
                 continue;
             }
-            if (n_splits == 1) {
-                uint32_t r[kChunks][32];
-#pragma unroll
-                for (int c = 0; c < kChunks; ++c) tmem_ld_32x32b_x32(t_row + 32 * c, r[c]);
-                tmem_ld_wait();
-                tc_fence_before();
-                bar_epi_and(true);
-                if (e == 0) mbar_arrive(bar_acce);  // the MMA warp may start the next tile
-                if (m < p.M) {
-#pragma unroll
-                    for (int c = 0; c < kChunks; ++c) {
-                        float v[32];
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[c][j]);
-                        epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
-                    }
-                }
-                continue;
-            }
             // the reducer
-            const bool pub = e != 0 || wait_published(p.tickets + 2 * t + 1, static_cast<unsigned>(n_splits - 1),
-                                                       abort_flag, p.status);
+            const bool pub = e != 0 || wait_published(p.tickets + 2 * t + 1, 1u, abort_flag, p.status);
             if (!bar_epi_and(pub && *abort_flag == 0)) break;
             __threadfence();
             {
-                // S = 2.  Every line this thread will read (the other split's partial, the
-                // residual row) is prefetched into L1 first, so the chunks' loads do not each
-                // wait a round trip to L2.  The prefetches follow the acquire of the publish
+                // S = 2.  Every line of the other split's partial this thread will read is
+                // prefetched into L1 first, so the chunks' loads do not each wait a round trip
+                // to L2.  The prefetches follow the acquire of the publish
                 // count, and no older copy of a partial line can sit in L1: L1 does not keep
                 // global data across launches, and within a launch each line is read once, here.
                 const float4 *oth = part + (1 - split) * split_stride;
                 if (m < p.M) {
 #pragma unroll
                     for (int j = 0; j < kVec; ++j) prefetch_l1(oth + j * 256);
-                    if constexpr (EPI == kEpiResidual || EPI == kEpiBiasResidual) {
-                        const uint16_t *rr = p.residual + static_cast<size_t>(m) * p.ldr + n;
-#pragma unroll
-                        for (int k = 0; k < BN / 2; k += 64) prefetch_l1(rr + k);
-                        prefetch_l1(rr + BN / 2 - 1);
-                    }
                 }
 #pragma unroll 1
                 for (int c = 0; c < kChunks; ++c) {
                     uint32_t own[32];
                     tmem_ld_32x32b_x32(t_row + 32 * c, own);
                     tmem_ld_wait();
-                    if (m < p.M) {
-                        float v[32];  // p0 + p1 (IEEE addition commutes: the same bits either way)
+                    float v[32];  // p0 + p1 (IEEE addition commutes: the same bits either way)
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 w = oth[(8 * c + j) * 256];
-                            v[4 * j] = __fadd_rn(__uint_as_float(own[4 * j]), w.x);
-                            v[4 * j + 1] = __fadd_rn(__uint_as_float(own[4 * j + 1]), w.y);
-                            v[4 * j + 2] = __fadd_rn(__uint_as_float(own[4 * j + 2]), w.z);
-                            v[4 * j + 3] = __fadd_rn(__uint_as_float(own[4 * j + 3]), w.w);
-                        }
-                        epilogue_chunk<32, EPI>(p, m, n + 32 * c, v);
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 w = m < p.M ? oth[(8 * c + j) * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        v[4 * j] = __fadd_rn(__uint_as_float(own[4 * j]), w.x);
+                        v[4 * j + 1] = __fadd_rn(__uint_as_float(own[4 * j + 1]), w.y);
+                        v[4 * j + 2] = __fadd_rn(__uint_as_float(own[4 * j + 2]), w.z);
+                        v[4 * j + 3] = __fadd_rn(__uint_as_float(own[4 * j + 3]), w.w);
                     }
+                    chunk_out<EPI>(p, m - lane, lane, n + 32 * c, v, stage);
                 }
             }
             tc_fence_before();
@@ -489,11 +584,11 @@ int gemm_persistent_grid(int M, int n_tiles, int splits) {
     return units < sms ? units : sms;
 }
 
-template <int BN, int EPI>
-static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+template <int BN, int EPI, bool SPLIT>
+static cudaError_t launch_split(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_persistent_kernel<BN, EPI>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_persistent_kernel<BN, EPI, SPLIT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, PCfg<BN>::kSmemBytes);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -508,7 +603,12 @@ static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<BN, EPI>, ta, tb, p);
+    return cudaLaunchKernelEx(&cfg, gemm_persistent_kernel<BN, EPI, SPLIT>, ta, tb, p);
+}
+
+template <int BN, int EPI>
+static cudaError_t launch_epi(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
+    return p.splits > 1 ? launch_split<BN, EPI, true>(ta, tb, p, s) : launch_split<BN, EPI, false>(ta, tb, p, s);
 }
 
 template <int BN>
@@ -536,7 +636,7 @@ cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb,
 
 cudaError_t probe_gemm_persistent() {
     cudaFuncAttributes fa;
-    return cudaFuncGetAttributes(&fa, gemm_persistent_kernel<256, kEpiNone>);
+    return cudaFuncGetAttributes(&fa, gemm_persistent_kernel<256, kEpiNone, false>);
 }
 
 }  // namespace nvfp4
