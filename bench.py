@@ -40,11 +40,11 @@ DIT = dict(M=41, H=1536, F=6144)
 # kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                 "sha256": "23aa09c1ccbca7ba4fc240270812bd703912f6e5d4592c2852307e231131f85e",
-                 "bytes": 4215168},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
+                 "sha256": "b84cb403dfe41ba41b9543b09e0380b9b3fa9e743f7e51f6a7daf3428cd4fab7",
+                 "bytes": 4214848},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "d6145caab9fe16acf1c1d1dff391d0982d8c2032b529bc85ff7e8eb0e52ab62e",
-                        "bytes": 38958080},  # profiles/gemm_persistent_prefill_m968_full.md
+                        "sha256": "1ff61190044507829e083d7bc600eea7b1d6b3bc823cf6c31bb39e89976234af",
+                        "bytes": 38956032},  # profiles/gemm_persistent_prefill_m968_full.md
 }
 
 
