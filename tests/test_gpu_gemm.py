@@ -156,10 +156,18 @@ def test_persistent_multi_tile_and_tails(orc, pair_mode):
 @pytest.mark.parametrize("epi", ["none", "bias_residual", "bias_gelu", "geglu"])
 def test_persistent_split_k(orc, epi):
     """Fewer output tiles than SMs and a long K: the many-row kernel splits K in two through
-    the workspace (M = 256, N = 512, K = 8192: 8 tiles of 128 x 128, 16 units of 16 K
-    tiles).  The second split of a tile to arrive adds the other's partial to its own."""
+    the workspace (M = 256, N = 512, K = 8192: 8 tiles of 128 x 128, 16 units, split 0 of 19
+    K tiles and split 1 of 13).  The second split of a tile to arrive adds the other's
+    partial to its own."""
     assert nvfp4.lib().nvfp4_gemm_workspace_bytes(256, 512, 8192) > 0  # the split schedule
     _run(orc, 256, 512, 8192, epi, rows=[0, 1, 77, 127, 128, 200, 255])
+
+
+def test_persistent_split_k_odd_k_tail(orc):
+    """Two unequal splits over an odd number of K tiles whose last one is ragged (K = 8320:
+    33 K tiles, the last of 128 elements): split 0 takes 20, split 1 the other 13."""
+    assert nvfp4.lib().nvfp4_gemm_workspace_bytes(256, 512, 8320) > 0
+    _run(orc, 256, 512, 8320, "bias_residual", rows=[0, 3, 127, 128, 254, 255])
 
 
 def test_persistent_split_k_prefill_down(orc):

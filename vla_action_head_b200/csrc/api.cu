@@ -195,6 +195,11 @@ int g_pair_mode = [] {
     const char *v = getenv("NVFP4_GEMM_PAIR");
     return v == nullptr ? 0 : (v[0] == '0' ? 0 : 1);
 }();
+// K tiles of the first of two splits: half, plus up to 3 so that the second split (its
+// partial published ~3 us after its accumulator is complete, ~0.6-0.8 us per K tile) is
+// usually done before the first arrives.
+int persistent_k0(int k_tiles) { return (k_tiles + 1) / 2 + std::min(3, (k_tiles - 2) / 4); }
+
 struct ManyRows {
     int block_n;  // 0: not applicable
     int splits;
@@ -210,9 +215,10 @@ ManyRows choose_persistent(int M, int N, int K) {
         if (N % bn != 0) continue;
         const int tiles = m_tiles * (N / bn);
         for (int s : {1, 2}) {
-            if (k_tiles % s != 0) continue;
+            if (s == 2 && k_tiles < 2) continue;
             const int units = tiles * s;
-            const double cost = ((units + sms - 1) / sms) * (k_tiles / s) * (bn == 256 ? 0.82 : 0.70) +
+            const double cost = ((units + sms - 1) / sms) * (s == 2 ? persistent_k0(k_tiles) : k_tiles) *
+                                    (bn == 256 ? 0.82 : 0.70) +
                                 (s > 1 ? 2.5 : 0.0);
             if (cost < best_cost) {
                 best_cost = cost;
@@ -350,6 +356,10 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     p.k_tiles = (K + 255) / 256;
     p.kt_per_split = sc.kt_per_split;
     p.splits = sc.splits;
+    if (persistent_bn > 0 && persistent_bn != kPairTiles) {
+        p.splits = many.splits;
+        p.kt_per_split = many.splits == 2 ? persistent_k0(p.k_tiles) : p.k_tiles;
+    }
     p.cluster = sc.cluster ? 1 : 0;
     p.n_tiles = N / sc.block_n;
     p.a_box_rows = static_cast<uint32_t>(M >= 128 ? 128 : (M + 7) / 8 * 8);

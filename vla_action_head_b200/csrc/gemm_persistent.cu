@@ -229,13 +229,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tiles = (p.M + 127) / 128;
     const int tiles = m_tiles * p.n_tiles;
-    // work units: (tile, split); split s (0 or 1) covers K tiles [s * kps, (s + 1) * kps) (kps
-    // divides the K tiles); unit u is tile u % tiles, split u / tiles
+    // work units: (tile, split); unit u is tile u % tiles, split u / tiles.  Split 0 covers K
+    // tiles [0, k0), split 1 [k0, k_tiles), k0 = p.kt_per_split (k_tiles without a split).
+    // The host makes split 0 a few K tiles longer, so that split 1 has usually published its
+    // partial by the time split 0 arrives and the reducer does not wait.
     constexpr int n_splits = SPLIT ? 2 : 1;
-    const int kps = p.kt_per_split;
+    const int k0 = SPLIT ? p.kt_per_split : p.k_tiles;
+    auto kt_begin_of = [&](int split) { return split != 0 ? k0 : 0; };
+    auto kt_count_of = [&](int split) { return split != 0 ? p.k_tiles - k0 : k0; };
     const int units = tiles * n_splits;
     const int my_tiles = static_cast<int>(blockIdx.x) < units ? (units - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-    const int steps = my_tiles * kps;
+    int steps = my_tiles * k0;
+    if constexpr (SPLIT) {
+        steps = 0;
+        for (int i = 0; i < my_tiles; ++i)
+            steps += kt_count_of((static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x)) / tiles);
+    }
     unsigned long long *trace = p.trace != nullptr ? p.trace + 8ull * blockIdx.x : nullptr;
     if (trace != nullptr && threadIdx.x == 0) trace[0] = globaltimer_ns();
 
@@ -269,25 +278,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto nkb_of = [&](int kt) { return min(4, p.k_atoms - 4 * kt); };
     auto unit_of = [&](int i) { return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x); };
     auto tile_of = [&](int i) { return unit_of(i) % tiles; };
-    // A walk over this CTA's steps: unit i, its tile t, step j of the unit = global K tile
-    // kt0 + j.  Advancing costs an increment; the divisions run once per unit.
+    // A walk over this CTA's steps: unit i, its tile t, step j of the unit's n K tiles = global
+    // K tile kt0 + j.  Advancing costs an increment; the divisions run once per unit.
     struct Walk {
-        int i, j, t, kt0;
+        int i, j, t, kt0, n;
     };
     auto walk_unit = [&](Walk &w) {
         const int u = unit_of(w.i);
         w.t = u % tiles;
-        w.kt0 = (u / tiles) * kps;
+        w.kt0 = kt_begin_of(u / tiles);
+        w.n = kt_count_of(u / tiles);
     };
     auto walk_next = [&](Walk &w) {
-        if (++w.j == kps) {
+        if (++w.j == w.n) {
             w.j = 0;
             ++w.i;
             walk_unit(w);
         }
     };
     auto walk_start = [&]() {
-        Walk w{0, 0, 0, 0};
+        Walk w{0, 0, 0, 0, 0};
         walk_unit(w);
         return w;
     };
@@ -367,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 tc_fence_after();
                 bool ok = true;
-                const int kt0 = (unit_of(i) / tiles) * kps;
-                for (int j = 0; j < kps; ++j, ++st) {
+                const int kt0 = kt_begin_of(unit_of(i) / tiles), cnt = kt_count_of(unit_of(i) / tiles);
+                for (int j = 0; j < cnt; ++j, ++st) {
                     const int s = st % kStages, slot = st % kSlots, kt = kt0 + j;
                     if (!mbar_wait(bar_full + 8 * s, (st / kStages) & 1, abort_flag, p.status, kStatusTimeoutFull) ||
                         !mbar_wait(bar_sfr + 8 * slot, (st / kSlots) & 1, abort_flag, p.status, kStatusTimeoutFull)) {
@@ -626,8 +636,11 @@ static cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const
 
 cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                                    cudaStream_t s) {
-    // 1 or 2 splits that tile the K tiles exactly; a split run needs its tickets and partials
-    if (p.splits < 1 || p.splits > 2 || p.kt_per_split * p.splits != p.k_tiles) return cudaErrorInvalidValue;
+    // 1 split of all K tiles, or 2 of k0 and k_tiles - k0 >= 1; a split run needs its tickets
+    // and partials
+    if (p.splits < 1 || p.splits > 2) return cudaErrorInvalidValue;
+    if (p.splits == 1 ? p.kt_per_split != p.k_tiles : (p.kt_per_split < 1 || p.kt_per_split >= p.k_tiles))
+        return cudaErrorInvalidValue;
     if (p.splits > 1 && (p.tickets == nullptr || p.partials == nullptr)) return cudaErrorInvalidValue;
     if (block_n == 256) return launch_bn<256>(ta, tb, p, s);
     if (block_n == 128) return launch_bn<128>(ta, tb, p, s);
