@@ -43,8 +43,8 @@ TRAFFIC = {
                  "sha256": "b84cb403dfe41ba41b9543b09e0380b9b3fa9e743f7e51f6a7daf3428cd4fab7",
                  "bytes": 4214848},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "1ff61190044507829e083d7bc600eea7b1d6b3bc823cf6c31bb39e89976234af",
-                        "bytes": 38956032},  # profiles/gemm_persistent_prefill_m968_full.md
+                        "sha256": "c224d89bf9815bdefeac6014e2f3724e4559664ebf9882d6f04ab74de64b7599",
+                        "bytes": 38957312},  # profiles/gemm_persistent_prefill_m968_full.md
 }
 
 
