@@ -196,6 +196,37 @@ def test_persistent_split_k_deterministic_and_tickets_reset(orc):
     assert not tickets.any()
 
 
+def test_split_k_wait_expires_and_context_survives(orc):
+    """Failure detection without a GPU fault.  Every tile's arrival ticket is preset to 1, as
+    if a split had arrived and never published its partial: both real splits of each tile
+    then take the reducer's role and wait for a partial that nobody writes.  The bounded wait
+    expires (about 2 s), the kernel records a timeout and returns, and the host reads
+    NVFP4_ERR_TIMEOUT.  The same GEMM then runs correctly on a cleared workspace."""
+    import torch
+    M, N, K = 256, 512, 8192
+    L = nvfp4.lib()
+    need = L.nvfp4_gemm_workspace_bytes(M, N, K)
+    assert need > 256  # 8 tiles: 256 bytes of counters, then the partials
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 37, M, N, K)
+    A, W = to_gpu_fp4(ac, asf, ga, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+    ws = nvfp4.Workspace(torch.device("cuda"))
+    buf, _ = ws.get(need)
+    buf[:256].view(torch.int32)[0::2] = 1  # arrival tickets; the published counts stay 0
+    nvfp4.gemm(A, W, "none", workspace=ws)
+    torch.cuda.synchronize()
+    with pytest.raises(nvfp4.NVFP4Error) as err:
+        nvfp4.device_status()
+    assert err.value.status == 7  # timeout
+    nvfp4.device_status()  # read and cleared
+    buf.zero_()
+    rows = [0, 100, 255]
+    ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi="none", rows=rows)
+    got = host(nvfp4.gemm(A, W, "none", workspace=ws))[rows]
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    check_gemm_bf16(got, ref["v"], what=("after timeout", M, N, K))
+
+
 def test_pair_and_one_cta_agree(orc):
     """The two many-row kernels give the same bytes (same per-element fp32 sums)."""
     import torch
