@@ -170,6 +170,14 @@ def test_persistent_split_k_odd_k_tail(orc):
     _run(orc, 256, 512, 8320, "bias_residual", rows=[0, 3, 127, 128, 254, 255])
 
 
+@pytest.mark.parametrize("epi", ["residual", "geglu"])
+def test_persistent_split_k_one_row_tail(orc, epi):
+    """M = 129: the second 128-row tile holds one valid row (lane 0 of the first epilogue
+    warp), so the staged bf16 stores and the split partials must skip the other 127."""
+    assert nvfp4.lib().nvfp4_gemm_workspace_bytes(129, 512, 8192) > 0
+    _run(orc, 129, 512, 8192, epi, rows=[0, 64, 127, 128])
+
+
 def test_persistent_split_k_prefill_down(orc):
     """The prefill down projection: 968 x 2048 x 16384 + residual, 64 tiles of 128 x 256,
     K split in two (128 units), the M tail of 72 rows."""
