@@ -43,7 +43,7 @@ TRAFFIC = {
                  "sha256": "b84cb403dfe41ba41b9543b09e0380b9b3fa9e743f7e51f6a7daf3428cd4fab7",
                  "bytes": 4214848},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "c224d89bf9815bdefeac6014e2f3724e4559664ebf9882d6f04ab74de64b7599",
+                        "sha256": "c7bc3b25c57f86ebe234c4b75a45614279175693494c0868f4ba008f3c515a1f",
                         "bytes": 38957312},  # profiles/gemm_persistent_prefill_m968_full.md
 }
 

@@ -489,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 continue;
             }
-            // Split K, arrive then publish: a split takes the tile's arrival ticket first.  The
-            // last to arrive reduces; every other one copies its fp32 partial to the workspace in
-            // the threads' own order (float4 (c, j) of epilogue thread e at ((split * tiles + t) *
-            // 8 kChunks + 8 c + j) * 256 + e: a warp's store covers 512 contiguous bytes) and
-            // counts itself published.  The reducer waits (bounded) for the S - 1 others, which
-            // arrived before it and wait on nothing, then adds the partials in split order 0..S-1,
-            // its own straight from tensor memory (the same sum whichever split arrives last).
+            // Split K in two, arrive then publish: a split takes the tile's arrival ticket first.
+            // The first to arrive copies its fp32 partial to the workspace in the threads' own
+            // order (float4 (c, j) of epilogue thread e at ((split * tiles + t) * 8 kChunks +
+            // 8 c + j) * 256 + e: a warp's store covers 512 contiguous bytes) and counts itself
+            // published.  The second reduces: it waits (bounded) for that count, which the first
+            // sets without waiting on anything, and adds the partial to its own accumulator read
+            // straight from tensor memory.
             const int split = unit_of(i) / tiles;
             constexpr int kVec = kChunks * 8;  // float4 per thread
             float4 *part = reinterpret_cast<float4 *>(p.partials) + static_cast<size_t>(t) * kVec * 256 + e;
@@ -529,11 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!bar_epi_and(pub && *abort_flag == 0)) break;
             __threadfence();
             {
-                // S = 2.  Every line of the other split's partial this thread will read is
-                // prefetched into L1 first, so the chunks' loads do not each wait a round trip
-                // to L2.  The prefetches follow the acquire of the publish
-                // count, and no older copy of a partial line can sit in L1: L1 does not keep
-                // global data across launches, and within a launch each line is read once, here.
+                // Every line of the other split's partial this thread will read is prefetched
+                // into L1 first, so the chunks' loads do not each wait a round trip to L2.  The
+                // prefetches follow the acquire of the published count, and no older copy of a
+                // partial line can sit in L1: L1 does not keep global data across launches, and
+                // within a launch each line is read once, here.
                 const float4 *oth = part + (1 - split) * split_stride;
                 if (m < p.M) {
 #pragma unroll
