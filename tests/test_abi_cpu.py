@@ -48,6 +48,12 @@ def test_workspace_sizes(L):
     assert L.nvfp4_gemm_workspace_bytes(968, 2048, 16384) == 512 + 2 * 1024 * 2048 * 4
     assert L.nvfp4_gemm_workspace_bytes(968, 32768, 2048) == 0  # 1024 tiles: no split
     assert L.nvfp4_gemm_workspace_bytes(968, 2560, 2048) == 0  # 80 tiles, 8 K tiles: no split
+    # 8 tiles of 128 x 128 and 32 K tiles: split in two (8 tiles' counters in 256 bytes)
+    assert L.nvfp4_gemm_workspace_bytes(256, 512, 8192) == 256 + 2 * 256 * 512 * 4
+    assert L.nvfp4_gemm_workspace_bytes(129, 512, 8192) == 256 + 2 * 256 * 512 * 4  # whole tiles
+    # 128 tiles of 128 x 128 cover the SMs at 16 K tiles: no split
+    assert L.nvfp4_gemm_workspace_bytes(968, 2048, 4096) == 0
+    assert L.nvfp4_gemm_workspace_bytes(256, 256, 512) == 0  # 2 K tiles: a split does not pay
 
 
 def _t(codes=0x1000, sf=0x2000, g=1.0, rows=4, K=64):
