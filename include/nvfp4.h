@@ -228,7 +228,9 @@ nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw
  *   bf16 epilogues write out_bf16 [M, ldo]; FP4 epilogues (BIAS_GELU, GEGLU) write
  *   out_codes [M, N_out/2] and out_sf (nvfp4_sf_bytes(M, N_out), pre-zeroed) quantized
  *   with out_global_scale, N_out = N (BIAS_GELU) or N/2 (GEGLU).
- *   workspace: >= nvfp4_gemm_workspace_bytes(M, N, K) bytes, zeroed once at allocation.
+ *   workspace: >= nvfp4_gemm_workspace_bytes(M, N, K) bytes, zeroed once at allocation;
+ *   used by one GEMM at a time (GEMMs that may run concurrently, e.g. on two streams, each
+ *   need their own).
  * Constraints: M >= 0 (0 is a no-op), K % 32 == 0 (TMA 16-byte rows; a K % 64 tail is
  * covered by the zero scale padding, [PI05] §Encoder Attention QKV NVFP4 + Scale-Factor
  * Zero-Init), N % 64 == 0. */

@@ -244,7 +244,11 @@ _default_ws = {}
 
 def gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None,
          out_global_scale=1.0, workspace: Optional[Workspace] = None, block_n=0, splits=0):
-    """a: M x K, w: N x K.  bf16 epilogues return bf16 [M, N]; FP4 epilogues an NVFP4Tensor."""
+    """a: M x K, w: N x K.  bf16 epilogues return bf16 [M, N]; FP4 epilogues an NVFP4Tensor.
+
+    workspace: split-K scratch (counters + fp32 partials), grown on demand.  Without one the
+    device's shared default is used, which is right for GEMMs issued on one stream; GEMMs
+    that may run concurrently (several streams) each need their own Workspace."""
     torch = _torch()
     M, N, K = a.rows, w.rows, a.K
     e = EPI[epi]
