@@ -13,7 +13,7 @@ replays of each DiT GEMM over L distinct weight copies), the M = 968 prefill lay
 TFLOPS (tensor-bound), the 18-layer action-expert stack, the M sweep on 1536 -> 6144, and
 the oracle on the host cores (cpu_baseline).
 
---impl reference times the oracle (the reference arm of this build) on the same workload.
+--impl reference times the oracle (the benchmark's reference arm) on the same workload.
 Multi-GPU (torchrun): independent replicas, one per rank; timing is the max over ranks.
 """
 import argparse
