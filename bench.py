@@ -36,15 +36,16 @@ FP4_OVER_BF16 = 4.0  # nominal dense ratio, 9 PF / 2.25 PF
 DIT = dict(M=41, H=1536, F=6144)
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels,
-# from the ncu captures summarised in profiles/ (commands there), keyed by a hash of the
-# kernel sources they were taken on: once a source changes the figure is reported as null.
+# from one ncu capture of each kernel (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum
+# --clock-control none -k regex:<kernel>` over `bench.py --profile-case <case>`), keyed by a hash
+# of the kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
                  "sha256": "3e94fcfbaab9669e1370efea1e832e41bcdcca7db1b9d2df5de1e05fd0a71d9a",
-                 "bytes": 4214848},  # mean of the 4 DiT GEMM launches (profiles/gemm_kernel_dit_m41_full.md)
+                 "bytes": 4214848},  # mean of the 4 DiT GEMM launches (case dit-gemms)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
                         "sha256": "73113762e02c301864f5983f6d0b89445e25b1e7e4292692390170b5132b5ed4",
-                        "bytes": 38957312},  # profiles/gemm_persistent_prefill_m968_full.md
+                        "bytes": 38957312},  # the gate/up launch of case prefill-gemms
 }
 
 

@@ -138,14 +138,6 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * rows done (norm ops) or accumulator drained to shared memory (GEMM ops). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
-/* Schedule option for the default (block_n = 0, splits = 0) schedule at M > 128: whether the
- * CTA-pair kernel (256 x 256 tiles on 2-CTA clusters, tcgen05 cta_group::2; N % 256 == 0)
- * may run.  -1: where its cost model prefers it; 0: never (the initial value, unless the
- * environment variable NVFP4_GEMM_PAIR is 1); 1: wherever N % 256 == 0.  Results are the
- * same either way (the same per-element fp32 sums).  Host-side state, not thread safe.
- * NVFP4_ERR_INVALID_ARG for other values. */
-nvfp4_status nvfp4_set_pair_mode(int mode);
-
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
 
 /* Per row of x [M, K] (leading dimension ldx, bf16 or fp32): the norm `kind`, then the
@@ -240,8 +232,9 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int
                         float out_global_scale, void *workspace, size_t ws_bytes,
                         nvfp4_stream_t stream);
 
-/* nvfp4_gemm for callers that cannot allocate device memory: no workspace argument.  The
- * paper has no counterpart to this entry point.  It serves code that is not allowed to
+/* nvfp4_gemm for callers that cannot allocate device memory: no workspace argument.  None
+ * of the source pages describes such an entry point; it is this library's own addition, and
+ * it has no counterpart there to cite.  It serves code that is not allowed to
  * call cudaMalloc (or any allocator) once it is running -- for example a plugin inside a
  * host runtime that owns every device allocation, or a real-time control loop that must
  * not allocate after start-up.  The split-K workspace instead comes from a fixed 4 MiB
@@ -255,6 +248,7 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int
  *     before any stream capture.
  *   - Every call shares the one buffer, which keeps the previous call's contents: calls that
  *     may overlap on the GPU (other streams, other host threads) race on it; serialise them.
+ *   - A call that fails the argument checks returns before it touches the buffer.
  * Otherwise the contract and results are those of nvfp4_gemm. */
 nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K,
                                 nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,

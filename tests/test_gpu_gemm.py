@@ -57,6 +57,42 @@ def test_default_schedule_bias(orc, M, N, K):
     _run(orc, M, N, K, "bias")
 
 
+# Every GEMM of the benchmarked workloads at its full size, through the DEFAULT schedule
+# (the one bench.py times: latency-model tile width and split factor at M <= 128, the
+# persistent kernel above), against the oracle.  Row samples where the oracle would take
+# long; the samples include the first and last rows and the M tail.
+CONFIG_GEMMS = [
+    # tiny: 41 x 256 -> 512 + bias
+    (41, 512, 256, "bias", None),
+    # DiT layer at M = 41, hidden 1536, FFN 6144
+    (41, 4608, 1536, "bias", None),
+    (41, 1536, 1536, "bias_residual", None),
+    (41, 6144, 1536, "bias_gelu", None),
+    (41, 1536, 6144, "bias_residual", None),
+    # action-expert layer at M = 50, width 1024, context 2048, gated MLP 2 x 4096
+    (50, 2560, 1024, "none", None),
+    (50, 1024, 2048, "residual", None),
+    (50, 8192, 1024, "geglu", None),
+    (50, 1024, 4096, "residual", None),
+    # prefill layer at M = 968, width 2048, MLP 2 x 16384
+    (968, 2560, 2048, "none", [0, 1, 127, 128, 517, 895, 896, 967]),
+    (968, 32768, 2048, "geglu", [0, 200, 895, 967]),
+    (968, 2048, 16384, "residual", [0, 128, 767, 967]),
+]
+
+
+@pytest.mark.parametrize("M,N,K,epi,rows", CONFIG_GEMMS, ids=[f"{m}x{n}x{k}-{e}" for m, n, k, e, _ in CONFIG_GEMMS])
+def test_config_gemms_default_schedule(orc, M, N, K, epi, rows):
+    _run(orc, M, N, K, epi, wl=50, rows=rows)
+
+
+@pytest.mark.parametrize("M", [1, 16, 41, 128, 512, 968])
+def test_m_sweep_default_schedule(orc, M):
+    """The M sweep on the 1536 -> 6144 GEMM (+bias), default schedule."""
+    rows = None if M <= 128 else sorted({0, 1, 127, 128, M // 2, M - 1})
+    _run(orc, M, 6144, 1536, "bias", wl=51, rows=rows)
+
+
 @pytest.mark.parametrize("bn", [64, 128, 256])
 @pytest.mark.parametrize("sp", [1, 2, 3, -2, -3])
 def test_every_tile_and_split(orc, bn, sp):
@@ -125,27 +161,17 @@ def test_device_status_clean():
 
 
 # The default schedule for many rows runs a persistent kernel: one CTA per SM walking
-# 128 x 256 or 128 x 128 tiles, or (N % 256 == 0) CTA pairs walking 256 x 256 tiles with
-# tcgen05 cta_group::2.  pair_mode pins which one; explicit (block_n, splits) runs the
-# one-tile-per-CTA kernel.
-@pytest.fixture(params=[0, 1], ids=["one_cta", "cta_pair"])
-def pair_mode(request):
-    nvfp4.set_pair_mode(request.param)
-    yield request.param
-    nvfp4.set_pair_mode(0)
-
-
+# 128 x 256 or 128 x 128 tiles; an explicit (block_n, splits) runs the one-tile-per-CTA kernel.
 @pytest.mark.parametrize("epi", ["none", "bias", "residual", "bias_residual", "bias_gelu", "geglu"])
 @pytest.mark.parametrize("N,rows", [(512, None), (10240, [0, 5, 127, 128, 255, 256, 299])])
-def test_persistent_epilogues(orc, pair_mode, epi, N, rows):
-    """One CTA per tile: N = 512 runs 128-wide tiles (12 of them), N = 10240 256-wide ones
-    (120).  CTA pairs: 4 and 80 tiles of 256 x 256; the last pair's second CTA holds no
-    valid row (M = 300)."""
+def test_persistent_epilogues(orc, epi, N, rows):
+    """N = 512 runs 128-wide tiles (12 of them), N = 10240 256-wide ones (120); M = 300
+    leaves the last 128-row tile 44 valid rows."""
     _run(orc, 300, N, 768, epi, rows=rows)
 
 
-def test_persistent_multi_tile_and_tails(orc, pair_mode):
-    """More tiles than SMs (each CTA or pair walks several), the M tail of 968 = 7 * 128 + 72,
+def test_persistent_multi_tile_and_tails(orc):
+    """More tiles than SMs (each CTA walks several), the M tail of 968 = 7 * 128 + 72,
     and a last K tile with an odd number of 64-wide blocks (K = 4160)."""
     rows = [0, 1, 63, 127, 128, 500, 767, 895, 896, 900, 960, 967]
     _run(orc, 968, 5120, 1024, "none", rows=rows)
@@ -233,24 +259,3 @@ def test_split_k_wait_expires_and_context_survives(orc):
     torch.cuda.synchronize()
     nvfp4.device_status()
     check_gemm_bf16(got, ref["v"], what=("after timeout", M, N, K))
-
-
-def test_pair_and_one_cta_agree(orc):
-    """The two many-row kernels give the same bytes (same per-element fp32 sums)."""
-    import torch
-    M, N, K = 700, 1024, 1536
-    x = synth.bf16_normal(synth.seed_of(35, synth.X), (M, K))
-    w = synth.bf16_normal(synth.seed_of(35, synth.W0), (N, K), 0.0, 0.02)
-    ac, asf = orc.quantize_norm(x, "none")
-    wc, wsf, gw = orc.quantize_weight(w)
-    A, W = to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
-    outs = []
-    for mode in (0, 1):
-        nvfp4.set_pair_mode(mode)
-        try:
-            outs.append(host(nvfp4.gemm(A, W, "none")))
-            torch.cuda.synchronize()
-            nvfp4.device_status()
-        finally:
-            nvfp4.set_pair_mode(0)
-    assert np.array_equal(outs[0], outs[1])

@@ -76,21 +76,6 @@ bool make_code_map(CUtensorMap *m, const void *ptr, int rows, int row_bytes, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scale atoms (512 bytes each: 128 rows x 4 k-blocks) as a 2-D array of 16-bit words,
-// `atoms` rows of 256; the box is 4 consecutive atoms (a 256-wide K tile of one 128-row
-// group).  Rows past the array read as zeros.
-bool make_sf_map(CUtensorMap *m, const void *ptr, int atoms) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return false;
-    cuuint64_t dims[2] = {256u, static_cast<cuuint64_t>(atoms)};
-    cuuint64_t strides[1] = {512u};
-    cuuint32_t box[2] = {256u, 4u};
-    cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 unsigned long long *g_trace = nullptr;  // diagnostics: per-CTA GEMM timestamps
 size_t g_trace_words = 0;
 size_t g_trace_cursor = 0;
@@ -183,18 +168,11 @@ Schedule choose(int M, int N, int K, bool fp4_out) {
 }
 
 // The many-row schedule: block_n 256 or 128 = the one-CTA persistent kernel with that tile
-// width and `splits` (1 or 2) K splits (through the workspace), or kPairTiles = 256 x 256
-// tiles on CTA pairs.  Cost (us): waves x K tiles per unit x the measured time of a K tile
-// (0.82 at 256 columns, 0.70 at 128: the wider tile does twice the work for 1.17x the time),
-// + 2.5 for the partial's round trip; splits must divide the K tiles.  (Four splits of the
-// 968 x 2048 x 16384 down projection measured slower than two: 41.5 against 36.6 us.)  The pair kernel is off unless
-// nvfp4_set_pair_mode (or NVFP4_GEMM_PAIR=1) turns it on: on B200 its copies of the scale
-// atoms into both CTAs' tensor memory cost about twice those of one CTA, and the 256 x 256
-// tiles ran slower than the one-CTA 128 x 256 tiles (prefill gate/up 55 us against 45 us).
-int g_pair_mode = [] {
-    const char *v = getenv("NVFP4_GEMM_PAIR");
-    return v == nullptr ? 0 : (v[0] == '0' ? 0 : 1);
-}();
+// width and `splits` (1 or 2) K splits (through the workspace).  Cost (us): waves x K tiles
+// per unit x the measured time of a K tile (0.82 at 256 columns, 0.70 at 128: the wider
+// tile does twice the work for 1.17x the time), + 2.5 for the partial's round trip; splits
+// must divide the K tiles.  (Four splits of the 968 x 2048 x 16384 down projection measured
+// slower than two: 41.5 against 36.6 us.)
 // K tiles of the first of two splits: half, plus up to 3 so that the second split (its
 // partial published ~3 us after its accumulator is complete, ~0.6-0.8 us per K tile) is
 // usually done before the first arrives.
@@ -205,7 +183,6 @@ struct ManyRows {
     int splits;
 };
 ManyRows choose_persistent(int M, int N, int K) {
-    const int pair_mode = g_pair_mode;
     const int sms = sm_count_cached();
     const int m_tiles = (M + 127) / 128;
     const int k_tiles = (K + 255) / 256;
@@ -225,11 +202,6 @@ ManyRows choose_persistent(int M, int N, int K) {
                 best = ManyRows{bn, s};
             }
         }
-    }
-    if (N % 256 == 0 && pair_mode != 0) {
-        const int tiles = ((M + 255) / 256) * (N / 256), units = gemm_pair_clusters();
-        const double cost = ((tiles + units - 1) / units) * k_tiles * 0.82 * 0.7;
-        if (cost < best_cost || pair_mode == 1) best = ManyRows{kPairTiles, 1};
     }
     return best;
 }
@@ -297,32 +269,10 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
                        const void *bias, const void *residual, int ldr, void *out_bf16, int ldo, uint8_t *out_codes,
                        uint8_t *out_sf, float out_global_scale, void *workspace, size_t ws_bytes, int block_n,
                        int splits, cudaStream_t stream) {
-    if (A == nullptr || W == nullptr) return NVFP4_ERR_INVALID_ARG;
-    if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
-    if (A->rows != M || W->rows != N || A->K != K || W->K != K) return NVFP4_ERR_INVALID_ARG;
-    if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 5) return NVFP4_ERR_INVALID_ARG;
-    if (K % 32 != 0 || N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (!scale_ok(A->global_scale) || !scale_ok(W->global_scale)) return NVFP4_ERR_INVALID_ARG;
-    if (M == 0) return NVFP4_OK;  // nothing to read or write
-    const bool fp4_out = (epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
-    const bool need_bias = (epi == NVFP4_EPI_BIAS || epi == NVFP4_EPI_BIAS_RESIDUAL || epi == NVFP4_EPI_BIAS_GELU);
-    const bool need_res = (epi == NVFP4_EPI_RESIDUAL || epi == NVFP4_EPI_BIAS_RESIDUAL);
-    if (need_bias && bias == nullptr) return NVFP4_ERR_INVALID_ARG;
-    if (need_res && (residual == nullptr || ldr < N)) return NVFP4_ERR_INVALID_ARG;
-    if (need_res && ldr % 8 != 0) return NVFP4_ERR_MISALIGNED;
-    if (fp4_out) {
-        if (out_codes == nullptr || out_sf == nullptr || !scale_ok(out_global_scale)) return NVFP4_ERR_INVALID_ARG;
-        if (!aligned16(out_codes) || !aligned16(out_sf)) return NVFP4_ERR_MISALIGNED;
-    } else {
-        if (out_bf16 == nullptr || ldo < N) return NVFP4_ERR_INVALID_ARG;
-        if (ldo % 8 != 0 || !aligned16(out_bf16)) return NVFP4_ERR_MISALIGNED;
-    }
-    if (A->codes == nullptr || A->sf == nullptr || W->codes == nullptr || W->sf == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(A->codes) || !aligned16(A->sf) || !aligned16(W->codes) || !aligned16(W->sf))
-        return NVFP4_ERR_MISALIGNED;
-    if ((bias && !aligned16(bias)) || (need_res && !aligned16(residual))) return NVFP4_ERR_MISALIGNED;
-    nvfp4_status st = check_device();
+    nvfp4_status st = validate_gemm(A, W, M, N, K, epi, bias, residual, ldr, out_bf16, ldo, out_codes, out_sf,
+                                    out_global_scale);
+    if (st != NVFP4_OK || M == 0) return st;  // M == 0: nothing to read or write
+    st = check_device();
     if (st != NVFP4_OK) return st;
 
     Schedule sc;
@@ -330,7 +280,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     ManyRows many{0, 1};
     if (block_n == 0 && splits == 0 && M > 128 && (many = choose_persistent(M, N, K)).block_n > 0) {
         persistent_bn = many.block_n;
-        sc = finish(persistent_bn == kPairTiles ? 256 : persistent_bn, many.splits, K, false);
+        sc = finish(persistent_bn, many.splits, K, false);
     } else if (block_n == 0 && splits == 0) {
         sc = choose(M, N, K, epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
     } else if (block_n == 0 && splits == -1) {
@@ -356,7 +306,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     p.k_tiles = (K + 255) / 256;
     p.kt_per_split = sc.kt_per_split;
     p.splits = sc.splits;
-    if (persistent_bn > 0 && persistent_bn != kPairTiles) {
+    if (persistent_bn > 0) {
         p.splits = many.splits;
         p.kt_per_split = many.splits == 2 ? persistent_k0(p.k_tiles) : p.k_tiles;
     }
@@ -380,27 +330,21 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
         p.tickets = static_cast<uint32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + ticket_bytes(tiles, persistent_bn > 0));
     }
-    const size_t ctas = persistent_bn == kPairTiles ? static_cast<size_t>(p.n_tiles) * ((M + 255) / 256) * 2
-                                                    : static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
+    const size_t ctas = static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
     if (g_trace != nullptr && g_trace_cursor + 8 * ctas <= g_trace_words) {
         p.trace = g_trace + g_trace_cursor;
         g_trace_cursor += 8 * ctas;
     }
-    const bool pair = persistent_bn == kPairTiles;
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb;
     if (!make_code_map(&ta, A->codes, M, K / 2, static_cast<int>(p.a_box_rows)) ||
-        !make_code_map(&tb, W->codes, N, K / 2, pair ? 128 : sc.block_n))
-        return NVFP4_ERR_CUDA;
-    if (pair && (!make_sf_map(&tsa, A->sf, (M + 127) / 128 * p.k_atoms) ||
-                 !make_sf_map(&tsb, W->sf, (N + 127) / 128 * p.k_atoms)))
+        !make_code_map(&tb, W->codes, N, K / 2, sc.block_n))
         return NVFP4_ERR_CUDA;
     // default schedule for many rows: the persistent kernel; an explicit (block_n, splits)
     // request runs the one-tile-per-CTA kernel
     const bool persistent = persistent_bn > 0;
     if (persistent && (p.status = status_word()) == nullptr) return NVFP4_ERR_CUDA;
-    cudaError_t e = pair         ? launch_gemm_pair(ta, tb, tsa, tsb, p, stream)
-                    : persistent ? launch_gemm_persistent(ta, tb, p, persistent_bn, stream)
-                                 : launch_gemm(ta, tb, p, sc.block_n, stream);
+    cudaError_t e = persistent ? launch_gemm_persistent(ta, tb, p, persistent_bn, stream)
+                               : launch_gemm(ta, tb, p, sc.block_n, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return from_cuda(e);
 }
@@ -474,7 +418,7 @@ nvfp4_status nvfp4_probe(void) {
     if (st != NVFP4_OK) return st;
     // the kernels of this library must load on the device
     if (probe_norm_kernels() != cudaSuccess || probe_gemm_kernels() != cudaSuccess ||
-        probe_gemm_persistent() != cudaSuccess || probe_gemm_pair() != cudaSuccess ||
+        probe_gemm_persistent() != cudaSuccess ||
         probe_gemm_grouped() != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
@@ -519,9 +463,7 @@ size_t nvfp4_gemm_workspace_bytes(int M, int N, int K) {
     if (M <= 0 || N <= 0 || K <= 0 || N % 64 != 0) return 0;
     if (M > 128) {
         const ManyRows many = choose_persistent(M, N, K);
-        if (many.block_n > 0 && many.block_n != kPairTiles)
-            return workspace_for(M, N, finish(many.block_n, many.splits, K, false), true);
-        if (many.block_n == kPairTiles) return 0;
+        if (many.block_n > 0) return workspace_for(M, N, finish(many.block_n, many.splits, K, false), true);
     }
     return workspace_for(M, N, choose(M, N, K, false));
 }
@@ -534,12 +476,6 @@ size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int split
     Schedule sc = finish(block_n, splits < 0 ? -splits : splits, K, splits > 0);
     if (sc.cluster && M > 128) sc = finish(block_n, sc.splits, K, false);
     return workspace_for(M, N, sc);
-}
-
-nvfp4_status nvfp4_set_pair_mode(int mode) {
-    if (mode < -1 || mode > 1) return NVFP4_ERR_INVALID_ARG;
-    g_pair_mode = mode;
-    return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
@@ -657,13 +593,16 @@ nvfp4_status nvfp4_gemm_noalloc(const nvfp4_tensor *A, const nvfp4_tensor *W, in
                                 nvfp4_epilogue epi, const void *bias, const void *residual, int ldr,
                                 void *out_bf16, int ldo, uint8_t *out_codes, uint8_t *out_sf,
                                 float out_global_scale, nvfp4_stream_t stream) {
-    size_t need = 0;
-    if (A != nullptr && W != nullptr && M > 0 && N > 0 && K > 0 && N % 64 == 0)
-        need = workspace_for(M, N, choose_workspace(M, N, K));
+    // A call that is rejected touches nothing on the device: the arguments are checked
+    // before the shared buffer's tickets are cleared.
+    nvfp4_status st = validate_gemm(A, W, M, N, K, epi, bias, residual, ldr, out_bf16, ldo, out_codes, out_sf,
+                                    out_global_scale);
+    if (st != NVFP4_OK || M == 0) return st;
+    const size_t need = workspace_for(M, N, choose_workspace(M, N, K));
     void *ws = nullptr;
     size_t ws_bytes = 0;
     if (need > 0) {
-        const nvfp4_status st = check_device();
+        st = check_device();
         if (st != NVFP4_OK) return st;
         if (noalloc_scratch(&ws, &ws_bytes) != cudaSuccess) return NVFP4_ERR_CUDA;
         if (need > ws_bytes) return NVFP4_ERR_WORKSPACE;  // shape needs more than the fixed scratch

@@ -26,6 +26,7 @@
 // unwinds: copies and MMAs in flight are drained, tensor memory is freed.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <atomic>
 #include <cstdlib>
 #include <type_traits>
 #include <cuda_runtime.h>
@@ -505,21 +506,23 @@ cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmAr
 
 // Device address of g_noalloc_scratch for the current device.  Host code only sees a
 // host-side stand-in under that name, so the address is looked up once per device (with
-// that device current) and cached; no allocation is involved.
+// that device current) and cached; no allocation is involved.  The cache entries are
+// atomics: host threads making their first calls at once each look the address up and
+// store the same value.
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes) {
     constexpr int kMaxDevices = 64;
-    static void *addr[kMaxDevices] = {};
+    static std::atomic<void *> addr[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    if (addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    void *a = addr[dev].load(std::memory_order_acquire);
+    if (a == nullptr) {
+        e = cudaGetSymbolAddress(&a, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        addr[dev] = p;
+        addr[dev].store(a, std::memory_order_release);
     }
-    *ptr = addr[dev];
+    *ptr = a;
     *bytes = kNoAllocScratchBytes;
     return cudaSuccess;
 }

@@ -51,16 +51,6 @@ cudaError_t launch_gemm_persistent(const CUtensorMap &ta, const CUtensorMap &tb,
                                    cudaStream_t s);
 cudaError_t probe_gemm_persistent();
 
-// CTA-pair kernel for many rows (gemm_pair.cu): 256 x 256 tiles, each on a 2-CTA cluster
-// (tcgen05 cta_group::2), one split.  ta: A codes, 128-row boxes; tb: W codes, 128-row
-// boxes (half a tile); tsa / tsb: the scale atoms as 2-D maps (make_sf_map).  Grid: two
-// CTAs per tile, at most gemm_pair_clusters() pairs.
-constexpr int kPairTiles = 512;  // schedule code of the pair kernel
-int gemm_pair_clusters();
-cudaError_t launch_gemm_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &tsa,
-                             const CUtensorMap &tsb, const GemmArgs &p, cudaStream_t s);
-cudaError_t probe_gemm_pair();
-
 // Grouped kernel (gemm_grouped.cu): independent problems, one epilogue kind, 128 x 128 tiles
 // numbered problem by problem, one CTA per SM.  probs[n] and maps[2n] (A with a_box_rows-row
 // boxes, W with 128-row boxes) and tab[4n + 1] (first tile of each problem and the total,

@@ -244,62 +244,6 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // ---------------------------------------------------------------------------------------
-// CTA pairs (tcgen05 cta_group::2): the two CTAs of a 2-CTA cluster share one MMA of
-// M = 256.  The leader (rank 0) issues the MMAs, scale copies and commits; each CTA holds
-// its own 128 rows of A and 128 rows of the B tile, at the same shared-memory offsets.
-// TMA load whose completion is counted on the leader's mbarrier (`leader_bar`, a
-// shared::cluster address from mapa_shared(bar, 0)); the data lands in this CTA.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *tmap, int x, int y,
-                                                 uint32_t leader_bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(leader_bar), "l"(policy)
-        : "memory");
-}
-// Allocation, permit release and deallocation of the same columns in both CTAs; one warp of
-// each CTA executes each of them.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// Scale-atom copy into the tensor memory of both CTAs, each from its own shared memory at
-// the same descriptor address.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-// D (256 x N, rows 0..127 in the leader's TMEM, 128..255 in the peer's) (+)= A x B^T with
-// per-16 UE4M3 block scales.
-__device__ __forceinline__ void tc_mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                                     uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-        "}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
-}
-// Arrives once on the executing CTA's `bar` when this thread's prior cta_group::2 tcgen05
-// operations complete.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-// The same, arriving on the mbarrier at offset `bar` in every CTA of `cta_mask`.
-__device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
-    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 ::"r"(bar), "h"(cta_mask)
-                 : "memory");
-}
-
-// ---------------------------------------------------------------------------------------
 // Matrix descriptors (tcgen05 shared-memory descriptor format, version 1 on sm_100):
 //   [0,14) start address >> 4, [16,30) leading-dim byte offset >> 4,
 //   [32,46) stride-dim byte offset >> 4, [46,48) version = 1, [49,52) base offset,

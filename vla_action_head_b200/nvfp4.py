@@ -77,7 +77,6 @@ def lib():
             "nvfp4_gemm_workspace_bytes_ex": (SZ, [I, I, I, I, I]),
             "nvfp4_get_device_status": (I, [P]),
             "nvfp4_set_gemm_trace": (I, [P, SZ]),
-            "nvfp4_set_pair_mode": (I, [I]),
             "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
             "nvfp4_residual_quantize_norm": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, P, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
@@ -280,12 +279,6 @@ def gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, o
 
 def probe():
     _check("nvfp4_probe", lib().nvfp4_probe())
-
-
-def set_pair_mode(mode: int):
-    """-1: the CTA-pair GEMM kernel where its cost model prefers it; 0: never (the default);
-    1: wherever it applies (N % 256 == 0, M > 128, default schedule)."""
-    _check("nvfp4_set_pair_mode", lib().nvfp4_set_pair_mode(int(mode)))
 
 
 def device_status():
