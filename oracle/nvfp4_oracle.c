@@ -431,6 +431,202 @@ float orc_quantize_weight_mse(const uint16_t *w, int N, int K, int ldw, int inte
     return g;
 }
 
+/* ------------------------------------------------------------------------------------ */
+/* 16-point Hadamard rotation of one block ("Pi0.5 Thor NVFP4 End-to-End Results",
+ * §Full-INT4 Decoder Activations + Hadamard Rotation: every 16-value block of both GEMM
+ * operands is rotated by the orthonormal 16 x 16 Hadamard matrix before quantization;
+ * lane-parallel kernels run it as a 4-stage shfl_xor butterfly, vectorized kernels as an
+ * in-register fast Walsh-Hadamard transform; the rotation leaves the GEMM unchanged).
+ * The matrix is Sylvester's H16, entry (i, j) = (-1)^popcount(i & j), times 1/4, which
+ * makes it orthonormal and its own inverse.
+ * READING: the four butterfly stages pair element i with element i ^ d for d = 1, 2, 4, 8
+ * in that order; of each pair the element whose index has bit d clear becomes a + b and
+ * the other a - b (a the lower-index value), each one fp32 addition or subtraction
+ * rounded to nearest even; the 1/4 is applied last, one fp32 multiply per element (exact
+ * unless the result is subnormal).                                                       */
+void orc_hadamard16(float *y) {
+    for (int d = 1; d < 16; d <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & d) == 0) {
+                float a = y[i], b = y[i | d];
+                y[i] = a + b;
+                y[i | d] = a - b;
+            }
+    for (int i = 0; i < 16; ++i) y[i] = y[i] * 0.25f;
+}
+
+/* The same rotation in fp64 (the reference value of a rotated fp64 activation). */
+static void hadamard16_f64(double *y) {
+    for (int d = 1; d < 16; d <<= 1)
+        for (int i = 0; i < 16; ++i)
+            if ((i & d) == 0) {
+                double a = y[i], b = y[i | d];
+                y[i] = a + b;
+                y[i | d] = a - b;
+            }
+    for (int i = 0; i < 16; ++i) y[i] = y[i] * 0.25;
+}
+
+/* Uniform INT4 elements, E0M3 ("Pi0.5 ...", §E0M3 Uniform-INT4 Decoder Weights: a
+ * sign-magnitude uniform INT4 grid, magnitudes 0..7, beside E2M1; per-16 UE4M3 block
+ * scales computed as amax / 7).
+ * READING: code bit 3 is the sign and bits 0..2 the magnitude, so code c decodes to
+ * +-(c & 7); encoding rounds |v| to the nearest integer, ties to the even integer (the
+ * rounding the E2M1 path uses), and saturates at 7; the sign of v is kept as in E2M1, so
+ * a negative value that rounds to 0 gives 0x8.  Inputs are finite.                       */
+float orc_e0m3_decode(uint8_t code) {
+    double m = (double)(code & 7u);
+    return (float)((code & 8u) ? -m : m);
+}
+
+uint8_t orc_e0m3_encode(float v) {
+    uint8_t sign = signbit(v) ? 8u : 0u;
+    double a = fabs((double)v);
+    if (a >= 7.0) return (uint8_t)(sign | 7u);
+    double fl = floor(a);
+    double fr = a - fl; /* exact: a < 8 has at most 24 significant bits */
+    int q = (int)fl;
+    if (fr > 0.5 || (fr == 0.5 && (q & 1) != 0)) q += 1;
+    return (uint8_t)(sign | (uint8_t)q);
+}
+
+/* One E0M3 block: the E2M1 block quantizer's steps with 7 in place of 6.
+ *   a = max|y|;  d = 7*g;  t = a/d;  s = E4M3(t);  S = dec(s)*g
+ *   dec(s) == 0 -> every code +0;  else r = 1/S, code_i = E0M3(y_i * r)
+ * READING: one IEEE fp32 operation per step, as for E2M1.                                 */
+uint8_t orc_quantize_block16_e0m3(const float *y, float g, uint8_t *codes8) {
+    float a = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float m = fabsf(y[i]);
+        if (m > a) a = m;
+    }
+    float d = 7.0f * g;
+    float t = a / d;
+    uint8_t s = orc_e4m3_encode(t);
+    float ds = orc_e4m3_decode(s);
+    if (ds == 0.0f) {
+        memset(codes8, 0, 8);
+        return s;
+    }
+    float S = ds * g;
+    float r = 1.0f / S;
+    for (int j = 0; j < 8; ++j) {
+        float v0 = y[2 * j] * r;
+        float v1 = y[2 * j + 1] * r;
+        codes8[j] = (uint8_t)(orc_e0m3_encode(v0) | (orc_e0m3_encode(v1) << 4));
+    }
+    return s;
+}
+
+/* A block under the quantizer options: rotated first if ORC_Q_ROTATE, then the E2M1 or
+ * (ORC_Q_E0M3) the E0M3 block quantizer.  y is not modified.                             */
+uint8_t orc_quantize_block16_ex(const float *y, float g, int flags, uint8_t *codes8) {
+    float blk[16];
+    memcpy(blk, y, sizeof blk);
+    if (flags & ORC_Q_ROTATE) orc_hadamard16(blk);
+    return (flags & ORC_Q_E0M3) ? orc_quantize_block16_e0m3(blk, g, codes8) : orc_quantize_block16(blk, g, codes8);
+}
+
+void orc_quantize_rows_ex(const float *y, int rows, int K, int ldy, float g, int flags,
+                          uint8_t *codes, uint8_t *sf) {
+    int nblk = (K + 15) / 16;
+    size_t row_bytes = (size_t)nblk * 8;
+    float blk[16];
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? y[(size_t)r * ldy + k] : 0.0f;
+            }
+            sf[orc_sf_offset(r, b, K)] =
+                orc_quantize_block16_ex(blk, g, flags, codes + (size_t)r * row_bytes + (size_t)b * 8);
+        }
+    }
+}
+
+/* Norm then quantize under the options (the rotation applies to the normalized y). */
+void orc_quantize_norm_ex(const void *x, int in_fp32, int rows, int K, int ldx, int kind,
+                          const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,
+                          const uint16_t *mod_shift, float eps, float g, int flags,
+                          uint8_t *codes, uint8_t *sf) {
+    float *y = (float *)malloc(sizeof(float) * (size_t)K);
+    size_t esz = in_fp32 ? 4 : 2;
+    int nblk = (K + 15) / 16;
+    for (int r = 0; r < rows; ++r) {
+        const char *xr = (const char *)x + (size_t)r * ldx * esz;
+        orc_norm_rows(xr, in_fp32, 1, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, y);
+        float blk[16];
+        for (int b = 0; b < nblk; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? y[k] : 0.0f;
+            }
+            sf[orc_sf_offset(r, b, K)] =
+                orc_quantize_block16_ex(blk, g, flags, codes + (size_t)r * nblk * 8 + (size_t)b * 8);
+        }
+    }
+    free(y);
+}
+
+/* Offline weight quantizer under the options.  The values quantized are the (optionally
+ * rotated) 16-element blocks of W along K, rows optionally gate/up interleaved as in
+ * orc_quantize_weight; with `mse` (E2M1 only) the block scales are the MSE search's.
+ * READING: the global scale is amax over the values actually quantized (the rotated
+ * blocks when rotating, since a rotated block's amax can reach 4x the original's) divided
+ * by (top grid magnitude x 448): 6 x 448 = 2688 for E2M1, 7 x 448 = 3136 for E0M3, so the
+ * largest block scale lands on the E4M3 maximum; an all-zero tensor takes g = 1.  The
+ * pages give E0M3 weights amax/7 block scales only, so mse with E0M3 is not defined and
+ * the E0M3 amax quantizer is used.                                                        */
+float orc_quantize_weight_ex(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up, int flags,
+                             int mse, uint8_t *codes, uint8_t *sf) {
+    int nblk = (K + 15) / 16;
+    float *vals = (float *)malloc(sizeof(float) * (size_t)N * nblk * 16);
+    float amax = 0.0f;
+    for (int r = 0; r < N; ++r) {
+        int src = r;
+        if (interleave_gate_up) src = (r % 2 == 0) ? r / 2 : N / 2 + r / 2;
+        for (int b = 0; b < nblk; ++b) {
+            float *blk = vals + ((size_t)r * nblk + b) * 16;
+            for (int i = 0; i < 16; ++i) {
+                int k = b * 16 + i;
+                blk[i] = (k < K) ? bf16_to_f32(w[(size_t)src * ldw + k]) : 0.0f;
+            }
+            if (flags & ORC_Q_ROTATE) orc_hadamard16(blk);
+            for (int i = 0; i < 16; ++i) {
+                float m = fabsf(blk[i]);
+                if (m > amax) amax = m;
+            }
+        }
+    }
+    float g = (amax == 0.0f) ? 1.0f : amax / ((flags & ORC_Q_E0M3) ? 3136.0f : 2688.0f);
+    for (int r = 0; r < N; ++r)
+        for (int b = 0; b < nblk; ++b) {
+            const float *blk = vals + ((size_t)r * nblk + b) * 16;
+            uint8_t *c8 = codes + (size_t)r * nblk * 8 + (size_t)b * 8;
+            uint8_t s;
+            if (flags & ORC_Q_E0M3) s = orc_quantize_block16_e0m3(blk, g, c8);
+            else if (mse) s = orc_quantize_block16_mse(blk, g, c8);
+            else s = orc_quantize_block16(blk, g, c8);
+            sf[orc_sf_offset(r, b, K)] = s;
+        }
+    free(vals);
+    return g;
+}
+
+/* Dequantize under the element grid of `flags` (E0M3 or E2M1); a rotation is not undone:
+ * the result is the (rotated) block the codes represent.                                  */
+void orc_dequantize_ex(const uint8_t *codes, const uint8_t *sf, float g, int rows, int K, int flags,
+                       double *out) {
+    int nblk = (K + 15) / 16;
+    for (int r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k) {
+            uint8_t byte = codes[(size_t)r * nblk * 8 + (size_t)k / 2];
+            uint8_t c = (k % 2 == 0) ? (byte & 15u) : (byte >> 4);
+            double e = (flags & ORC_Q_E0M3) ? (double)orc_e0m3_decode(c) : (double)orc_e2m1_decode(c);
+            out[(size_t)r * K + k] = e * (double)orc_e4m3_decode(sf[orc_sf_offset(r, k / 16, K)]) * (double)g;
+        }
+}
+
 /* Dequantized value of element k of row `row`: val(code) * dec(scale) * g, exact in fp64. */
 static double deq_elem(const uint8_t *codes, const uint8_t *sf, float g, int row, int k, int K) {
     int nblk = (K + 15) / 16;
@@ -462,6 +658,10 @@ double orc_gelu_tanh(double z) {
  *   v[m,n]   = acc + bias[n] + residual[m,n]        (terms present per epilogue)
  *   BIAS_GELU: h = gelu(v), N_out = N;   GEGLU: h[m,j] = gelu(v[m,2j]) * v[m,2j+1], N_out = N/2
  *   FP4 output = the block quantizer applied to (float)h along n with g_out.
+ *   BIAS_GELU_RHT / GEGLU_RHT: the same, each 16-value block of (float)h rotated by
+ *   orc_hadamard16 before the block quantizer ("Pi0.5 ...", §Full-INT4 Decoder Activations +
+ *   Hadamard Rotation: the GeGLU exit is one of the rotated activation exits, so the next
+ *   GEMM's rotated weights see a rotated input); h_out then holds the fp64 rotation of h.
  * Dequantized operands include their global scales, so acc already carries gA * gW.    */
 void orc_gemm(const uint8_t *a_codes, const uint8_t *a_sf, float gA, int M,
               const uint8_t *w_codes, const uint8_t *w_sf, float gW, int N, int K,
@@ -475,6 +675,9 @@ void orc_gemm(const uint8_t *a_codes, const uint8_t *a_sf, float gA, int M,
         int m = m_idx ? m_idx[i] : i;
         for (int k = 0; k < K; ++k) arows[(size_t)i * K + k] = deq_elem(a_codes, a_sf, gA, m, k, K);
     }
+    int rot = (epi == ORC_EPI_BIAS_GELU_RHT || epi == ORC_EPI_GEGLU_RHT);
+    if (epi == ORC_EPI_BIAS_GELU_RHT) epi = ORC_EPI_BIAS_GELU;
+    if (epi == ORC_EPI_GEGLU_RHT) epi = ORC_EPI_GEGLU;
     int use_bias = (epi == ORC_EPI_BIAS || epi == ORC_EPI_BIAS_RESIDUAL || epi == ORC_EPI_BIAS_GELU ||
                     epi == ORC_EPI_GEGLU) && bias != NULL;
     int use_res = (epi == ORC_EPI_RESIDUAL || epi == ORC_EPI_BIAS_RESIDUAL);
@@ -503,6 +706,8 @@ void orc_gemm(const uint8_t *a_codes, const uint8_t *a_sf, float gA, int M,
                 if (h_out) h_out[(size_t)i * n_out + j] = h;
                 hf[j] = (float)h;
             }
+            if (h_out && rot)
+                for (int b = 0; b + 16 <= n_out; b += 16) hadamard16_f64(h_out + (size_t)i * n_out + b);
             if (out_codes && out_sf) {
                 float blk[16];
                 for (int b = 0; b < oblk; ++b) {
@@ -510,8 +715,8 @@ void orc_gemm(const uint8_t *a_codes, const uint8_t *a_sf, float gA, int M,
                         int j = b * 16 + t;
                         blk[t] = (j < n_out) ? hf[j] : 0.0f;
                     }
-                    uint8_t s = orc_quantize_block16(blk, g_out,
-                                                     out_codes + (size_t)m * oblk * 8 + (size_t)b * 8);
+                    uint8_t s = orc_quantize_block16_ex(blk, g_out, rot ? ORC_Q_ROTATE : 0,
+                                                        out_codes + (size_t)m * oblk * 8 + (size_t)b * 8);
                     out_sf[orc_sf_offset(m, b, n_out)] = s;
                 }
             }

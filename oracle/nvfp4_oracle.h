@@ -20,6 +20,9 @@
  *    Scale-Factor Zero-Init).
  *  - Offline weight quantization, optional pairwise gate/up row interleave
  *    ("Pi0.5 ...", §Implemented Path; §Fused GeGLU Epilogue for the P1 Encoder FFN).
+ *  - The 16-point Hadamard block rotation and uniform INT4 (E0M3) elements ("Pi0.5 ...",
+ *    §Full-INT4 Decoder Activations + Hadamard Rotation; §E0M3 Uniform-INT4 Decoder
+ *    Weights), as options of the quantizers and of the FP4-output epilogues.
  *  - Block-scaled GEMM with bias / residual / tanh-GELU->FP4 / GeGLU->FP4 epilogues,
  *    GELU applied to the unrounded accumulator ("GROOT N1.7 ...", §What is in the tier;
  *    "Pi0.5 ...", §Fused GeGLU FFN in the Decoder), evaluated here in fp64.
@@ -42,7 +45,10 @@ extern "C" {
 enum { ORC_NORM_NONE = 0, ORC_NORM_LAYERNORM = 1, ORC_NORM_RMSNORM = 2, ORC_NORM_ADALN = 3,
        ORC_NORM_ADARMS = 4 };
 enum { ORC_EPI_NONE = 0, ORC_EPI_BIAS = 1, ORC_EPI_RESIDUAL = 2, ORC_EPI_BIAS_RESIDUAL = 3,
-       ORC_EPI_BIAS_GELU = 4, ORC_EPI_GEGLU = 5 };
+       ORC_EPI_BIAS_GELU = 4, ORC_EPI_GEGLU = 5, ORC_EPI_BIAS_GELU_RHT = 6, ORC_EPI_GEGLU_RHT = 7 };
+/* quantizer options: ROTATE = 16-point Hadamard rotation of each block before quantizing;
+   E0M3 = uniform INT4 elements (magnitudes 0..7, block scale amax / 7) instead of E2M1 */
+enum { ORC_Q_ROTATE = 1, ORC_Q_E0M3 = 2 };
 
 /* element codecs */
 float   orc_e2m1_decode(uint8_t code);
@@ -94,6 +100,24 @@ double orc_block_sse(const float *y, float g, uint8_t s, uint8_t *codes8);
 uint8_t orc_quantize_block16_mse(const float *y, float g, uint8_t *codes8);
 float orc_quantize_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up,
                               uint8_t *codes, uint8_t *sf);
+
+/* 16-point Hadamard rotation (in place, fp32 butterfly), E0M3 codec and block quantizer,
+ * and the quantizers / dequantizer under the options above. */
+void    orc_hadamard16(float *y);
+float   orc_e0m3_decode(uint8_t code);
+uint8_t orc_e0m3_encode(float v);
+uint8_t orc_quantize_block16_e0m3(const float *y, float g, uint8_t *codes8);
+uint8_t orc_quantize_block16_ex(const float *y, float g, int flags, uint8_t *codes8);
+void orc_quantize_rows_ex(const float *y, int rows, int K, int ldy, float g, int flags,
+                          uint8_t *codes, uint8_t *sf);
+void orc_quantize_norm_ex(const void *x, int in_fp32, int rows, int K, int ldx, int kind,
+                          const uint16_t *gamma, const uint16_t *beta, const uint16_t *mod_scale,
+                          const uint16_t *mod_shift, float eps, float g, int flags,
+                          uint8_t *codes, uint8_t *sf);
+float orc_quantize_weight_ex(const uint16_t *w, int N, int K, int ldw, int interleave_gate_up, int flags,
+                             int mse, uint8_t *codes, uint8_t *sf);
+void orc_dequantize_ex(const uint8_t *codes, const uint8_t *sf, float g, int rows, int K, int flags,
+                       double *out);
 
 /* dequantize rows -> fp64 [rows, K] */
 void orc_dequantize(const uint8_t *codes, const uint8_t *sf, float g, int rows, int K,

@@ -11,7 +11,9 @@ import numpy as np
 from . import build_oracle
 
 NORM = {"none": 0, "layernorm": 1, "rmsnorm": 2, "adaln": 3, "adarms": 4}
-EPI = {"none": 0, "bias": 1, "residual": 2, "bias_residual": 3, "bias_gelu": 4, "geglu": 5}
+EPI = {"none": 0, "bias": 1, "residual": 2, "bias_residual": 3, "bias_gelu": 4, "geglu": 5,
+       "bias_gelu_rht": 6, "geglu_rht": 7}
+ROTATE, E0M3 = 1, 2  # quantizer option bits
 
 _lib = None
 
@@ -66,6 +68,25 @@ def lib():
         L.orc_f32_to_bf16_array.argtypes = [P, C.c_size_t, P]
         L.orc_gated_residual.restype = None
         L.orc_gated_residual.argtypes = [P, P, P, C.c_int, C.c_int, P]
+        L.orc_hadamard16.restype = None
+        L.orc_hadamard16.argtypes = [P]
+        L.orc_e0m3_decode.restype = C.c_float
+        L.orc_e0m3_decode.argtypes = [C.c_uint8]
+        L.orc_e0m3_encode.restype = C.c_uint8
+        L.orc_e0m3_encode.argtypes = [C.c_float]
+        L.orc_quantize_block16_e0m3.restype = C.c_uint8
+        L.orc_quantize_block16_e0m3.argtypes = [P, C.c_float, P]
+        L.orc_quantize_block16_ex.restype = C.c_uint8
+        L.orc_quantize_block16_ex.argtypes = [P, C.c_float, C.c_int, P]
+        L.orc_quantize_rows_ex.restype = None
+        L.orc_quantize_rows_ex.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_float, C.c_int, P, P]
+        L.orc_quantize_norm_ex.restype = None
+        L.orc_quantize_norm_ex.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P,
+                                           P, C.c_float, C.c_float, C.c_int, P, P]
+        L.orc_quantize_weight_ex.restype = C.c_float
+        L.orc_quantize_weight_ex.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, P, P]
+        L.orc_dequantize_ex.restype = None
+        L.orc_dequantize_ex.argtypes = [P, P, C.c_float, C.c_int, C.c_int, C.c_int, P]
         _lib = L
     return _lib
 
@@ -133,13 +154,44 @@ def quantize_block16(y, g):
     return codes, int(s)
 
 
-def quantize_rows(y, g):
+def quantize_rows(y, g, flags=0):
+    """flags: ROTATE (Hadamard-rotate each block first) | E0M3 (uniform INT4 elements)."""
     y = _c(y, np.float32)
     rows, K = y.shape
     codes = np.zeros((rows, (K + 15) // 16 * 8), np.uint8)
     sf = np.zeros(sf_bytes(rows, K), np.uint8)
-    lib().orc_quantize_rows(_p(y), rows, K, K, float(g), _p(codes), _p(sf))
+    if flags:
+        lib().orc_quantize_rows_ex(_p(y), rows, K, K, float(g), int(flags), _p(codes), _p(sf))
+    else:
+        lib().orc_quantize_rows(_p(y), rows, K, K, float(g), _p(codes), _p(sf))
     return codes, sf
+
+
+def hadamard16(y):
+    """The fp32 16-point Hadamard rotation of each 16-value row of y ([..., 16])."""
+    y = np.array(y, dtype=np.float32, order="C")
+    flat = y.reshape(-1, 16)
+    for i in range(flat.shape[0]):
+        lib().orc_hadamard16(flat[i].ctypes.data_as(C.c_void_p))
+    return y
+
+
+def e0m3_decode(codes):
+    tbl = np.array([lib().orc_e0m3_decode(i) for i in range(16)], dtype=np.float32)
+    return tbl[np.asarray(codes, dtype=np.uint8) & 15]
+
+
+def e0m3_encode(v):
+    v = np.ascontiguousarray(v, np.float32)
+    return np.array([lib().orc_e0m3_encode(float(t)) for t in v.ravel()], np.uint8).reshape(v.shape)
+
+
+def quantize_block16_ex(y, g, flags):
+    y = _c(y, np.float32)
+    assert y.size == 16
+    codes = np.zeros(8, np.uint8)
+    s = lib().orc_quantize_block16_ex(_p(y), float(g), int(flags), _p(codes))
+    return codes, int(s)
 
 
 def norm_rows(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6):
@@ -154,15 +206,19 @@ def norm_rows(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6):
     return y
 
 
-def quantize_norm(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, g=1.0):
+def quantize_norm(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, g=1.0, flags=0):
+    """flags: ROTATE | E0M3 options of the quantizer step (0: the plain NVFP4 path)."""
     in_fp32 = 1 if np.asarray(x).dtype == np.float32 else 0
     x = _c(x, np.float32 if in_fp32 else np.uint16)
     rows, K = x.shape
     codes = np.zeros((rows, (K + 15) // 16 * 8), np.uint8)
     sf = np.zeros(sf_bytes(rows, K), np.uint8)
-    lib().orc_quantize_norm(_p(x), in_fp32, rows, K, K, NORM[kind], _p(_c(gamma, np.uint16)),
-                            _p(_c(beta, np.uint16)), _p(_c(scale, np.uint16)),
-                            _p(_c(shift, np.uint16)), float(eps), float(g), _p(codes), _p(sf))
+    args = (_p(x), in_fp32, rows, K, K, NORM[kind], _p(_c(gamma, np.uint16)), _p(_c(beta, np.uint16)),
+            _p(_c(scale, np.uint16)), _p(_c(shift, np.uint16)), float(eps), float(g))
+    if flags:
+        lib().orc_quantize_norm_ex(*args, int(flags), _p(codes), _p(sf))
+    else:
+        lib().orc_quantize_norm(*args, _p(codes), _p(sf))
     return codes, sf
 
 
@@ -212,6 +268,17 @@ def quantize_weight_mse(w, interleave_gate_up=False):
     return codes, sf, float(np.float32(g))
 
 
+def quantize_weight_ex(w, interleave_gate_up=False, flags=0, mse=False):
+    """The weight quantizer under the options (ROTATE | E0M3); mse: MSE-searched E2M1 scales."""
+    w = _c(w, np.uint16)
+    N, K = w.shape
+    codes = np.zeros((N, (K + 15) // 16 * 8), np.uint8)
+    sf = np.zeros(sf_bytes(N, K), np.uint8)
+    g = lib().orc_quantize_weight_ex(_p(w), N, K, K, int(bool(interleave_gate_up)), int(flags), int(bool(mse)),
+                                     _p(codes), _p(sf))
+    return codes, sf, float(np.float32(g))
+
+
 def block_sse(y, g, s):
     """(E(s), 8 code bytes) of one 16-value fp32 block at scale byte s."""
     y = _c(y, np.float32)
@@ -227,11 +294,15 @@ def quantize_block16_mse(y, g):
     return int(s), codes
 
 
-def dequantize(codes, sf, g, rows, K):
+def dequantize(codes, sf, g, rows, K, flags=0):
+    """flags & E0M3: the codes are E0M3 (uniform INT4); a rotation is not undone."""
     codes = _c(codes, np.uint8)
     sf = _c(sf, np.uint8)
     out = np.empty((rows, K), np.float64)
-    lib().orc_dequantize(_p(codes), _p(sf), float(g), rows, K, _p(out))
+    if flags:
+        lib().orc_dequantize_ex(_p(codes), _p(sf), float(g), rows, K, int(flags), _p(out))
+    else:
+        lib().orc_dequantize(_p(codes), _p(sf), float(g), rows, K, _p(out))
     return out
 
 
@@ -249,8 +320,8 @@ def gemm(a_codes, a_sf, gA, M, w_codes, w_sf, gW, N, K, epi="none", bias=None, r
     n_rows = M if m_idx is None else m_idx.size
     v = np.empty((n_rows, N), np.float64)
     h = codes = sf = None
-    if EPI[epi] in (4, 5):
-        n_out = N // 2 if EPI[epi] == 5 else N
+    if EPI[epi] in (4, 5, 6, 7):
+        n_out = N // 2 if EPI[epi] in (5, 7) else N
         h = np.empty((n_rows, n_out), np.float64)
         codes = np.zeros((M, (n_out + 15) // 16 * 8), np.uint8)
         sf = np.zeros(sf_bytes(M, n_out), np.uint8)
