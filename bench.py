@@ -286,6 +286,188 @@ def cpu_baseline_dit(steps=1, threads=1):
     return dt / steps * 1e6  # us per layer
 
 
+def _cpu_bits(seed, shape, mean, std):
+    import numpy as np
+    import torch
+
+    from vla_action_head_b200 import synth
+    return synth.bf16_normal_torch(seed, shape, mean, std, device="cpu").view(torch.int16).numpy().view(np.uint16)
+
+
+def _rows_gemm(threads):
+    """orc.gemm, with the output rows split over `threads` host threads when > 1 (the oracle
+    call releases the interpreter lock)."""
+    import numpy as np
+
+    from oracle import oracle as orc
+    if threads <= 1:
+        return orc.gemm, None
+    from concurrent.futures import ThreadPoolExecutor
+    pool = ThreadPoolExecutor(threads)
+
+    def gemm(*a, rows=None, **kw):
+        M = a[3]
+        sel = np.arange(M) if rows is None else np.asarray(rows)
+        parts = [p for p in np.array_split(sel, threads) if len(p)]
+        res = list(pool.map(lambda r: orc.gemm(*a, rows=r, **kw), parts))
+        out = {"v": np.concatenate([r["v"] for r in res])}
+        if res[0]["codes"] is not None:  # each part fills its own rows of zeroed buffers
+            out["codes"] = np.bitwise_or.reduce([r["codes"] for r in res])
+            out["sf"] = np.bitwise_or.reduce([r["sf"] for r in res])
+        return out
+    return gemm, pool
+
+
+def cpu_baseline_tiny(reps=3, threads=1):
+    """The oracle on the tiny workload: LayerNorm -> NVFP4 of 41 x 256, GEMM 41 x 512 x 256 +
+    bias.  us per norm + GEMM (mean of `reps`)."""
+    from oracle import oracle as orc
+    from vla_action_head_b200 import synth
+    s = lambda tid: synth.seed_of(1, tid)  # noqa: E731
+    x = _cpu_bits(s(synth.X), (41, 256), 0, 1)
+    ga, be = _cpu_bits(s(synth.GAMMA), (256,), 1, 0.1), _cpu_bits(s(synth.BETA), (256,), 0, 0.1)
+    wc, wsf, gw = orc.quantize_weight(_cpu_bits(s(synth.W0), (512, 256), 0, 0.02))
+    bias = _cpu_bits(s(synth.BIAS0), (512,), 0, 0.01)
+    gemm, pool = _rows_gemm(threads)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        a, asf = orc.quantize_norm(x, "layernorm", gamma=ga, beta=be, eps=1e-5)
+        gemm(a, asf, 1.0, 41, wc, wsf, gw, 512, 256, epi="bias", bias=bias)
+    dt = (time.perf_counter() - t0) / reps
+    if pool is not None:
+        pool.shutdown()
+    return dt * 1e6
+
+
+def cpu_baseline_ae(reps=3, threads=1):
+    """The oracle on one action-expert layer (M = 50, width 1024, context 2048, gated MLP
+    2 x 4096): 2 AdaRMSNorm -> NVFP4, context quantize, QKV, o + residual, gate/up GeGLU ->
+    FP4, down + residual.  us per layer (mean of `reps`)."""
+    from oracle import oracle as orc
+    from vla_action_head_b200 import synth
+    s = lambda tid: synth.seed_of(3, tid)  # noqa: E731
+    M, H, A, F = 50, 1024, 2048, 4096
+    x = _cpu_bits(s(synth.X), (M, H), 0, 1)
+    ctx = _cpu_bits(s(synth.CONTEXT), (M, A), 0, 1)
+    s1, s2 = _cpu_bits(s(synth.MOD_SCALE), (H,), 0, 0.1), _cpu_bits(s(synth.MOD_SHIFT), (H,), 0, 0.1)
+    shapes = [(2560, H), (H, A), (2 * F, H), (H, F)]
+    W = [orc.quantize_weight(_cpu_bits(s(synth.W0 + i), shp, 0, 0.02), interleave_gate_up=(i == 2))
+         for i, shp in enumerate(shapes)]
+    gemm, pool = _rows_gemm(threads)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        a1, a1s = orc.quantize_norm(x, "adarms", scale=s1, eps=1e-6)
+        gemm(a1, a1s, 1.0, M, *W[0], 2560, H, epi="none")
+        c, cs = orc.quantize_norm(ctx, "none")
+        h = synth.f32_to_bf16_bits(gemm(c, cs, 1.0, M, *W[1], H, A, epi="residual", residual=x)["v"])
+        a2, a2s = orc.quantize_norm(h, "adarms", scale=s2, eps=1e-6)
+        u = gemm(a2, a2s, 1.0, M, *W[2], 2 * F, H, epi="geglu")
+        gemm(u["codes"], u["sf"], 1.0, M, *W[3], H, F, epi="residual", residual=h)
+    dt = (time.perf_counter() - t0) / reps
+    if pool is not None:
+        pool.shutdown()
+    return dt * 1e6
+
+
+def _fit_rows(run, M, threads, per_thread=(8, 24)):
+    """Time run(rows) on two evenly spread row samples of per_thread x threads rows each (best
+    of two), fit t = a + b x rows (a: the weight decode each call repeats, b: the products of
+    one row) and evaluate at M rows.  Returns (us, the sample sizes)."""
+    import numpy as np
+    ns = [min(M, k * threads) for k in per_thread]
+    ts = []
+    for n in ns:
+        sel = np.linspace(0, M - 1, n).astype(np.int64)
+        best = None
+        for _ in range(2):
+            t0 = time.perf_counter()
+            run(sel)
+            dt = time.perf_counter() - t0
+            best = dt if best is None else min(best, dt)
+        ts.append(best)
+    if ns[1] == ns[0]:
+        return ts[0] * 1e6, ns
+    slope = (ts[1] - ts[0]) / (ns[1] - ns[0])
+    return (ts[0] + slope * (M - ns[0])) * 1e6, ns
+
+
+def cpu_baseline_prefill(threads=1):
+    """The oracle on one prefill layer (M = 968, width 2048, MLP 2 x 16384): 2 RMSNorm ->
+    NVFP4 over all rows, and the three GEMMs timed on two row samples and extrapolated in
+    rows (_fit_rows).  Returns (us per layer, description of the sample)."""
+    from oracle import oracle as orc
+    from vla_action_head_b200 import synth
+    s = lambda tid: synth.seed_of(4, tid)  # noqa: E731
+    M, H, F = 968, 2048, 16384
+    x = _cpu_bits(s(synth.X), (M, H), 0, 1)
+    g1, g2 = _cpu_bits(s(synth.GAMMA), (H,), 1, 0.1), _cpu_bits(s(synth.BETA), (H,), 1, 0.1)
+    Wq = orc.quantize_weight(_cpu_bits(s(synth.W0), (2560, H), 0, 0.02))
+    Wg = orc.quantize_weight(_cpu_bits(s(synth.W0 + 2), (2 * F, H), 0, 0.02), interleave_gate_up=True)
+    Wd = orc.quantize_weight(_cpu_bits(s(synth.W0 + 3), (H, F), 0, 0.02))
+    gemm, pool = _rows_gemm(threads)
+    t0 = time.perf_counter()
+    a1, a1s = orc.quantize_norm(x, "rmsnorm", gamma=g1, eps=1e-6)
+    a2, a2s = orc.quantize_norm(x, "rmsnorm", gamma=g2, eps=1e-6)
+    t_norm = time.perf_counter() - t0
+
+    def gemms(sel):
+        gemm(a1, a1s, 1.0, M, *Wq, 2560, H, epi="none", rows=sel)
+        u = gemm(a2, a2s, 1.0, M, *Wg, 2 * F, H, epi="geglu", rows=sel)
+        # u holds the sampled rows (the rest zero): the down GEMM reads the same rows
+        gemm(u["codes"], u["sf"], 1.0, M, *Wd, H, F, epi="residual", residual=x, rows=sel)
+    us, ns = _fit_rows(gemms, M, threads)
+    if pool is not None:
+        pool.shutdown()
+    return t_norm * 1e6 + us, (f"norms over all 968 rows; the 3 GEMMs timed on {ns[0]} and {ns[1]} sampled rows "
+                               "and extrapolated linearly in rows to 968")
+
+
+def cpu_baseline_sweep(threads=1):
+    """The oracle on the 1536 -> 6144 GEMM (+bias) at each M of the sweep; M > 41 timed on
+    two row samples and extrapolated in rows (_fit_rows).  {M: us}."""
+    from oracle import oracle as orc
+    from vla_action_head_b200 import synth
+    W = orc.quantize_weight(_cpu_bits(synth.seed_of(5, 1000), (6144, 1536), 0, 0.02))
+    bias = _cpu_bits(synth.seed_of(5, 2000), (6144,), 0, 0.01)
+    gemm, pool = _rows_gemm(threads)
+    out = {}
+    for Ms in (1, 16, 41, 128, 512, 968):
+        a, asf = orc.quantize_norm(_cpu_bits(synth.seed_of(5, Ms), (Ms, 1536), 0, 1), "none")
+        if Ms <= 41:
+            t0 = time.perf_counter()
+            gemm(a, asf, 1.0, Ms, *W, 6144, 1536, epi="bias", bias=bias)
+            out[Ms] = (time.perf_counter() - t0) * 1e6
+            continue
+        out[Ms], _ = _fit_rows(lambda sel: gemm(a, asf, 1.0, Ms, *W, 6144, 1536, epi="bias", bias=bias, rows=sel),
+                               Ms, threads)
+    if pool is not None:
+        pool.shutdown()
+    return out
+
+
+def cpu_baselines_all(nthr):
+    """The oracle beside every workload, single-threaded and on `nthr` host threads."""
+    res = {}
+    for name, fn, unit, reps in [("tiny_41x256_512", cpu_baseline_tiny, "µs per norm + GEMM", 3),
+                                 ("action_expert_layer_m50", cpu_baseline_ae, "µs/layer", 3)]:
+        for thr in (1, nthr):
+            us = fn(reps=reps, threads=thr)
+            res.setdefault(name, {"unit": unit, "kind": "oracle", "sample": f"the whole workload, mean of {reps}"})
+            res[name]["us_1_thread" if thr == 1 else f"us_{nthr}_threads"] = round(us, 1)
+    for thr in (1, nthr):
+        us, sample = cpu_baseline_prefill(threads=thr)
+        res.setdefault("prefill_layer_m968", {"unit": "µs/layer", "kind": "oracle", "sample": sample})
+        res["prefill_layer_m968"]["us_1_thread" if thr == 1 else f"us_{nthr}_threads"] = round(us, 1)
+    for thr in (1, nthr):
+        sw = cpu_baseline_sweep(threads=thr)
+        res.setdefault("m_sweep_1536x6144", {"unit": "µs per GEMM", "kind": "oracle",
+                                             "sample": "M <= 41 whole; larger M on 8 and 24 sampled rows per "
+                                                       "thread, extrapolated linearly in rows"})
+        res["m_sweep_1536x6144"]["us_1_thread" if thr == 1 else f"us_{nthr}_threads"] = {
+            str(k): round(v, 1) for k, v in sw.items()}
+    return res
+
+
 def cpu_model():
     try:
         with open("/proc/cpuinfo") as f:
@@ -497,6 +679,10 @@ def main():
                                             f"partitioned over {nthr} host threads"}
         except Exception as e:
             line["cpu_baseline_threads"] = {"value": None, "sample": str(e)[:200]}
+        try:
+            line["cpu_baseline_configs"] = cpu_baselines_all(len(os.sched_getaffinity(0)))
+        except Exception as e:
+            line["cpu_baseline_configs"] = {"error": repr(e)[:200]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:

@@ -72,8 +72,37 @@ typedef enum {
     NVFP4_EPI_RESIDUAL = 2,      /* + residual[m, n]                          -> bf16   */
     NVFP4_EPI_BIAS_RESIDUAL = 3, /* + bias[n] + residual[m, n]                -> bf16   */
     NVFP4_EPI_BIAS_GELU = 4,     /* gelu_tanh(acc*gA*gW + bias[n])            -> FP4    */
-    NVFP4_EPI_GEGLU = 5          /* gelu_tanh(v[m,2j]) * v[m,2j+1], v = acc*gA*gW (+bias) -> FP4, width N/2 */
+    NVFP4_EPI_GEGLU = 5,         /* gelu_tanh(v[m,2j]) * v[m,2j+1], v = acc*gA*gW (+bias) -> FP4, width N/2 */
+    /* BIAS_GELU / GEGLU with each 16-value output block rotated by the 16-point Hadamard
+     * matrix before it is quantized (NVFP4_QUANT_ROTATE below): the rotated activation
+     * exit that feeds a GEMM whose weights were quantized with NVFP4_QUANT_ROTATE
+     * ([PI05] §Full-INT4 Decoder Activations + Hadamard Rotation). */
+    NVFP4_EPI_BIAS_GELU_RHT = 6,
+    NVFP4_EPI_GEGLU_RHT = 7
 } nvfp4_epilogue;
+
+/* Quantizer options (bit flags) of the *_ex quantizers:
+ *   NVFP4_QUANT_ROTATE  rotate each 16-element block by the orthonormal Sylvester Hadamard
+ *                       matrix H16 / 4 before quantizing it ([PI05] §Full-INT4 Decoder
+ *                       Activations + Hadamard Rotation).  Rotating the blocks of both GEMM
+ *                       operands leaves the product unchanged (H16 H16^T = 16 I), so the
+ *                       block-scaled GEMM consumes rotated operands as they are.  The
+ *                       rotation is the in-register butterfly: stages d = 1, 2, 4, 8 pair
+ *                       element i with i ^ d (a + b at the lower index, a - b at the upper),
+ *                       each one fp32 add, then each element times 1/4.
+ *   NVFP4_QUANT_E0M3    uniform INT4 elements instead of E2M1 ([PI05] §E0M3 Uniform-INT4
+ *                       Decoder Weights): code bit 3 = sign, bits 0..2 = round-half-even of
+ *                       |y| / S saturated at 7; block scale s = E4M3(amax / (7 g)).  These
+ *                       codes are a storage format: nvfp4_gemm reads E2M1 codes only (the
+ *                       tensor-core E0M3 element format is not documented for sm_100a).
+ *   NVFP4_QUANT_MSE     weights only: MSE-searched block scales (as
+ *                       nvfp4_quantize_weight_mse); not with E0M3. */
+typedef enum {
+    NVFP4_QUANT_DEFAULT = 0,
+    NVFP4_QUANT_ROTATE = 1,
+    NVFP4_QUANT_E0M3 = 2,
+    NVFP4_QUANT_MSE = 4
+} nvfp4_quant_flags;
 
 typedef enum { NVFP4_IN_BF16 = 0, NVFP4_IN_FP32 = 1 } nvfp4_in_dtype;
 
@@ -114,10 +143,13 @@ nvfp4_status nvfp4_sf_zero(uint8_t *sf, int rows, int K, nvfp4_stream_t stream);
  * memory) and needs no workspace; schedules that reduce through global memory (more than 8
  * splits, the ones selected by negative `splits` in nvfp4_gemm_ex, and the many-row (M > 128)
  * schedule when it splits K in two because the shape has fewer output tiles than SMs, e.g.
- * 968 x 2048 x 16384) need tile counters + fp32 partials (splits x M x N x 4 bytes; the
- * many-row schedule rounds M up to whole 128-row tiles).  A
- * workspace must be zeroed once at allocation; every call leaves its ticket words zero
- * again (after NVFP4_ERR_TIMEOUT, zero it again). */
+ * 968 x 2048 x 16384) need a fixed 16 KiB region of tile counters followed by the fp32
+ * partials (splits x M x N x 4 bytes; the many-row schedule rounds M up to whole 128-row
+ * tiles).  A workspace must be zeroed once at allocation; every call leaves its counters
+ * zero again, and no call's partials overlap the counter region, so one workspace may serve
+ * GEMMs of different shapes one after another (after NVFP4_ERR_TIMEOUT, zero it again).
+ * Schedules whose counters exceed the region (more than 4096 tiles, 2048 for the many-row
+ * kernel) return NVFP4_ERR_UNSUPPORTED_SHAPE. */
 size_t nvfp4_gemm_workspace_bytes(int M, int N, int K);
 
 /* Reads and clears the library's device status word after synchronising `stream`:
@@ -183,6 +215,22 @@ nvfp4_status nvfp4_residual_quantize_norm(const void *x, const void *d, const vo
                                           float eps, float global_scale, void *h_out, uint8_t *codes,
                                           uint8_t *sf, nvfp4_stream_t stream);
 
+/* nvfp4_quantize_norm and nvfp4_residual_quantize_norm with quantizer options `flags`
+ * (NVFP4_QUANT_ROTATE | NVFP4_QUANT_E0M3; other bits: NVFP4_ERR_INVALID_ARG).  The rotation
+ * applies to the normalized y; with E0M3 the block scale is E4M3(amax / (7 g)).  Otherwise
+ * the arguments, constraints and results are those of the calls without _ex. */
+nvfp4_status nvfp4_quantize_norm_ex(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx,
+                                    nvfp4_norm kind, const void *gamma, const void *beta,
+                                    const void *mod_scale, const void *mod_shift, float eps,
+                                    float global_scale, int flags, uint8_t *codes, uint8_t *sf,
+                                    nvfp4_stream_t stream);
+nvfp4_status nvfp4_residual_quantize_norm_ex(const void *x, const void *d, const void *gate, int M,
+                                             int K, int ldx, int ldd, int ldh, nvfp4_norm kind,
+                                             const void *gamma, const void *beta,
+                                             const void *mod_scale, const void *mod_shift,
+                                             float eps, float global_scale, int flags, void *h_out,
+                                             uint8_t *codes, uint8_t *sf, nvfp4_stream_t stream);
+
 /* ---- offline weight quantize --------------------------------------------------------- */
 
 /* W bf16 [N, K] (ldw) -> codes [N, K/2] + sf (nvfp4_sf_bytes(N, K), pre-zeroed) with the
@@ -208,6 +256,19 @@ nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw
                                        float *global_scale_out, void *scratch,
                                        nvfp4_stream_t stream);
 
+/* The weight quantizer with options `flags` (NVFP4_QUANT_ROTATE | NVFP4_QUANT_E0M3 |
+ * NVFP4_QUANT_MSE; E0M3 with MSE or other bits: NVFP4_ERR_INVALID_ARG).  The values
+ * quantized are W's 16-element blocks along K, Hadamard-rotated with NVFP4_QUANT_ROTATE,
+ * and the global scale is their amax over (top grid magnitude x 448): amax / 2688 for E2M1,
+ * amax / 3136 for E0M3 (1 for an all-zero W) -- a rotated block's amax can be up to 4x the
+ * original's, so the amax is taken after the rotation.  ([PI05] §Full-INT4 Decoder
+ * Activations + Hadamard Rotation; §E0M3 Uniform-INT4 Decoder Weights: per-16 UE4M3 scales,
+ * amax / 7.)  Arguments otherwise as nvfp4_quantize_weight; synchronises `stream`. */
+nvfp4_status nvfp4_quantize_weight_ex(const void *w_bf16, int N, int K, int ldw,
+                                      int interleave_gate_up, int flags, uint8_t *codes,
+                                      uint8_t *sf, float *global_scale_out, void *scratch,
+                                      nvfp4_stream_t stream);
+
 /* ---- block-scaled NVFP4 GEMM with fused epilogue ------------------------------------ */
 
 /* acc[m, n] = sum_k dec(A)[m, k] * dec(W)[n, k] over the E2M1 codes and UE4M3 block scales
@@ -217,9 +278,10 @@ nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw
  * GeGLU FFN in the Decoder: GELU on the fp32 accumulator, gate/up interleaved pairwise).
  *   A: M x K activations, W: N x K weights (A->rows == M, W->rows == N, both ->K == K).
  *   bias: bf16 [N] or NULL; residual: bf16 [M, ldr] (RESIDUAL / BIAS_RESIDUAL only).
- *   bf16 epilogues write out_bf16 [M, ldo]; FP4 epilogues (BIAS_GELU, GEGLU) write
+ *   bf16 epilogues write out_bf16 [M, ldo]; FP4 epilogues (BIAS_GELU, GEGLU, and their
+ *   rotated *_RHT forms) write
  *   out_codes [M, N_out/2] and out_sf (nvfp4_sf_bytes(M, N_out), pre-zeroed) quantized
- *   with out_global_scale, N_out = N (BIAS_GELU) or N/2 (GEGLU).
+ *   with out_global_scale, N_out = N (BIAS_GELU[_RHT]) or N/2 (GEGLU[_RHT]).
  *   workspace: >= nvfp4_gemm_workspace_bytes(M, N, K) bytes, zeroed once at allocation;
  *   used by one GEMM at a time (GEMMs that may run concurrently, e.g. on two streams, each
  *   need their own).

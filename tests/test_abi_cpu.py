@@ -43,14 +43,17 @@ def test_workspace_sizes(L):
     assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 0, -1) > 0
     assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 96, 1) == 0  # N % 96 != 0
     # many rows: 64 tiles of 128 x 256 on 148 SMs, K = 16384 split in two through the
-    # workspace (two counters per tile, 512 bytes + two fp32 partials of 8 whole 128-row
+    # workspace (the fixed 16 KiB counter region, then two fp32 partials of 8 whole 128-row
     # tiles x N)
-    assert L.nvfp4_gemm_workspace_bytes(968, 2048, 16384) == 512 + 2 * 1024 * 2048 * 4
+    region = 16384
+    assert L.nvfp4_gemm_workspace_bytes(968, 2048, 16384) == region + 2 * 1024 * 2048 * 4
     assert L.nvfp4_gemm_workspace_bytes(968, 32768, 2048) == 0  # 1024 tiles: no split
     assert L.nvfp4_gemm_workspace_bytes(968, 2560, 2048) == 0  # 80 tiles, 8 K tiles: no split
-    # 8 tiles of 128 x 128 and 32 K tiles: split in two (8 tiles' counters in 256 bytes)
-    assert L.nvfp4_gemm_workspace_bytes(256, 512, 8192) == 256 + 2 * 256 * 512 * 4
-    assert L.nvfp4_gemm_workspace_bytes(129, 512, 8192) == 256 + 2 * 256 * 512 * 4  # whole tiles
+    # 8 tiles of 128 x 128 and 32 K tiles: split in two
+    assert L.nvfp4_gemm_workspace_bytes(256, 512, 8192) == region + 2 * 256 * 512 * 4
+    assert L.nvfp4_gemm_workspace_bytes(129, 512, 8192) == region + 2 * 256 * 512 * 4  # whole tiles
+    # the one-tile kernel's partials (splits x M x N) also start after the counter region
+    assert L.nvfp4_gemm_workspace_bytes_ex(41, 1536, 6144, 64, -12) == region + 12 * 41 * 1536 * 4
     # 128 tiles of 128 x 128 cover the SMs at 16 K tiles: no split
     assert L.nvfp4_gemm_workspace_bytes(968, 2048, 4096) == 0
     assert L.nvfp4_gemm_workspace_bytes(256, 256, 512) == 0  # 2 K tiles: a split does not pay

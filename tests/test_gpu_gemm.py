@@ -226,8 +226,28 @@ def test_persistent_split_k_deterministic_and_tickets_reset(orc):
     assert np.array_equal(o1, o2)
     need = nvfp4.lib().nvfp4_gemm_workspace_bytes(M, N, K)
     buf, _ = ws.get(need)
-    tickets = host(buf[:256].view(torch.int32))
+    tickets = host(buf[:16384].view(torch.int32))  # the whole counter region
     assert not tickets.any()
+
+
+def test_workspace_shared_across_shapes(orc):
+    """One workspace serves split-K GEMMs of different shapes in turn: the one-tile kernel's
+    partials (many splits, few tiles) never land where the many-row kernel (64 tiles) keeps
+    its counters, so the later GEMM still finds its counters zero."""
+    import torch
+    ws = nvfp4.Workspace(torch.device("cuda"))
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 38, 41, 1536, 6144)
+    A, W = to_gpu_fp4(ac, asf, ga, 41, 6144), to_gpu_fp4(wc, wsf, gw, 1536, 6144)
+    nvfp4.gemm(A, W, "none", workspace=ws, block_n=64, splits=-12)  # partials over 3 MB
+    M, N, K = 968, 2048, 16384
+    (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 39, M, N, K)
+    A, W = to_gpu_fp4(ac, asf, ga, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
+    rows = [0, 300, 967]
+    got = host(nvfp4.gemm(A, W, "none", workspace=ws))[rows]
+    torch.cuda.synchronize()
+    nvfp4.device_status()
+    ref = orc.gemm(ac, asf, ga, M, wc, wsf, gw, N, K, epi="none", rows=rows)
+    check_gemm_bf16(got, ref["v"], what="split-K after another shape's partials")
 
 
 def test_split_k_wait_expires_and_context_survives(orc):
@@ -240,7 +260,7 @@ def test_split_k_wait_expires_and_context_survives(orc):
     M, N, K = 256, 512, 8192
     L = nvfp4.lib()
     need = L.nvfp4_gemm_workspace_bytes(M, N, K)
-    assert need > 256  # 8 tiles: 256 bytes of counters, then the partials
+    assert need > 16384  # the 16 KiB counter region (8 tiles use 64 bytes of it), then the partials
     (ac, asf, ga), (wc, wsf, gw) = _operands(orc, 37, M, N, K)
     A, W = to_gpu_fp4(ac, asf, ga, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
     ws = nvfp4.Workspace(torch.device("cuda"))

@@ -53,7 +53,7 @@ def test_grouped_mixed_shapes_match_oracle(orc, with_bias):
         check_gemm_bf16(host(p[2]), ref, what=("grouped", g, shapes[g]))
 
 
-@pytest.mark.parametrize("epi", ["residual", "bias_gelu", "geglu"])
+@pytest.mark.parametrize("epi", ["residual", "bias_gelu", "geglu", "bias_gelu_rht", "geglu_rht"])
 def test_grouped_kernel_epilogues(orc, epi):
     """The grouped kernel's other epilogue kinds, including FP4 outputs, on problems of
     different M (one above 128 rows: two m-tiles) and K."""
@@ -64,13 +64,14 @@ def test_grouped_kernel_epilogues(orc, epi):
         x = synth.bf16_normal(synth.seed_of(90 + g, synth.CONTEXT), (M, K))
         w = synth.bf16_normal(synth.seed_of(90 + g, synth.W0), (N, K), 0.0, 0.02)
         ac, asf = orc.quantize_norm(x, "none")
-        wc, wsf, gw = orc.quantize_weight(w, interleave_gate_up=(epi == "geglu"))
-        bias = synth.bf16_normal(synth.seed_of(90 + g, synth.BIAS0), (N,), 0.0, 0.01) if epi == "bias_gelu" else None
+        wc, wsf, gw = orc.quantize_weight(w, interleave_gate_up=epi.startswith("geglu"))
+        bias = (synth.bf16_normal(synth.seed_of(90 + g, synth.BIAS0), (N,), 0.0, 0.01)
+                if epi.startswith("bias_gelu") else None)
         res = synth.bf16_normal(synth.seed_of(90 + g, synth.RESIDUAL), (M, N)) if epi == "residual" else None
         ref = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi=epi, bias=bias, residual=res)
         A, W = to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K)
-        if epi in ("bias_gelu", "geglu"):
-            out = nvfp4.empty_fp4(M, N // 2 if epi == "geglu" else N)
+        if "gelu" in epi or "geglu" in epi:
+            out = nvfp4.empty_fp4(M, N // 2 if epi.startswith("geglu") else N)
         else:
             out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         probs.append(nvfp4.op_gemm(A, W, epi, bias=dev_bf16(bias) if bias is not None else None,
@@ -81,7 +82,7 @@ def test_grouped_kernel_epilogues(orc, epi):
     prog.run()
     _sync()
     for ref, out, M, N, K in refs:
-        if epi in ("bias_gelu", "geglu"):
+        if "gelu" in epi or "geglu" in epi:
             check_fp4_output(orc, host(out.codes), host(out.sf), ref["codes"], ref["sf"], ref["h"], 1.0, M, out.K,
                              what=(M, N, K, epi))
         else:

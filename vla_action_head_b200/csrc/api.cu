@@ -221,17 +221,28 @@ Schedule choose_workspace(int M, int N, int K) {
     return choose(M, N, K, false);
 }
 
-// Tile counters (padded to 256 bytes) + the fp32 partials.  One-tile kernel: one ticket per
-// tile, splits x M x N partials.  Persistent kernel (`persistent`): an arrival ticket and a
-// published count per tile, splits x whole 128-row tiles x N partials.
-size_t ticket_bytes(size_t tiles, bool persistent) { return (tiles * (persistent ? 8 : 4) + 255) / 256 * 256; }
+// Workspace layout: a fixed region of tile counters, then the fp32 partials.  One-tile
+// kernel: one ticket per tile, splits x M x N partials.  Persistent kernel (`persistent`):
+// an arrival ticket and a published count per tile, splits x whole 128-row tiles x N
+// partials.  The counters of every schedule sit in the same fixed region, which no
+// schedule's partials overlap: a workspace reused across shapes keeps its counters zero
+// (every kernel returns the counters it used to zero), so no call finds another shape's
+// partial values where it expects counters.
+constexpr size_t kTicketRegion = 16384;
+size_t ticket_words_bytes(size_t tiles, bool persistent) { return tiles * (persistent ? 8 : 4); }
 
 size_t workspace_for(int M, int N, const Schedule &s, bool persistent = false) {
     if (s.splits <= 1 || s.cluster) return 0;
-    const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / s.block_n);
     const size_t rows = persistent ? static_cast<size_t>((M + 127) / 128) * 128 : static_cast<size_t>(M);
-    return ticket_bytes(tiles, persistent) + static_cast<size_t>(s.splits) * rows * N * sizeof(float);
+    return kTicketRegion + static_cast<size_t>(s.splits) * rows * N * sizeof(float);
 }
+
+// Kernel epilogue kind of an ABI epilogue, and whether its FP4 output blocks are rotated:
+// the *_RHT kinds are BIAS_GELU / GEGLU with each output block Hadamard-rotated first.
+int kernel_epi(nvfp4_epilogue e) {
+    return e == NVFP4_EPI_BIAS_GELU_RHT ? kEpiBiasGelu : e == NVFP4_EPI_GEGLU_RHT ? kEpiGeglu : static_cast<int>(e);
+}
+int epi_rotates(nvfp4_epilogue e) { return (e == NVFP4_EPI_BIAS_GELU_RHT || e == NVFP4_EPI_GEGLU_RHT) ? 1 : 0; }
 
 // Argument checks shared by nvfp4_gemm* and the GEMM op of a program (no device access).
 nvfp4_status validate_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,
@@ -240,12 +251,12 @@ nvfp4_status validate_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, 
     if (A == nullptr || W == nullptr) return NVFP4_ERR_INVALID_ARG;
     if (M < 0 || N <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
     if (A->rows != M || W->rows != N || A->K != K || W->K != K) return NVFP4_ERR_INVALID_ARG;
-    if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 5) return NVFP4_ERR_INVALID_ARG;
+    if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 7) return NVFP4_ERR_INVALID_ARG;
     if (K % 32 != 0 || N % 64 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!scale_ok(A->global_scale) || !scale_ok(W->global_scale)) return NVFP4_ERR_INVALID_ARG;
     if (M == 0) return NVFP4_OK;
-    const bool fp4_out = (epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
-    const bool need_bias = (epi == NVFP4_EPI_BIAS || epi == NVFP4_EPI_BIAS_RESIDUAL || epi == NVFP4_EPI_BIAS_GELU);
+    const bool fp4_out = (kernel_epi(epi) == kEpiBiasGelu || kernel_epi(epi) == kEpiGeglu);
+    const bool need_bias = (epi == NVFP4_EPI_BIAS || epi == NVFP4_EPI_BIAS_RESIDUAL || kernel_epi(epi) == kEpiBiasGelu);
     const bool need_res = (epi == NVFP4_EPI_RESIDUAL || epi == NVFP4_EPI_BIAS_RESIDUAL);
     if (need_bias && bias == nullptr) return NVFP4_ERR_INVALID_ARG;
     if (need_res && (residual == nullptr || ldr < N)) return NVFP4_ERR_INVALID_ARG;
@@ -282,7 +293,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
         persistent_bn = many.block_n;
         sc = finish(persistent_bn, many.splits, K, false);
     } else if (block_n == 0 && splits == 0) {
-        sc = choose(M, N, K, epi == NVFP4_EPI_BIAS_GELU || epi == NVFP4_EPI_GEGLU);
+        sc = choose(M, N, K, kernel_epi(epi) == kEpiBiasGelu || kernel_epi(epi) == kEpiGeglu);
     } else if (block_n == 0 && splits == -1) {
         sc = choose_workspace(M, N, K);
     } else {
@@ -294,6 +305,8 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     }
     const size_t need = workspace_for(M, N, sc, persistent_bn > 0);
     if (need > 0) {
+        const size_t tiles = static_cast<size_t>((M + 127) / 128) * (N / sc.block_n);
+        if (ticket_words_bytes(tiles, persistent_bn > 0) > kTicketRegion) return NVFP4_ERR_UNSUPPORTED_SHAPE;
         if (workspace == nullptr || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
         if (!aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
     }
@@ -316,7 +329,8 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     p.sfa = A->sf;
     p.sfb = W->sf;
     p.alpha = A->global_scale * W->global_scale;
-    p.epi = static_cast<int>(epi);
+    p.epi = kernel_epi(epi);
+    p.out_rotate = epi_rotates(epi);
     p.bias = static_cast<const uint16_t *>(bias);
     p.residual = static_cast<const uint16_t *>(residual);
     p.ldr = ldr;
@@ -328,7 +342,7 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     if (need > 0) {
         const size_t tiles = static_cast<size_t>((M + 127) / 128) * p.n_tiles;
         p.tickets = static_cast<uint32_t *>(workspace);
-        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + ticket_bytes(tiles, persistent_bn > 0));
+        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kTicketRegion);
     }
     const size_t ctas = static_cast<size_t>(p.n_tiles) * ((M + 127) / 128) * p.splits;
     if (g_trace != nullptr && g_trace_cursor + 8 * ctas <= g_trace_words) {
@@ -359,8 +373,10 @@ struct Residual {
 
 nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, nvfp4_norm kind, const void *gamma,
                        const void *beta, const void *mod_scale, const void *mod_shift, float eps, float g,
-                       uint8_t *codes, uint8_t *sf, float *y_out, cudaStream_t stream, const Residual &res = {}) {
+                       uint8_t *codes, uint8_t *sf, float *y_out, cudaStream_t stream, const Residual &res = {},
+                       int qflags = 0) {
     if (M < 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+    if ((qflags & ~(NVFP4_QUANT_ROTATE | NVFP4_QUANT_E0M3)) != 0) return NVFP4_ERR_INVALID_ARG;
     if (dt != NVFP4_IN_BF16 && dt != NVFP4_IN_FP32) return NVFP4_ERR_INVALID_ARG;
     if (static_cast<int>(kind) < 0 || static_cast<int>(kind) > 4) return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0 || K > (dt == NVFP4_IN_FP32 ? 16384 : 32768)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -404,6 +420,7 @@ nvfp4_status norm_impl(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, 
     a.codes = codes;
     a.sf = sf;
     a.y_out = y_out;
+    a.qflags = qflags;
     cudaError_t e = launch_norm_quant(a, dt == NVFP4_IN_FP32, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return from_cuda(e);
@@ -498,6 +515,30 @@ nvfp4_status nvfp4_quantize_norm(const void *x, nvfp4_in_dtype dt, int M, int K,
                      nullptr, stream);
 }
 
+nvfp4_status nvfp4_quantize_norm_ex(const void *x, nvfp4_in_dtype dt, int M, int K, int ldx, nvfp4_norm kind,
+                                    const void *gamma, const void *beta, const void *mod_scale, const void *mod_shift,
+                                    float eps, float global_scale, int flags, uint8_t *codes, uint8_t *sf,
+                                    nvfp4_stream_t stream) {
+    return norm_impl(x, dt, M, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, global_scale, codes, sf,
+                     nullptr, stream, Residual{}, flags);
+}
+
+nvfp4_status nvfp4_residual_quantize_norm_ex(const void *x, const void *d, const void *gate, int M, int K, int ldx,
+                                             int ldd, int ldh, nvfp4_norm kind, const void *gamma, const void *beta,
+                                             const void *mod_scale, const void *mod_shift, float eps,
+                                             float global_scale, int flags, void *h_out, uint8_t *codes, uint8_t *sf,
+                                             nvfp4_stream_t stream) {
+    if (M > 0 && d == nullptr) return NVFP4_ERR_INVALID_ARG;
+    Residual r;
+    r.d = d;
+    r.ldd = ldd;
+    r.gate = gate;
+    r.h = h_out;
+    r.ldh = ldh;
+    return norm_impl(x, NVFP4_IN_BF16, M, K, ldx, kind, gamma, beta, mod_scale, mod_shift, eps, global_scale, codes,
+                     sf, nullptr, stream, r, flags);
+}
+
 nvfp4_status nvfp4_residual_quantize_norm(const void *x, const void *d, const void *gate, int M, int K, int ldx,
                                           int ldd, int ldh, nvfp4_norm kind, const void *gamma, const void *beta,
                                           const void *mod_scale, const void *mod_shift, float eps, float global_scale,
@@ -523,7 +564,13 @@ nvfp4_status nvfp4_norm_f32(const void *x, nvfp4_in_dtype dt, int M, int K, int 
 
 static nvfp4_status quantize_weight_impl(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up,
                                          uint8_t *codes, uint8_t *sf, float *global_scale_out, void *scratch,
-                                         bool mse, cudaStream_t stream) {
+                                         int flags, cudaStream_t stream) {
+    if ((flags & ~(NVFP4_QUANT_ROTATE | NVFP4_QUANT_E0M3 | NVFP4_QUANT_MSE)) != 0) return NVFP4_ERR_INVALID_ARG;
+    // E0M3 weights take amax / 7 block scales; an MSE search is defined for E2M1 only
+    if ((flags & NVFP4_QUANT_E0M3) && (flags & NVFP4_QUANT_MSE)) return NVFP4_ERR_INVALID_ARG;
+    const bool mse = (flags & NVFP4_QUANT_MSE) != 0;
+    const int rotate = (flags & NVFP4_QUANT_ROTATE) ? 1 : 0;
+    const int qflags = flags & (NVFP4_QUANT_ROTATE | NVFP4_QUANT_E0M3);
     if (w_bf16 == nullptr || codes == nullptr || sf == nullptr || global_scale_out == nullptr || scratch == nullptr)
         return NVFP4_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0 || ldw < K) return NVFP4_ERR_INVALID_ARG;
@@ -534,11 +581,11 @@ static nvfp4_status quantize_weight_impl(const void *w_bf16, int N, int K, int l
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
     uint32_t *amax = static_cast<uint32_t *>(scratch);
-    cudaError_t e = launch_weight_amax(static_cast<const uint16_t *>(w_bf16), N, K, ldw, amax, stream);
+    cudaError_t e = launch_weight_amax(static_cast<const uint16_t *>(w_bf16), N, K, ldw, rotate, amax, stream);
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     if (mse) {
-        e = launch_weight_mse(static_cast<const uint16_t *>(w_bf16), N, K, ldw, interleave_gate_up ? 1 : 0, amax,
-                              codes, sf, stream);
+        e = launch_weight_mse(static_cast<const uint16_t *>(w_bf16), N, K, ldw, interleave_gate_up ? 1 : 0, rotate,
+                              amax, codes, sf, stream);
         if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     }
     NormArgs a = {};
@@ -553,6 +600,7 @@ static nvfp4_status quantize_weight_impl(const void *w_bf16, int N, int K, int l
     a.interleave = interleave_gate_up ? 1 : 0;
     a.codes = codes;
     a.sf = sf;
+    a.qflags = qflags;
     if (!mse) {
         e = launch_norm_quant(a, false, stream);
         if (e == cudaSuccess) e = cudaGetLastError();
@@ -564,21 +612,28 @@ static nvfp4_status quantize_weight_impl(const void *w_bf16, int N, int K, int l
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
     float am;
     std::memcpy(&am, &bits, sizeof am);
-    *global_scale_out = (am == 0.0f) ? 1.0f : am / 2688.0f;
+    *global_scale_out = (am == 0.0f) ? 1.0f : am / ((qflags & NVFP4_QUANT_E0M3) ? 3136.0f : 2688.0f);
     return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_quantize_weight(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up, uint8_t *codes,
                                    uint8_t *sf, float *global_scale_out, void *scratch, nvfp4_stream_t stream) {
-    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, false,
+    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, 0,
+                                stream);
+}
+
+nvfp4_status nvfp4_quantize_weight_ex(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up, int flags,
+                                      uint8_t *codes, uint8_t *sf, float *global_scale_out, void *scratch,
+                                      nvfp4_stream_t stream) {
+    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, flags,
                                 stream);
 }
 
 nvfp4_status nvfp4_quantize_weight_mse(const void *w_bf16, int N, int K, int ldw, int interleave_gate_up,
                                        uint8_t *codes, uint8_t *sf, float *global_scale_out, void *scratch,
                                        nvfp4_stream_t stream) {
-    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch, true,
-                                stream);
+    return quantize_weight_impl(w_bf16, N, K, ldw, interleave_gate_up, codes, sf, global_scale_out, scratch,
+                                NVFP4_QUANT_MSE, stream);
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int N, int K, nvfp4_epilogue epi,
@@ -783,7 +838,8 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             e.sfa = o.A.sf;
             e.sfb = o.W.sf;
             e.alpha = o.A.global_scale * o.W.global_scale;
-            e.epi = static_cast<int>(o.epi);
+            e.epi = kernel_epi(o.epi);
+            e.out_rotate = epi_rotates(o.epi);
             e.bias = static_cast<const uint16_t *>(o.bias);
             e.residual = static_cast<const uint16_t *>(o.residual);
             e.ldr = o.ldr;
@@ -871,7 +927,8 @@ static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t 
         p.sfa = o.A.sf;
         p.sfb = o.W.sf;
         p.alpha = o.A.global_scale * o.W.global_scale;
-        p.epi = static_cast<int>(o.epi);
+        p.epi = kernel_epi(o.epi);
+        p.out_rotate = epi_rotates(o.epi);
         p.bias = static_cast<const uint16_t *>(o.bias);
         p.residual = static_cast<const uint16_t *>(o.residual);
         p.ldr = o.ldr;
@@ -905,7 +962,7 @@ static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t 
     const int sms = sm_count_cached();
     prog->grid = total < sms ? total : sms;
     prog->kind = 1;
-    prog->epi = static_cast<int>(ops[0].epi);
+    prog->epi = kernel_epi(ops[0].epi);
     prog->tiles = total;
     prog->waits = 0;
     *st = NVFP4_OK;

@@ -36,6 +36,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Every field of p is read once into a local first: the byte stores of the FP4 outputs may
 // alias any memory as far as the compiler knows, and p may live in global memory.
 // EPI >= 0 fixes the epilogue kind at compile time (only that path is generated).
+// p.out_rotate: the FP4 epilogues rotate each 16-value output block by the 16-point
+// Hadamard matrix before quantizing it ("Pi0.5 Thor NVFP4 End-to-End Results", §Full-INT4
+// Decoder Activations + Hadamard Rotation: the GeGLU exit is one of the rotated exits).
 template <int W, int EPI = -1, class P>
 __device__ __forceinline__ void epilogue_chunk_w(const P &p, int m, int n, float *v, const uint32_t *bw,
                                                  const uint32_t *rw) {
@@ -46,6 +49,7 @@ __device__ __forceinline__ void epilogue_chunk_w(const P &p, int m, int n, float
     uint16_t *const out = p.out;
     uint8_t *const out_codes = p.out_codes;
     uint8_t *const out_sf = p.out_sf;
+    const bool rot = p.out_rotate != 0;
     const bool has_bias = bw != nullptr &&
                           (epi == kEpiBias || epi == kEpiBiasResidual || epi == kEpiBiasGelu || epi == kEpiGeglu);
     const bool has_res = rw != nullptr && (epi == kEpiResidual || epi == kEpiBiasResidual);
@@ -73,6 +77,7 @@ __device__ __forceinline__ void epilogue_chunk_w(const P &p, int m, int n, float
             float y[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) y[i] = gelu_tanh_f(v[16 * h + i]);
+            if (rot) fwht16(y);
             uint2 c;
             const uint32_t s = quantize_block16(y, g_out, d6g, c);
             const int col = n + 16 * h;
@@ -87,6 +92,7 @@ __device__ __forceinline__ void epilogue_chunk_w(const P &p, int m, int n, float
             float y[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) y[j] = __fmul_rn(gelu_tanh_f(v[2 * j]), v[2 * j + 1]);
+            if (rot) fwht16(y);
             uint2 c;
             const uint32_t s = quantize_block16(y, g_out, d6g, c);
             const int col = n >> 1;  // first output column of this block

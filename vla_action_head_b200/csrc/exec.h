@@ -41,6 +41,7 @@ struct ExecOp {
     int ldo;
     uint8_t *out_codes, *out_sf;
     float g_out;
+    int out_rotate;  // FP4 epilogues: Hadamard-rotate each output block before quantizing
 };
 
 struct ExecParams {

@@ -32,6 +32,7 @@ struct GemmArgs {
     uint8_t *out_codes;
     uint8_t *out_sf;
     float g_out;
+    int out_rotate;     // FP4 epilogues: Hadamard-rotate each output block before quantizing
     float *partials;    // split-K: [splits, M, N] fp32 (persistent kernel: [2, tiles, 128 x BN])
     uint32_t *tickets;  // split-K: one word per output tile (persistent kernel: two)
     unsigned long long *trace;  // optional per-CTA timestamps (diagnostics), 8 words per CTA

@@ -22,20 +22,42 @@ __global__ void __launch_bounds__(128) norm_quant_kernel(const NormArgs p) {
     norm_row<TPR, BPT, F32>(p, blockIdx.x * kRowsPerCta + threadIdx.x / TPR, threadIdx.x % TPR, red);
 }
 
-// Weight amax: max |w| over N x K bf16, folded into *amax_bits with an atomic max on the
-// fp32 bit pattern (monotonic for non-negative floats).
-__global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t *w, int N, int K, int ldw,
+// Weight amax: max |w| over N x K bf16 (rotate: over the Hadamard-rotated 16-element blocks
+// along K, the values the quantizer then encodes), folded into *amax_bits with an atomic max
+// on the fp32 bit pattern (monotonic for non-negative floats).
+__global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t *w, int N, int K, int ldw, int rotate,
                                                           uint32_t *amax_bits) {
-    const int kv = K >> 3;  // 16-byte vectors per row
-    const size_t total = static_cast<size_t>(N) * kv;
     float a = 0.0f;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const size_t r = i / kv, c = i % kv;
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + r * ldw) + c);
-        const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
+    if (!rotate) {
+        const int kv = K >> 3;  // 16-byte vectors per row
+        const size_t total = static_cast<size_t>(N) * kv;
+        for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+             i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+            const size_t r = i / kv, c = i % kv;
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(w + r * ldw) + c);
+            const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16lo(ws[j])), fabsf(bf16hi(ws[j]))));
+            for (int j = 0; j < 4; ++j) a = fmaxf(a, fmaxf(fabsf(bf16lo(ws[j])), fabsf(bf16hi(ws[j]))));
+        }
+    } else {
+        const int kb = K >> 4;  // 16-element blocks per row
+        const size_t total = static_cast<size_t>(N) * kb;
+        for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+             i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+            const size_t r = i / kb, c = i % kb;
+            const uint4 *q = reinterpret_cast<const uint4 *>(w + r * ldw + c * 16);
+            const uint4 u0 = __ldg(q), u1 = __ldg(q + 1);
+            const uint32_t ws[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            float y[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                y[2 * j] = bf16lo(ws[j]);
+                y[2 * j + 1] = bf16hi(ws[j]);
+            }
+            fwht16(y);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(y[j]));
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -54,7 +76,8 @@ __global__ void __launch_bounds__(256) weight_amax_kernel(const uint16_t *w, int
 // tried with the codes the amax quantizer writes at that scale (q_i = E2M1(y_i * rcp(dec(s)
 // g)), all +0 when dec(s) = 0); the block error E(s) = sum_i (y_i - val(q_i) dec(s) g)^2 is
 // formed in fp64 with one rounding per operation, terms in index order; the byte of least E
-// wins, the smaller byte on ties.  g = amax(|W|) / 2688, as for the amax scales.
+// wins, the smaller byte on ties.  g = amax(|W|) / 2688, as for the amax scales.  With
+// `rotate` the blocks are Hadamard-rotated first (and the amax is the rotated values').
 // E2M1 code -> value: magnitudes 0, 0.5, 1, 1.5 (m / 2), 2, 3, 4 (m - 2) and 6.
 __device__ __forceinline__ float e2m1_value(uint32_t q) {
     const uint32_t m = q & 7u;
@@ -87,7 +110,8 @@ __device__ __forceinline__ double block_sse(const float (&y)[16], float g, uint3
 
 // One warp per block; lane L tries bytes L, L + 32, L + 64, L + 96 (< 127).
 __global__ void __launch_bounds__(256) weight_mse_kernel(const uint16_t *w, int N, int K, int ldw, int interleave,
-                                                         const uint32_t *amax_bits, uint8_t *codes, uint8_t *sf) {
+                                                         int rotate, const uint32_t *amax_bits, uint8_t *codes,
+                                                         uint8_t *sf) {
     const int lane = threadIdx.x & 31;
     const int nblk = K >> 4;
     const long long blk = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -103,6 +127,7 @@ __global__ void __launch_bounds__(256) weight_mse_kernel(const uint16_t *w, int 
         y[2 * j] = bf16lo(ws[j]);
         y[2 * j + 1] = bf16hi(ws[j]);
     }
+    if (rotate) fwht16(y);
     const float amax = __uint_as_float(*amax_bits);
     const float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
     double best_e = 0.0;
@@ -179,12 +204,13 @@ cudaError_t launch_norm_quant(const NormArgs &a, bool f32_in, cudaStream_t s) {
     return f32_in ? launch_tpr<128, true>(a, bpt, s) : launch_tpr<128, false>(a, bpt, s);
 }
 
-cudaError_t launch_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave, const uint32_t *amax_bits,
-                              uint8_t *codes, uint8_t *sf, cudaStream_t s) {
+cudaError_t launch_weight_mse(const uint16_t *w, int N, int K, int ldw, int interleave, int rotate,
+                              const uint32_t *amax_bits, uint8_t *codes, uint8_t *sf, cudaStream_t s) {
     const long long blocks = static_cast<long long>(N) * (K >> 4);
     const long long ctas = (blocks + 7) / 8;
     if (ctas > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
-    weight_mse_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(w, N, K, ldw, interleave, amax_bits, codes, sf);
+    weight_mse_kernel<<<static_cast<unsigned>(ctas), 256, 0, s>>>(w, N, K, ldw, interleave, rotate, amax_bits, codes,
+                                                                   sf);
     return cudaGetLastError();
 }
 
@@ -193,7 +219,7 @@ cudaError_t probe_norm_kernels() {
     return cudaFuncGetAttributes(&fa, norm_quant_kernel<32, 1, false>);
 }
 
-cudaError_t launch_weight_amax(const uint16_t *w, int N, int K, int ldw, uint32_t *amax_bits,
+cudaError_t launch_weight_amax(const uint16_t *w, int N, int K, int ldw, int rotate, uint32_t *amax_bits,
                                cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
@@ -201,7 +227,7 @@ cudaError_t launch_weight_amax(const uint16_t *w, int N, int K, int ldw, uint32_
     size_t blocks = (vecs + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks == 0) blocks = 1;
-    weight_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, K, ldw, amax_bits);
+    weight_amax_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, N, K, ldw, rotate, amax_bits);
     return cudaGetLastError();
 }
 

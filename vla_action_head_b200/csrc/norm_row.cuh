@@ -78,6 +78,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
     const void *const x = p.x;
     const float eps = p.eps, g_arg = p.g;
     const uint32_t *const amax_bits = p.amax_bits;
+    const int qflags = p.qflags;
     uint8_t *const codes_out = p.codes;
     uint8_t *const sf_out = p.sf;
     float *const y_out = p.y_out;
@@ -230,11 +231,12 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
     if (!row_ok) return;
 
     float g = g_arg;
+    const float qmax = quant_qmax(qflags);
     if (amax_bits != nullptr) {
         const float amax = __uint_as_float(*amax_bits);
-        g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, __fmul_rn(qmax, 448.0f));
     }
-    const float d6g = __fmul_rn(6.0f, g);
+    const float dqg = __fmul_rn(qmax, g);
 
     // ---- normalize + quantize each block from registers ----
 #pragma unroll
@@ -289,7 +291,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
             continue;
         }
         uint2 c;
-        const uint32_t s = quantize_block16(y, g, d6g, c);
+        const uint32_t s = quantize_block16_opt(y, g, dqg, qflags, c);
         *reinterpret_cast<uint2 *>(codes_out + static_cast<size_t>(row) * (K >> 1) + b * 8) = c;
         sf_out[sf_offset(row, b, k_atoms)] = static_cast<uint8_t>(s);
     }

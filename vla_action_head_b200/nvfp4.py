@@ -19,7 +19,9 @@ LIB_PATH = os.environ.get("NVFP4_LIB") or os.path.join(HERE, "libnvfp4.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 NORM = {"none": 0, "layernorm": 1, "rmsnorm": 2, "adaln": 3, "adarms": 4}
-EPI = {"none": 0, "bias": 1, "residual": 2, "bias_residual": 3, "bias_gelu": 4, "geglu": 5}
+EPI = {"none": 0, "bias": 1, "residual": 2, "bias_residual": 3, "bias_gelu": 4, "geglu": 5,
+       "bias_gelu_rht": 6, "geglu_rht": 7}
+QUANT_ROTATE, QUANT_E0M3, QUANT_MSE = 1, 2, 4  # nvfp4_quant_flags
 IN_BF16, IN_FP32 = 0, 1
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "misaligned",
           4: "workspace", 5: "unsupported device", 6: "CUDA error", 7: "timeout"}
@@ -82,6 +84,10 @@ def lib():
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
             "nvfp4_quantize_weight": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
             "nvfp4_quantize_weight_mse": (I, [P, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
+            "nvfp4_quantize_weight_ex": (I, [P, I, I, I, I, I, P, P, C.POINTER(C.c_float), P, P]),
+            "nvfp4_quantize_norm_ex": (I, [P, I, I, I, I, I, P, P, P, P, F, F, I, P, P, P]),
+            "nvfp4_residual_quantize_norm_ex": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, I, P, P, P,
+                                                    P]),
             "nvfp4_gemm": (I, [C.POINTER(_Tensor), C.POINTER(_Tensor), I, I, I, I, P, P, I, P, I, P, P,
                                F, P, SZ, P]),
             "nvfp4_program_bytes": (SZ, [I]),
@@ -153,23 +159,35 @@ def empty_fp4(rows, K, device="cuda", global_scale=1.0):
     return NVFP4Tensor(codes, sf, global_scale, rows, K)
 
 
+def _qflags(rotate, fmt):
+    if fmt not in ("e2m1", "e0m3"):
+        raise ValueError(f"fmt must be 'e2m1' or 'e0m3', got {fmt!r}")
+    return (QUANT_ROTATE if rotate else 0) | (QUANT_E0M3 if fmt == "e0m3" else 0)
+
+
 def quantize_norm(x, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
-                  global_scale=1.0, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:
+                  global_scale=1.0, out: Optional[NVFP4Tensor] = None, rotate=False, fmt="e2m1") -> NVFP4Tensor:
+    """rotate: Hadamard-rotate each 16-element block before quantizing; fmt "e0m3": uniform
+    INT4 elements (a storage format; the GEMM reads E2M1)."""
     torch = _torch()
     M, K = x.shape
     dt = IN_FP32 if x.dtype == torch.float32 else IN_BF16
     if out is None:
         out = empty_fp4(M, K, x.device, global_scale)
-    st = lib().nvfp4_quantize_norm(_ptr(x), dt, M, K, x.stride(0), NORM[kind], _ptr(gamma), _ptr(beta),
-                                   _ptr(scale), _ptr(shift), eps, global_scale, _ptr(out.codes),
-                                   _ptr(out.sf), _stream())
+    flags = _qflags(rotate, fmt)
+    args = (_ptr(x), dt, M, K, x.stride(0), NORM[kind], _ptr(gamma), _ptr(beta), _ptr(scale), _ptr(shift), eps,
+            global_scale)
+    if flags:
+        st = lib().nvfp4_quantize_norm_ex(*args, flags, _ptr(out.codes), _ptr(out.sf), _stream())
+    else:
+        st = lib().nvfp4_quantize_norm(*args, _ptr(out.codes), _ptr(out.sf), _stream())
     _check("nvfp4_quantize_norm", st)
     out.global_scale = global_scale
     return out
 
 
 def residual_quantize_norm(x, d, gate, kind="adarms", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
-                           global_scale=1.0, h_out=None, out: Optional[NVFP4Tensor] = None):
+                           global_scale=1.0, h_out=None, out: Optional[NVFP4Tensor] = None, rotate=False, fmt="e2m1"):
     """h = bf16(x + gate * d) (gate None: 1), stored to h_out (may be x itself), then the norm
     `kind` -> NVFP4 of h.  Returns (h_out, NVFP4Tensor)."""
     torch = _torch()
@@ -178,10 +196,14 @@ def residual_quantize_norm(x, d, gate, kind="adarms", gamma=None, beta=None, sca
         h_out = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
     if out is None:
         out = empty_fp4(M, K, x.device, global_scale)
-    st = lib().nvfp4_residual_quantize_norm(_ptr(x), _ptr(d), _ptr(gate), M, K, x.stride(0), d.stride(0),
-                                            h_out.stride(0), NORM[kind], _ptr(gamma), _ptr(beta), _ptr(scale),
-                                            _ptr(shift), eps, global_scale, _ptr(h_out), _ptr(out.codes),
-                                            _ptr(out.sf), _stream())
+    flags = _qflags(rotate, fmt)
+    args = (_ptr(x), _ptr(d), _ptr(gate), M, K, x.stride(0), d.stride(0), h_out.stride(0), NORM[kind], _ptr(gamma),
+            _ptr(beta), _ptr(scale), _ptr(shift), eps, global_scale)
+    if flags:
+        st = lib().nvfp4_residual_quantize_norm_ex(*args, flags, _ptr(h_out), _ptr(out.codes), _ptr(out.sf),
+                                                   _stream())
+    else:
+        st = lib().nvfp4_residual_quantize_norm(*args, _ptr(h_out), _ptr(out.codes), _ptr(out.sf), _stream())
     _check("nvfp4_residual_quantize_norm", st)
     out.global_scale = global_scale
     return h_out, out
@@ -202,11 +224,12 @@ def norm_f32(x, kind, gamma=None, beta=None, scale=None, shift=None, eps=1e-6, o
 _scratch = {}
 
 
-def quantize_weight(w, interleave_gate_up=False, scales="amax") -> NVFP4Tensor:
+def quantize_weight(w, interleave_gate_up=False, scales="amax", rotate=False, fmt="e2m1") -> NVFP4Tensor:
     """bf16 W [N, K] -> NVFP4; scales "amax" (block amax / 6) or "mse" (the scale byte of
-    least block squared error)."""
+    least block squared error); rotate: Hadamard-rotated blocks; fmt "e0m3": uniform INT4."""
     if scales not in ("amax", "mse"):
         raise ValueError(f"scales must be 'amax' or 'mse', got {scales!r}")
+    flags = _qflags(rotate, fmt) | (QUANT_MSE if scales == "mse" else 0)
     torch = _torch()
     N, K = w.shape
     out = empty_fp4(N, K, w.device)
@@ -214,9 +237,15 @@ def quantize_weight(w, interleave_gate_up=False, scales="amax") -> NVFP4Tensor:
     if dev not in _scratch:
         _scratch[dev] = torch.zeros(256, dtype=torch.uint8, device=w.device)
     g = C.c_float(0.0)
-    name = "nvfp4_quantize_weight" if scales == "amax" else "nvfp4_quantize_weight_mse"
-    st = getattr(lib(), name)(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)), _ptr(out.codes),
-                              _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]), _stream())
+    if flags & (QUANT_ROTATE | QUANT_E0M3):
+        name = "nvfp4_quantize_weight_ex"
+        st = lib().nvfp4_quantize_weight_ex(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)), flags,
+                                            _ptr(out.codes), _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]),
+                                            _stream())
+    else:
+        name = "nvfp4_quantize_weight" if scales == "amax" else "nvfp4_quantize_weight_mse"
+        st = getattr(lib(), name)(_ptr(w), N, K, w.stride(0), int(bool(interleave_gate_up)), _ptr(out.codes),
+                                  _ptr(out.sf), C.byref(g), _ptr(_scratch[dev]), _stream())
     _check(name, st)
     out.global_scale = g.value
     return out
@@ -251,10 +280,10 @@ def gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, o
     torch = _torch()
     M, N, K = a.rows, w.rows, a.K
     e = EPI[epi]
-    fp4 = e in (4, 5)
+    fp4 = e in (4, 5, 6, 7)
     if out is None:
         if fp4:
-            out = empty_fp4(M, N // 2 if e == 5 else N, a.codes.device, out_global_scale)
+            out = empty_fp4(M, N // 2 if e in (5, 7) else N, a.codes.device, out_global_scale)
         else:
             out = torch.empty((M, N), dtype=torch.bfloat16, device=a.codes.device)
     if workspace is None:
@@ -317,7 +346,7 @@ def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None
     e = EPI[epi]
     op = _Op(type=1, M=a.rows, N=w.rows, K=a.K, A=a.c(), W=w.c(), epi=e, bias=_ptr(bias),
              residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0, dep=_dep(dep))
-    if e in (4, 5):
+    if e in (4, 5, 6, 7):
         op.out_codes, op.out_sf, op.out_global_scale = out.codes.data_ptr(), out.sf.data_ptr(), out_global_scale
     else:
         op.out_bf16, op.ldo, op.out_global_scale = out.data_ptr(), out.stride(0), 1.0
