@@ -189,14 +189,24 @@ def gemm_bytes(M, N, K, epi):
     return b
 
 
-def time_graph(g, reps, stream):
-    """ms per replay; replays and events on `stream`."""
+SOAK_S = 0.3  # untimed replays before a side measurement, so its clock sampler sees the load
+
+
+def time_graph(g, reps, stream, soak_s=None):
+    """ms per replay; replays and events on `stream`.  Before the timed replays the graph
+    replays untimed for about soak_s seconds (SOAK_S by default)."""
     import torch
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    soak_s = SOAK_S if soak_s is None else soak_s
     with torch.cuda.stream(stream):
         for _ in range(2):
             g.replay()
         torch.cuda.synchronize()
+        t_end = time.perf_counter() + soak_s
+        while time.perf_counter() < t_end:
+            for _ in range(8):
+                g.replay()
+            torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(reps):
             g.replay()
@@ -691,12 +701,36 @@ def main():
     return 0
 
 
+class ClockRecord:
+    """Samples the GPU clocks over one side measurement and stores them in entry["clocks"]."""
+
+    def __init__(self, gpu_index, entry_of):
+        self.gpu, self.entry_of = gpu_index, entry_of
+
+    def __enter__(self):
+        self.clk = Clocks(self.gpu)
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        rec = self.clk.stop()
+        if exc[0] is None:
+            self.entry_of()["clocks"] = rec
+        return False
+
+
 def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     import torch
 
     from vla_action_head_b200 import layers, nvfp4, synth
     M, H, F = DIT["M"], DIT["H"], DIT["F"]
     out = {}
+    gpu = dev.index if dev.index is not None else 0
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+
+    def clocked(key):
+        return ClockRecord(gpu, lambda: out[key])
+
     # ---- roofline of the GEMM kernel in the DiT layer (HBM-bound at M = 41) ----
     l0 = stack[0]
     per = {}
@@ -704,24 +738,25 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
     specs = [("qkv", l0.a1, "qkv", "bias", 3 * H, H), ("attn_out", l0.ctx_q, "o", "bias_residual", H, H),
              ("ffn_up", l0.a2, "up", "bias_gelu", F, H), ("ffn_down", l0.u, "down", "bias_residual", H, F)]
     res = torch.zeros((M, H), dtype=torch.bfloat16, device=dev)
-    with torch.cuda.stream(stream):
-        for name, A, attr, epi, N, K in specs:
-            lins = [getattr(s, attr) for s in stack]
-            if epi == "bias_gelu":
-                outs = [nvfp4.empty_fp4(M, N, dev) for _ in range(2)]
-            else:
-                outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-            ms = gemm_ring_time(A, lins, epi, outs, wsp, stream, res=res if "residual" in epi else None)
-            b = gemm_bytes(M, N, K, epi)
-            per[name] = {"us": round(ms * 1e3, 3), "gbs": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}
-            tot_b += b
-            tot_ms += ms
-    ach = tot_b / (tot_ms * 1e-3) / 1e9
-    out["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                       "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic("dit_gemm"),
-                       "algorithmic_bytes_per_launch": tot_b // len(specs),
-                       "kernel": "gemm_kernel (4 DiT GEMMs, M=41, L2-cold weights)", "peak_kind": pk_kind,
-                       "per_gemm": per}
+    with clocked("roofline"):
+        with torch.cuda.stream(stream):
+            for name, A, attr, epi, N, K in specs:
+                lins = [getattr(s, attr) for s in stack]
+                if epi == "bias_gelu":
+                    outs = [nvfp4.empty_fp4(M, N, dev) for _ in range(2)]
+                else:
+                    outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+                ms = gemm_ring_time(A, lins, epi, outs, wsp, stream, res=res if "residual" in epi else None)
+                b = gemm_bytes(M, N, K, epi)
+                per[name] = {"us": round(ms * 1e3, 3), "gbs": round(b / (ms * 1e-3) / 1e9, 1), "bytes": b}
+                tot_b += b
+                tot_ms += ms
+        ach = tot_b / (tot_ms * 1e-3) / 1e9
+        out["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                           "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic("dit_gemm"),
+                           "algorithmic_bytes_per_launch": tot_b // len(specs),
+                           "kernel": "gemm_kernel (4 DiT GEMMs, M=41, L2-cold weights)", "peak_kind": pk_kind,
+                           "per_gemm": per}
     # ---- grouped GEMM: 32 cross-attention K/V projections of one M = 41 context in one
     # launch; a ring of 4 groups with distinct weights (4 x 42.5 MB > L2) ----
     with torch.cuda.stream(stream):
@@ -747,18 +782,19 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
         grouped()
         chained()
     torch.cuda.synchronize()
-    g = capture(grouped, stream)
-    ms_g = time_graph(g, 20, stream) / len(groups)
-    del g
-    g = capture(chained, stream)
-    ms_c = time_graph(g, 20, stream) / len(groups)
-    del g
-    b_grp = G * gemm_bytes(M, Nc, Kc, "none")
-    out["grouped_cross_kv32"] = {"problems": f"{G} x {M}x{Nc}x{Kc}, shared context", "us": round(ms_g * 1e3, 2),
-                                 "gbs": round(b_grp / (ms_g * 1e-3) / 1e9, 1),
-                                 "frac_hbm": round(b_grp / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                                 "us_as_32_launches": round(ms_c * 1e3, 2), "bytes": b_grp,
-                                 "l2": "ring of 4 groups with distinct weights (170 MB > L2)"}
+    with clocked("grouped_cross_kv32"):
+        g = capture(grouped, stream)
+        ms_g = time_graph(g, 20, stream) / len(groups)
+        del g
+        g = capture(chained, stream)
+        ms_c = time_graph(g, 20, stream) / len(groups)
+        del g
+        b_grp = G * gemm_bytes(M, Nc, Kc, "none")
+        out["grouped_cross_kv32"] = {"problems": f"{G} x {M}x{Nc}x{Kc}, shared context",
+                                     "us": round(ms_g * 1e3, 2), "gbs": round(b_grp / (ms_g * 1e-3) / 1e9, 1),
+                                     "frac_hbm": round(b_grp / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                                     "us_as_32_launches": round(ms_c * 1e3, 2), "bytes": b_grp,
+                                     "l2": "ring of 4 groups with distinct weights (170 MB > L2)"}
     del groups, kv_lins, kv_outs, ctxq
     # ---- 18-layer action-expert stack (config 3 layers, one CUDA graph) ----
     with torch.cuda.stream(stream):
@@ -772,29 +808,30 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                 lay.forward(ab[i % 2], ca, ab[(i + 1) % 2])
         ae_fwd()
     torch.cuda.synchronize()
-    g = capture(ae_fwd, stream)
-    ms = time_graph(g, 50, stream)
-    del g
-    ae_w = sum(l.weight_bytes() for l in ae[0].linears())
-    out["action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
-                                    "weight_stream_gbs": round(18 * ae_w / (ms * 1e-3) / 1e9, 1)}
-    # its four GEMMs alone, each over the 18 layers' weights (L2-cold)
-    a0 = ae[0]
-    ae_per = {}
-    res50 = torch.zeros((50, 1024), dtype=torch.bfloat16, device=dev)
-    with torch.cuda.stream(stream):
-        for name, A, attr, epi, N, K in [("qkv", a0.a1, "qkv", "none", 2560, 1024),
-                                         ("o", a0.ctx_q, "o", "residual", 1024, 2048),
-                                         ("gate_up", a0.a2, "gate_up", "geglu", 8192, 1024),
-                                         ("down", a0.u, "down", "residual", 1024, 4096)]:
-            outs = ([nvfp4.empty_fp4(50, N // 2, dev) for _ in range(2)] if epi == "geglu" else
-                    [torch.empty((50, N), dtype=torch.bfloat16, device=dev) for _ in range(2)])
-            ms_g = gemm_ring_time(A, [getattr(l, attr) for l in ae], epi, outs, wsp, stream,
-                                  res=res50 if epi == "residual" else None)
-            b = gemm_bytes(50, N, K, epi)
-            ae_per[name] = {"us": round(ms_g * 1e3, 3), "gbs": round(b / (ms_g * 1e-3) / 1e9, 1), "bytes": b,
-                            "frac_hbm": round(b / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-    out["action_expert_stack18"]["per_gemm"] = ae_per
+    with clocked("action_expert_stack18"):
+        g = capture(ae_fwd, stream)
+        ms = time_graph(g, 50, stream)
+        del g
+        ae_w = sum(l.weight_bytes() for l in ae[0].linears())
+        # its four GEMMs alone, each over the 18 layers' weights (L2-cold)
+        a0 = ae[0]
+        ae_per = {}
+        res50 = torch.zeros((50, 1024), dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            for name, A, attr, epi, N, K in [("qkv", a0.a1, "qkv", "none", 2560, 1024),
+                                             ("o", a0.ctx_q, "o", "residual", 1024, 2048),
+                                             ("gate_up", a0.a2, "gate_up", "geglu", 8192, 1024),
+                                             ("down", a0.u, "down", "residual", 1024, 4096)]:
+                outs = ([nvfp4.empty_fp4(50, N // 2, dev) for _ in range(2)] if epi == "geglu" else
+                        [torch.empty((50, N), dtype=torch.bfloat16, device=dev) for _ in range(2)])
+                ms_g = gemm_ring_time(A, [getattr(l, attr) for l in ae], epi, outs, wsp, stream,
+                                      res=res50 if epi == "residual" else None)
+                b = gemm_bytes(50, N, K, epi)
+                ae_per[name] = {"us": round(ms_g * 1e3, 3), "gbs": round(b / (ms_g * 1e-3) / 1e9, 1), "bytes": b,
+                                "frac_hbm": round(b / (ms_g * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        out["action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
+                                        "weight_stream_gbs": round(18 * ae_w / (ms * 1e-3) / 1e9, 1),
+                                        "per_gemm": ae_per}
     del ae, xa, ab
     # ---- the same stack with the gated residual updates fused into the norm front-ends ----
     with torch.cuda.stream(stream):
@@ -809,54 +846,63 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                 d, gate = lay.forward(rg, d, gate, ca)
         gae_fwd()
     torch.cuda.synchronize()
-    g = capture(gae_fwd, stream)
-    ms = time_graph(g, 50, stream)
-    del g
-    gae_w = sum(l.weight_bytes() for l in gae[0].linears())
-    out["gated_action_expert_stack18"] = {"us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
-                                          "weight_stream_gbs": round(18 * gae_w / (ms * 1e-3) / 1e9, 1),
-                                          "front_end": "gated residual + AdaRMSNorm -> NVFP4 in one launch"}
+    with clocked("gated_action_expert_stack18"):
+        g = capture(gae_fwd, stream)
+        ms = time_graph(g, 50, stream)
+        del g
+        gae_w = sum(l.weight_bytes() for l in gae[0].linears())
+        out["gated_action_expert_stack18"] = {
+            "us_per_stack": round(ms * 1e3, 2), "us_per_layer": round(ms * 1e3 / 18, 3),
+            "weight_stream_gbs": round(18 * gae_w / (ms * 1e-3) / 1e9, 1),
+            "front_end": "gated residual + AdaRMSNorm -> NVFP4 in one launch"}
     del gae, r0, rg, ca
-    # ---- prefill layer at M = 968 (tensor-bound): ring of 4 distinct layers ----
+    # ---- prefill layers at M = 968 (tensor-bound): the 18-layer stack in one CUDA graph
+    # (1.07 GB of distinct weights), and each GEMM over the 18 layers' weights ----
     with torch.cuda.stream(stream):
-        pre = [layers.PrefillLayer(layer=i, device=dev, ws=wsp) for i in range(4)]
+        pre = [layers.PrefillLayer(layer=i, device=dev, ws=wsp) for i in range(18)]
         xp = synth.bf16_normal_torch(synth.seed_of(4, synth.X), (968, 2048), device=dev)
-        yp = torch.empty_like(xp)
+        pb = [xp.clone(), torch.empty_like(xp)]
 
         def pre_fwd():
-            for lay in pre:
-                lay.forward(xp, xp, yp)
+            for i, lay in enumerate(pre):
+                lay.forward(pb[i % 2], pb[i % 2], pb[(i + 1) % 2])
         pre_fwd()
     torch.cuda.synchronize()
-    g = capture(pre_fwd, stream)
-    ms = time_graph(g, 10, stream) / len(pre)
-    del g
-    fl = pre[0].flops()
-    tf = fl / (ms * 1e-3) / 1e12
-    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
-    # the gate_up GEMM alone (dominant kernel of the layer)
-    with torch.cuda.stream(stream):
-        outs = [nvfp4.empty_fp4(968, 16384, dev) for _ in range(2)]
-        ms_gu = gemm_ring_time(pre[0].a2, [p.gate_up for p in pre], "geglu", outs, wsp, stream, reps=10)
-        outs_q = [torch.empty((968, 2560), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        ms_q = gemm_ring_time(pre[0].a1, [p.qkv for p in pre], "none", outs_q, wsp, stream, reps=10)
-        # down: 64 tiles of 128 x 256 with K = 16384 split in two through the workspace
-        outs_d = [torch.empty((968, 2048), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        ms_dn = gemm_ring_time(pre[0].u, [p.down for p in pre], "residual", outs_d, wsp, stream, reps=10, res=xp)
-    tf_gu = 2.0 * 968 * 32768 * 2048 / (ms_gu * 1e-3) / 1e12
-    out["prefill_m968"] = {"us_per_layer": round(ms * 1e3, 2), "tflops": round(tf, 1),
-                           "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1),
-                           "qkv_us": round(ms_q * 1e3, 2),
-                           "qkv_tflops": round(2.0 * 968 * 2560 * 2048 / (ms_q * 1e-3) / 1e12, 1),
-                           "down_us": round(ms_dn * 1e3, 2),
-                           "down_tflops": round(2.0 * 968 * 2048 * 16384 / (ms_dn * 1e-3) / 1e12, 1)}
+    with clocked("prefill_stack18_m968"):
+        g = capture(pre_fwd, stream)
+        ms = time_graph(g, 10, stream)
+        del g
+        fl = pre[0].flops()
+        out["prefill_stack18_m968"] = {"us_per_stack": round(ms * 1e3, 1), "us_per_layer": round(ms * 1e3 / 18, 2),
+                                       "tflops": round(18 * fl / (ms * 1e-3) / 1e12, 1),
+                                       "frac_fp4_peak": round(18 * fl / (ms * 1e-3) / 1e12 / fp4_peak, 4),
+                                       "graph": "18 distinct layers, one CUDA graph"}
+    with clocked("prefill_m968"):
+        with torch.cuda.stream(stream):
+            outs = [nvfp4.empty_fp4(968, 16384, dev) for _ in range(2)]
+            ms_gu = gemm_ring_time(pre[0].a2, [p.gate_up for p in pre], "geglu", outs, wsp, stream, reps=10)
+            outs_q = [torch.empty((968, 2560), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            ms_q = gemm_ring_time(pre[0].a1, [p.qkv for p in pre], "none", outs_q, wsp, stream, reps=10)
+            # down: 64 tiles of 128 x 256 with K = 16384 split in two through the workspace
+            outs_d = [torch.empty((968, 2048), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            ms_dn = gemm_ring_time(pre[0].u, [p.down for p in pre], "residual", outs_d, wsp, stream, reps=10,
+                                   res=xp)
+        tf_gu = 2.0 * 968 * 32768 * 2048 / (ms_gu * 1e-3) / 1e12
+        out["prefill_m968"] = {"us_per_layer": out["prefill_stack18_m968"]["us_per_layer"],
+                               "tflops": out["prefill_stack18_m968"]["tflops"],
+                               "gate_up_us": round(ms_gu * 1e3, 2), "gate_up_tflops": round(tf_gu, 1),
+                               "qkv_us": round(ms_q * 1e3, 2),
+                               "qkv_tflops": round(2.0 * 968 * 2560 * 2048 / (ms_q * 1e-3) / 1e12, 1),
+                               "down_us": round(ms_dn * 1e3, 2),
+                               "down_tflops": round(2.0 * 968 * 2048 * 16384 / (ms_dn * 1e-3) / 1e12, 1)}
     out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_peak, 1),
                             "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4),
                             "traffic": traffic("prefill_gate_up"),
                             "algorithmic_bytes_per_launch": gemm_bytes(968, 32768, 2048, "geglu"),
                             "kernel": "gemm_persistent_kernel gate_up 968x32768x2048 GeGLU->FP4",
-                            "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)"}
-    del pre, xp, yp, outs, outs_q, outs_d
+                            "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)",
+                            "clocks": out["prefill_m968"]["clocks"]}
+    del pre, xp, pb, outs, outs_q, outs_d
     # ---- M sweep on the 1536 -> 6144 GEMM (bias, bf16 out), 48 distinct weights ----
     with torch.cuda.stream(stream):
         lins = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(5, 1000 + i), (6144, 1536), 0, 0.02,
@@ -864,48 +910,51 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                               synth.bf16_normal_torch(synth.seed_of(5, 2000 + i), (6144,), 0, 0.01, device=dev))
                 for i in range(48)]
     sweep = []
-    for Ms in (1, 16, 41, 128, 512, 968):
-        with torch.cuda.stream(stream):
-            xs = synth.bf16_normal_torch(synth.seed_of(5, Ms), (Ms, 1536), device=dev)
-            A = nvfp4.quantize_norm(xs, "none")
-            outs = [torch.empty((Ms, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-            ms = gemm_ring_time(A, lins, "bias", outs, wsp, stream, reps=10)
-        b = gemm_bytes(Ms, 6144, 1536, "bias")
-        gbs = b / (ms * 1e-3) / 1e9
-        tf = 2.0 * Ms * 6144 * 1536 / (ms * 1e-3) / 1e12
-        # the bound by arithmetic intensity against the ridge of the two measured peaks
-        hbm_bound = (2.0 * Ms * 6144 * 1536 / b) < fp4_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
-        sweep.append({"M": Ms, "us": round(ms * 1e3, 3), "gbs": round(gbs, 1), "tflops": round(tf, 2),
-                      "bound": "hbm" if hbm_bound else "tensor",
-                      "frac": round(gbs / pk["hbm_gbs"] if hbm_bound else tf / fp4_peak, 4)})
-    out["m_sweep_1536x6144"] = sweep
+    with clocked("m_sweep_1536x6144"):
+        for Ms in (1, 16, 41, 128, 512, 968):
+            with torch.cuda.stream(stream):
+                xs = synth.bf16_normal_torch(synth.seed_of(5, Ms), (Ms, 1536), device=dev)
+                A = nvfp4.quantize_norm(xs, "none")
+                outs = [torch.empty((Ms, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+                ms = gemm_ring_time(A, lins, "bias", outs, wsp, stream, reps=10)
+            b = gemm_bytes(Ms, 6144, 1536, "bias")
+            gbs = b / (ms * 1e-3) / 1e9
+            tf = 2.0 * Ms * 6144 * 1536 / (ms * 1e-3) / 1e12
+            # the bound by arithmetic intensity against the ridge of the two measured peaks
+            hbm_bound = (2.0 * Ms * 6144 * 1536 / b) < fp4_peak * 1e12 / (pk["hbm_gbs"] * 1e9)
+            sweep.append({"M": Ms, "us": round(ms * 1e3, 3), "gbs": round(gbs, 1), "tflops": round(tf, 2),
+                          "bound": "hbm" if hbm_bound else "tensor",
+                          "frac": round(gbs / pk["hbm_gbs"] if hbm_bound else tf / fp4_peak, 4)})
+        out["m_sweep_1536x6144"] = {"points": sweep}
     # ---- norm -> NVFP4 alone at the configs' shapes, over 48 distinct inputs per replay ----
     norm_res = {}
-    for label, Mn, Kn, kind in [("adaln_41x1536", 41, 1536, "adaln"), ("layernorm_41x1536", 41, 1536, "layernorm"),
-                                ("adarms_50x1024", 50, 1024, "adarms"), ("rmsnorm_968x2048", 968, 2048, "rmsnorm")]:
-        with torch.cuda.stream(stream):
-            xs = [synth.bf16_normal_torch(synth.seed_of(8, 500 + i), (Mn, Kn), device=dev) for i in range(48)]
-            gam = synth.bf16_normal_torch(synth.seed_of(8, synth.GAMMA), (Kn,), 1.0, 0.1, device=dev)
-            bet = synth.bf16_normal_torch(synth.seed_of(8, synth.BETA), (Kn,), 0.0, 0.1, device=dev)
-            sc = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SCALE), (Kn,), 0.0, 0.1, device=dev)
-            sh = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SHIFT), (Kn,), 0.0, 0.1, device=dev)
-            prm = {"layernorm": dict(gamma=gam, beta=bet, eps=1e-5), "rmsnorm": dict(gamma=gam, eps=1e-6),
-                   "adaln": dict(scale=sc, shift=sh, eps=1e-6), "adarms": dict(scale=sc, eps=1e-6)}[kind]
-            qo = nvfp4.empty_fp4(Mn, Kn, dev)
-
-            def norms(xs=xs, kind=kind, prm=prm, qo=qo):
-                for xi in xs:
-                    nvfp4.quantize_norm(xi, kind, out=qo, **prm)
-            norms()
-        torch.cuda.synchronize()
-        g = capture(norms, stream)
-        ms_n = time_graph(g, 10, stream) / len(xs)
-        del g
-        nb = 2 * Mn * Kn + Mn * Kn // 2 + Mn * Kn // 16 + 2 * Kn * (2 if kind in ("layernorm", "adaln") else 1)
-        norm_res[label] = {"us": round(ms_n * 1e3, 3), "gbs": round(nb / (ms_n * 1e-3) / 1e9, 1), "bytes": nb,
-                           "frac_hbm": round(nb / (ms_n * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
-        del xs
     out["norm_quant"] = norm_res
+    with clocked("norm_quant"):
+        for label, Mn, Kn, kind in [("adaln_41x1536", 41, 1536, "adaln"),
+                                    ("layernorm_41x1536", 41, 1536, "layernorm"),
+                                    ("adarms_50x1024", 50, 1024, "adarms"), ("rmsnorm_968x2048", 968, 2048, "rmsnorm")]:
+            with torch.cuda.stream(stream):
+                xs = [synth.bf16_normal_torch(synth.seed_of(8, 500 + i), (Mn, Kn), device=dev) for i in range(48)]
+                gam = synth.bf16_normal_torch(synth.seed_of(8, synth.GAMMA), (Kn,), 1.0, 0.1, device=dev)
+                bet = synth.bf16_normal_torch(synth.seed_of(8, synth.BETA), (Kn,), 0.0, 0.1, device=dev)
+                sc = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SCALE), (Kn,), 0.0, 0.1, device=dev)
+                sh = synth.bf16_normal_torch(synth.seed_of(8, synth.MOD_SHIFT), (Kn,), 0.0, 0.1, device=dev)
+                prm = {"layernorm": dict(gamma=gam, beta=bet, eps=1e-5), "rmsnorm": dict(gamma=gam, eps=1e-6),
+                       "adaln": dict(scale=sc, shift=sh, eps=1e-6), "adarms": dict(scale=sc, eps=1e-6)}[kind]
+                qo = nvfp4.empty_fp4(Mn, Kn, dev)
+
+                def norms(xs=xs, kind=kind, prm=prm, qo=qo):
+                    for xi in xs:
+                        nvfp4.quantize_norm(xi, kind, out=qo, **prm)
+                norms()
+            torch.cuda.synchronize()
+            g = capture(norms, stream)
+            ms_n = time_graph(g, 10, stream) / len(xs)
+            del g
+            nb = 2 * Mn * Kn + Mn * Kn // 2 + Mn * Kn // 16 + 2 * Kn * (2 if kind in ("layernorm", "adaln") else 1)
+            norm_res[label] = {"us": round(ms_n * 1e3, 3), "gbs": round(nb / (ms_n * 1e-3) / 1e9, 1), "bytes": nb,
+                               "frac_hbm": round(nb / (ms_n * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+            del xs
     # ---- tiny config: LayerNorm->NVFP4 of 41 x 256, then 41 x 512 x 256 GEMM + bias ----
     with torch.cuda.stream(stream):
         tl = [layers.Linear(synth.bf16_normal_torch(synth.seed_of(1, synth.W0 + 100 * i), (512, 256), 0, 0.02,
@@ -924,12 +973,19 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                 nvfp4.gemm(at, lin.w, "bias", bias=lin.bias, out=ot, workspace=wsp)
         tiny()
     torch.cuda.synchronize()
-    g = capture(tiny, stream)
-    ms = time_graph(g, 20, stream) / len(tl)
-    del g
-    out["tiny_41x256_512"] = {"us_per_norm_plus_gemm": round(ms * 1e3, 3),
-                              "gemm_bytes": gemm_bytes(41, 512, 256, "bias"),
-                              "l2": "48 distinct weight copies (L2-warm: 3.6 MB in total)"}
+    with clocked("tiny_41x256_512"):
+        g = capture(tiny, stream)
+        ms = time_graph(g, 20, stream) / len(tl)
+        del g
+        # algorithmic bytes of the pair: the norm's x, gamma, beta and FP4 output + the GEMM's
+        tb = (2 * 41 * 256 + 4 * 256 + 41 * 128 + 41 * 16) + gemm_bytes(41, 512, 256, "bias")
+        gbs_t = tb / (ms * 1e-3) / 1e9
+        out["tiny_41x256_512"] = {"us_per_norm_plus_gemm": round(ms * 1e3, 3),
+                                  "gemm_bytes": gemm_bytes(41, 512, 256, "bias"),
+                                  "roofline": {"bound": "hbm", "achieved": round(gbs_t, 1), "peak": pk["hbm_gbs"],
+                                               "unit": "GB/s", "frac": round(gbs_t / pk["hbm_gbs"], 4),
+                                               "bytes": tb, "peak_kind": pk_kind},
+                                  "l2": "48 distinct weight copies (L2-warm: 3.6 MB in total)"}
     torch.cuda.synchronize()
     nvfp4.device_status()
     return out
