@@ -895,12 +895,17 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                                "qkv_tflops": round(2.0 * 968 * 2560 * 2048 / (ms_q * 1e-3) / 1e12, 1),
                                "down_us": round(ms_dn * 1e3, 2),
                                "down_tflops": round(2.0 * 968 * 2048 * 16384 / (ms_dn * 1e-3) / 1e12, 1)}
-    out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_peak, 1),
-                            "unit": "TFLOP/s", "frac": round(tf_gu / fp4_peak, 4),
+    # the gate/up GEMM runs as 18 back-to-back launches after a soak, i.e. inside a long step:
+    # the sustained peak is the denominator; the burst one is shown beside it
+    fp4_sus = pk["bf16_tflops_sustained"] * FP4_OVER_BF16
+    out["roofline_m968"] = {"bound": "tensor", "achieved": round(tf_gu, 1), "peak": round(fp4_sus, 1),
+                            "unit": "TFLOP/s", "frac": round(tf_gu / fp4_sus, 4),
                             "traffic": traffic("prefill_gate_up"),
                             "algorithmic_bytes_per_launch": gemm_bytes(968, 32768, 2048, "geglu"),
                             "kernel": "gemm_persistent_kernel gate_up 968x32768x2048 GeGLU->FP4",
-                            "peak_kind": f"{pk_kind} bf16 burst x {FP4_OVER_BF16} (nominal fp4/bf16 dense ratio)",
+                            "peak_kind": f"{pk_kind} bf16 sustained x {FP4_OVER_BF16} (nominal fp4/bf16 dense "
+                                         "ratio); timed as 18 launches back to back after a soak",
+                            "peak_burst": round(fp4_peak, 1), "frac_burst": round(tf_gu / fp4_peak, 4),
                             "clocks": out["prefill_m968"]["clocks"]}
     del pre, xp, pb, outs, outs_q, outs_d
     # ---- M sweep on the 1536 -> 6144 GEMM (bias, bf16 out), 48 distinct weights ----

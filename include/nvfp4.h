@@ -403,7 +403,7 @@ size_t nvfp4_program_bytes(int n_ops);
  * problems' 128 x 128 output tiles through one TMA / tensor-core pipeline, so the weight
  * stream does not stop at problem boundaries (kind 1).  Other programs run on the executor.
  * Validates the ops (the rules of the standalone calls, plus: at most 4096 ops (else
- * NVFP4_ERR_UNSUPPORTED_SHAPE); GEMM M <= 64, N % 64 == 0, K % 32 == 0; norm K <= 4096, bf16
+ * NVFP4_ERR_UNSUPPORTED_SHAPE); GEMM M <= 64, N % 64 == 0, K % 32 == 0; norm K <= 16384, bf16
  * input; each dep names an earlier op), chooses each GEMM's schedule, encodes the TMA
  * descriptors and copies the program into `buffer` (device, >= nvfp4_program_bytes(n_ops),
  * 256-byte aligned).  Synchronous (set-up time); the buffers the ops name must stay valid

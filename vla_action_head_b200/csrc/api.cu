@@ -756,7 +756,7 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
         if (o.type == NVFP4_OP_QUANTIZE_NORM) {
             if (o.M <= 0 || o.K <= 0 || o.x == nullptr || o.ldx < o.K) return NVFP4_ERR_INVALID_ARG;
             if (static_cast<int>(o.norm) < 0 || static_cast<int>(o.norm) > 4) return NVFP4_ERR_INVALID_ARG;
-            if (o.K % 16 != 0 || o.K > 4096) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+            if (o.K % 16 != 0 || o.K > 16384) return NVFP4_ERR_UNSUPPORTED_SHAPE;
             if (o.out_codes == nullptr || o.out_sf == nullptr || !scale_ok(o.out_global_scale))
                 return NVFP4_ERR_INVALID_ARG;
             if (!(o.eps >= 0.0f) || !std::isfinite(o.eps)) return NVFP4_ERR_INVALID_ARG;
@@ -765,7 +765,7 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             for (const void *pp : {o.gamma, o.beta, o.mod_scale, o.mod_shift})
                 if (pp != nullptr && !aligned16(pp)) return NVFP4_ERR_MISALIGNED;
             e.type = kOpNorm;
-            e.units = static_cast<unsigned>(o.M);
+            e.units = static_cast<unsigned>(std::min(o.M, grid));  // one row per CTA at a time; each CTA signals once
             e.norm.x = o.x;
             e.norm.M = o.M;
             e.norm.K = o.K;
@@ -779,7 +779,7 @@ nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, s
             e.norm.g = o.out_global_scale;
             e.norm.codes = o.out_codes;
             e.norm.sf = o.out_sf;
-            e.bpt = (o.K / 16 + 31) / 32;
+            e.bpt = (o.K / 16 + 127) / 128;  // 16-element blocks per worker thread (a row on 128 threads)
         } else if (o.type == NVFP4_OP_GEMM) {
             st = validate_gemm(&o.A, &o.W, o.M, o.N, o.K, o.epi, o.bias, o.residual, o.ldr, o.out_bf16, o.ldo,
                                o.out_codes, o.out_sf, o.out_global_scale);

@@ -3,25 +3,28 @@
 //
 // At M <= 64 tokens a linear layer is a chain of small dependent steps (norm, QKV GEMM,
 // attention-output GEMM, norm, FFN up, FFN down).  As separate kernels each step pays a
-// launch and a grid completion; here every CTA walks the same program, ops are ordered by
-// per-op completion counters in global memory (release by the finishing CTAs, acquire by
-// the consumers), and the weight tiles of later ops stream into each CTA's shared-memory
-// ring while the current op waits for its input -- weights never depend on activations.
+// grid completion and a launch boundary; here every CTA walks the same program, ops are
+// ordered by per-op completion counters in global memory (one release reduction per
+// finishing CTA, an acquire poll by the consumers), and the weight tiles of later ops stream
+// into each CTA's shared-memory ring while the current op waits for its input -- weights
+// never depend on activations.
 //
 // Roles (256 threads):
-//   warp 0      weight producer: TMA loads of W code tiles + bulk loads of their scale
-//               atoms, for every GEMM unit of this CTA in program order, as far ahead as the
-//               ring allows.
+//   warp 0      weight producer: TMA loads of W code tiles + bulk loads of their scale atoms,
+//               for every GEMM unit of this CTA in program order, as far ahead as the ring
+//               allows; they land on the stage's weight barrier.
+//   warp 7      weight-scale copier: tcgen05.cp of each stage's W scale atoms into the stage's
+//               TMEM scale slot as soon as the weights land (ahead of the activations).
+//   warp 2      activation producer: waits until the op's input is complete, TMA loads the A
+//               code tiles + scale atoms of the unit (activation barrier), then copies the A
+//               scale atoms into the slots as each stage lands.
 //   warp 1      MMA issuer: tcgen05.mma kind::mxf4nvf4 block16 into one of two TMEM
-//               accumulators.
-//   warp 7      scale copier: tcgen05.cp of each stage's scale atoms into one of two TMEM
-//               scale slots, a stage ahead of the MMAs (copies issued by the MMA thread itself
-//               would run one after another between its MMAs).
-//   warp 2      activation producer: waits until the op's input is complete, then TMA loads
-//               the A code tiles + scale atoms into the same ring stages.
-//   warps 3..6  epilogue and norm workers: TMEM -> registers -> fused epilogue; split-K
-//               partials are added on the tile's owner CTA over distributed shared memory
-//               in split order (deterministic); norm ops run one row per warp.
+//               accumulators once a stage's weights, activations and both scale copies are in.
+//   warps 3..6  workers: GEMM epilogues and norm rows.  Split-K partials are pushed to the
+//               CTA that owns each column slice (distributed shared memory), which adds them
+//               in split order (deterministic) and runs the fused epilogue; a tile that is not
+//               split runs its epilogue straight from the accumulator.  A norm op runs one row
+//               per CTA on all 128 workers.
 // GEMM work: the grid is a set of clusters of C CTAs; for an op split S ways (S | C), the
 // S CTAs that share a tile are cluster neighbours.  At start each CTA marks, in a shared-memory
 // bit set, the ops it has work in; the roles walk only those (a grouped GEMM of many small
@@ -42,14 +45,14 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRing = 6;
+constexpr int kRing = 6;        // stages; the TMEM scale slot of a stage is the stage's own
 constexpr int kStageA = 8192;   // 64 rows x 128 bytes (M <= 64)
 constexpr int kStageW = 16384;  // 128 rows x 128 bytes (block_n <= 128)
 constexpr int kStageSfa = 2048;
 constexpr int kStageSfb = 2048;
 constexpr int kStage = kStageA + kStageW + kStageSfa + kStageSfb;
-constexpr int kRedLd = 128 + 4;
-constexpr int kRedBytes = 64 * kRedLd * 4;
+// split-K partials received as a slice owner: S slices x 64 rows x (bn / S + 4) floats
+constexpr int kRedBytes = 64 * (128 + 16) * 4;
 constexpr int kOffRed = kRing * kStage;
 // staged epilogue inputs of this CTA's column slice: residual rows (bf16) and bias
 constexpr int kStgLd = 128 + 8;
@@ -57,17 +60,18 @@ constexpr int kOffStg = kOffRed + kRedBytes;
 constexpr int kStgBytes = 64 * kStgLd * 2;
 constexpr int kOffStgBias = kOffStg + kStgBytes;
 constexpr int kOffBar = kOffStgBias + 256;
-// barriers: full[R], empty[R], acc_full[2], acc_empty[2], sf_ready[2], sf_free[2]
-constexpr int kOffMisc = kOffBar + (2 * kRing + 8) * 8;
-// misc words: [0] TMEM base, [1] abort flag, [2] red_in (partials received as owner),
-// [3] red_free (frees received as member)
+// barriers: full_w[R], full_a[R], empty[R], sf_ready[R], acc_full[2], acc_empty[2]
+constexpr int kOffMisc = kOffBar + (4 * kRing + 4) * 8;
+// misc words: [0] TMEM base, [1] abort flag, [2] red_in (partial slices received as an
+// owner), [3] red_free (owners done with this CTA's partials), [4..11] four doubles (norm rows)
 constexpr int kOffMask = kOffMisc + 64;  // one bit per op: this CTA has work in it
 constexpr int kSmemBytes = kOffMask + kExecMaxOps / 8 + 1024;
-constexpr int kTmemCols = 512;  // two 128-column accumulators + two scale slots
+constexpr int kTmemCols = 512;  // two 128-column accumulators + kRing scale slots
 constexpr int kColSf = 256;     // scale slot j: A atoms at kColSf + 32 j, W atoms 16 columns on
 constexpr int kSfSlot = 32;
 constexpr int kSfAtom = 512;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kColSf + kRing * kSfSlot <= kTmemCols, "tensor memory columns");
 
 __device__ __forceinline__ unsigned int ld_acquire_cluster_smem(uint32_t addr) {
     unsigned int v;
@@ -77,11 +81,16 @@ __device__ __forceinline__ unsigned int ld_acquire_cluster_smem(uint32_t addr) {
 __device__ __forceinline__ void red_add_release_cluster(uint32_t cluster_addr, unsigned int v) {
     asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
+// Completion of an op by this CTA: one release reduction at GPU scope (it orders the CTA's
+// earlier stores, which the named barrier before it made visible to this thread).
+__device__ __forceinline__ void red_add_release_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void bar_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Barrier of the 128 epilogue threads that also ANDs a flag across them: every decision to
+// Barrier of the 128 worker threads that also ANDs a flag across them: every decision to
 // abandon the work is taken by all four warps together (a named barrier has no timeout, so
 // no warp may leave while the others still expect it).
 __device__ __forceinline__ bool bar_epi_and(bool v) {
@@ -97,12 +106,14 @@ __device__ __forceinline__ bool bar_epi_and(bool v) {
     return r != 0;
 }
 
-// Bounded wait until *p >= target (acquire, gpu scope).
+// Bounded wait until *p >= target (acquire, gpu scope): a tight poll first, then a short
+// back-off.
 __device__ bool wait_counter(const unsigned int *p, unsigned int target, volatile int *abort_flag, uint32_t *status) {
-    if (ld_acquire_gpu(p) >= target) return true;
+    for (int i = 0; i < 256; ++i)
+        if (ld_acquire_gpu(p) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        __nanosleep(64);
+        __nanosleep(32);
         if (ld_acquire_gpu(p) >= target) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -135,7 +146,8 @@ __device__ __forceinline__ int op_rounds(const ExecOp &op, int teams, int C) {
     const int per_round = teams * (C / op.splits);
     return (op.n_tiles + per_round - 1) / per_round;
 }
-// The GEMM unit of (team, rank) in round r, if any.
+// The GEMM unit of (team, rank) in round r, if any.  owner_rank: the cluster rank of the
+// group's split 0 (the group's CTAs are owner_rank .. owner_rank + splits - 1).
 __device__ __forceinline__ bool op_unit(const ExecOp &op, int team, int rank, int teams, int C, int r, Unit &u) {
     const int per_team = C / op.splits;
     const int t = team >= op.team0 ? team - op.team0 : team - op.team0 + teams;  // rotated team index
@@ -152,7 +164,7 @@ __device__ __forceinline__ bool op_unit(const ExecOp &op, int team, int rank, in
 // Whether CTA (team, rank) has any work in op i: a norm row, or a GEMM unit in round 0
 // (later rounds only add tiles to CTAs that have one in round 0).
 __device__ __forceinline__ bool has_work(const ExecOp &op, int team, int rank, int teams, int C) {
-    if (op.type == kOpNorm) return static_cast<int>(blockIdx.x) * 4 < op.norm.M;
+    if (op.type == kOpNorm) return static_cast<int>(blockIdx.x) < op.norm.M;
     Unit u;
     return op_unit(op, team, rank, teams, C, 0, u);
 }
@@ -165,22 +177,22 @@ __device__ __forceinline__ int next_op(const uint32_t *mask, int n_ops, int i) {
     return n_ops;
 }
 
-// Kept out of line: the norm path has its own register allocation, apart from the
-// epilogue's.
+// One norm row on the 128 workers (thread e of them), kept out of line: the norm path has its
+// own register allocation, apart from the epilogue's.
 template <int BPT>
-__device__ __noinline__ void norm_row_bpt(const NormArgs &a, int row, int lane) {
-    norm_row<32, BPT, false>(a, row, lane, nullptr);
+__device__ __noinline__ void norm_row_bpt(const NormArgs &a, int row, int e, double *red) {
+    norm_row<128, BPT, false>(a, row, e, red);
 }
-__device__ void norm_row_any(const NormArgs &a, int bpt, int row, int lane) {
+__device__ void norm_row_any(const NormArgs &a, int bpt, int row, int e, double *red) {
     switch (bpt) {
-    case 1: norm_row_bpt<1>(a, row, lane); break;
-    case 2: norm_row_bpt<2>(a, row, lane); break;
-    case 3: norm_row_bpt<3>(a, row, lane); break;
-    case 4: norm_row_bpt<4>(a, row, lane); break;
-    case 5: norm_row_bpt<5>(a, row, lane); break;
-    case 6: norm_row_bpt<6>(a, row, lane); break;
-    case 7: norm_row_bpt<7>(a, row, lane); break;
-    default: norm_row_bpt<8>(a, row, lane); break;
+    case 1: norm_row_bpt<1>(a, row, e, red); break;
+    case 2: norm_row_bpt<2>(a, row, e, red); break;
+    case 3: norm_row_bpt<3>(a, row, e, red); break;
+    case 4: norm_row_bpt<4>(a, row, e, red); break;
+    case 5: norm_row_bpt<5>(a, row, e, red); break;
+    case 6: norm_row_bpt<6>(a, row, e, red); break;
+    case 7: norm_row_bpt<7>(a, row, e, red); break;
+    default: norm_row_bpt<8>(a, row, e, red); break;
     }
 }
 
@@ -188,17 +200,18 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar_full = sbase + kOffBar;
-    const uint32_t bar_empty = bar_full + 8 * kRing;
-    const uint32_t bar_accf = bar_empty + 8 * kRing;
+    const uint32_t bar_fw = sbase + kOffBar;         // R: the stage's weights + weight scales landed
+    const uint32_t bar_fa = bar_fw + 8 * kRing;      // R: the stage's activations + their scales landed
+    const uint32_t bar_empty = bar_fa + 8 * kRing;   // R: the stage's MMAs are done with it (and its slot)
+    const uint32_t bar_sfr = bar_empty + 8 * kRing;  // R: both scale copies of the stage are in TMEM
+    const uint32_t bar_accf = bar_sfr + 8 * kRing;
     const uint32_t bar_acce = bar_accf + 16;
-    const uint32_t bar_sfr = bar_acce + 16;  // 2: scale slot copied
-    const uint32_t bar_sff = bar_sfr + 16;   // 2: scale slot read by its MMAs
     uint32_t *opmask = reinterpret_cast<uint32_t *>(smem + kOffMask);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
     const uint32_t red_in_addr = sbase + kOffMisc + 8;
     const uint32_t red_free_addr = sbase + kOffMisc + 12;
+    double *norm_red = reinterpret_cast<double *>(smem + kOffMisc + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = P.cluster;
@@ -208,14 +221,14 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kRing; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_fw + 8 * s, 1);
+            mbar_init(bar_fa + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_sfr + 8 * s, 2);  // the weight-scale copier and the activation producer
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_accf + 8 * b, 1);
             mbar_init(bar_acce + 8 * b, 1);
-            mbar_init(bar_sfr + 8 * b, 1);
-            mbar_init(bar_sff + 8 * b, 1);
         }
         misc[1] = 0;
         misc[2] = 0;
@@ -241,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
 
     auto nkb_of = [&](const ExecOp &op, int kt) { return min(4, op.k_atoms - 4 * kt); };
     // diagnostics: per (op, CTA) [0] W issued first tile, [1] A dependency seen, [2] first
-    // stage full (MMA), [3] last MMA issued, [4] accumulator ready (epilogue), [5] partials in
-    // (split groups), [6] op signalled, [7] norm rows done / accumulator drained (GEMM)
+    // stage full (MMA), [3] last MMA issued, [4] accumulator ready, [5] partials in (split
+    // groups), [6] op signalled, [7] norm rows done / accumulator drained (GEMM)
     auto stamp = [&](int op_i, int k) {
         if (P.trace != nullptr) P.trace[(static_cast<size_t>(op_i) * gridDim.x + blockIdx.x) * 8 + k] = globaltimer_ns();
     };
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         const uint64_t pol = policy_evict_first();
         int step = 0;
         for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
-            const ExecOp op = P.ops[i];
+            const ExecOp &op = P.ops[i];  // read in place: a local copy would live in (L1-starved) local memory
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmB = P.maps + op.tm_b;
             const int rounds = op_rounds(op, teams, C);
@@ -265,10 +278,10 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                                               kStatusTimeoutEmpty))
                         goto done_w;
                     const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
-                    const uint32_t full = bar_full + 8 * slot;
+                    const uint32_t full = bar_fw + 8 * slot;
                     const uint32_t st = sbase + slot * kStage;
                     if (kt == u.kt0) stamp(i, 0);
-                    mbar_arrive_expect_tx(full, op.a_box_rows * 128u + static_cast<uint32_t>(op.bn) * 128u + 2 * nb);
+                    mbar_arrive_expect_tx(full, static_cast<uint32_t>(op.bn) * 128u + nb);
                     tma_load_2d(st + kStageA, tmB, kt * 128, u.tile * op.bn, full, pol);
                     const size_t grp = static_cast<size_t>((u.tile * op.bn) / 128);
                     bulk_load(st + kStageA + kStageW + kStageSfa, op.sfb + (grp * op.k_atoms + 4 * kt) * kSfAtom, nb,
@@ -277,12 +290,43 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
             }
         }
     done_w:;
+    } else if (warp == 7 && lane == 0) {
+        // ---------------------------- weight-scale copier ----------------------------
+        // The W scale atoms of a stage go into the stage's TMEM slot as soon as they land.  The
+        // slot is free then: the stage was released (its MMAs done) before these weights were
+        // loaded into it.
+        int step = 0;
+        for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
+            const ExecOp &op = P.ops[i];  // read in place: a local copy would live in (L1-starved) local memory
+            if (op.type != kOpGemm) continue;
+            const int rounds = op_rounds(op, teams, C);
+            for (int r = 0; r < rounds; ++r) {
+                Unit u;
+                if (!op_unit(op, team, rank, teams, C, r, u)) continue;
+                for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
+                    const int slot = step % kRing, use = step / kRing;
+                    if (!mbar_wait(bar_fw + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
+                        goto done_c;
+                    tc_fence_after();
+                    const int nkb = nkb_of(op, kt);
+                    const uint32_t st = sbase + slot * kStage;
+                    const uint32_t t_sf = tmem + kColSf + slot * kSfSlot;
+                    for (int kb = 0; kb < nkb; ++kb)
+                        tc_cp_32x128b_warpx4(t_sf + 16 + 4 * kb,
+                                             desc_sf_32x128b(st + kStageA + kStageW + kStageSfa + kb * kSfAtom));
+                    tc_commit(bar_sfr + 8 * slot);  // arrives once the copies have landed
+                }
+            }
+        }
+    done_c:;
     } else if (warp == 2 && lane == 0) {
         // ---------------------------- activation producer ----------------------------
+        // Per unit: every A stage is requested at once, then each stage's A scale atoms are
+        // copied into its TMEM slot as it lands.
         const uint64_t pol = policy_evict_last();
         int step = 0;
         for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
-            const ExecOp op = P.ops[i];
+            const ExecOp &op = P.ops[i];  // read in place: a local copy would live in (L1-starved) local memory
             if (op.type != kOpGemm) continue;
             const CUtensorMap *tmA = P.maps + op.tm_a;
             bool ready = false;
@@ -296,16 +340,36 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                     ready = true;
                     stamp(i, 1);
                 }
-                for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
-                    const int slot = step % kRing, use = step / kRing;
-                    if (use > 0 && !mbar_wait(bar_empty + 8 * slot, (use - 1) & 1, abort_flag, P.status,
-                                              kStatusTimeoutEmpty))
-                        goto done_a;
-                    const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
-                    const uint32_t full = bar_full + 8 * slot;
-                    const uint32_t st = sbase + slot * kStage;
-                    tma_load_2d(st, tmA, kt * 128, 0, full, pol);
-                    bulk_load(st + kStageA + kStageW, op.sfa + static_cast<size_t>(4 * kt) * kSfAtom, nb, full, pol);
+                // batches of at most kRing stages: a stage is reused only after its MMAs, which
+                // wait for the scale copies this thread makes after the batch's loads
+                for (int kb0 = u.kt0; kb0 < u.kt1; kb0 += kRing) {
+                    const int kb1 = min(u.kt1, kb0 + kRing), step0 = step;
+                    for (int kt = kb0; kt < kb1; ++kt, ++step) {
+                        const int slot = step % kRing, use = step / kRing;
+                        if (use > 0 && !mbar_wait(bar_empty + 8 * slot, (use - 1) & 1, abort_flag, P.status,
+                                                  kStatusTimeoutEmpty))
+                            goto done_a;
+                        const uint32_t nb = static_cast<uint32_t>(nkb_of(op, kt)) * kSfAtom;
+                        const uint32_t full = bar_fa + 8 * slot;
+                        const uint32_t st = sbase + slot * kStage;
+                        mbar_arrive_expect_tx(full, op.a_box_rows * 128u + nb);
+                        tma_load_2d(st, tmA, kt * 128, 0, full, pol);
+                        bulk_load(st + kStageA + kStageW, op.sfa + static_cast<size_t>(4 * kt) * kSfAtom, nb, full,
+                                  pol);
+                    }
+                    step = step0;
+                    for (int kt = kb0; kt < kb1; ++kt, ++step) {
+                        const int slot = step % kRing, use = step / kRing;
+                        if (!mbar_wait(bar_fa + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
+                            goto done_a;
+                        tc_fence_after();
+                        const int nkb = nkb_of(op, kt);
+                        const uint32_t st = sbase + slot * kStage;
+                        const uint32_t t_sf = tmem + kColSf + slot * kSfSlot;
+                        for (int kb = 0; kb < nkb; ++kb)
+                            tc_cp_32x128b_warpx4(t_sf + 4 * kb, desc_sf_32x128b(st + kStageA + kStageW + kb * kSfAtom));
+                        tc_commit(bar_sfr + 8 * slot);
+                    }
                 }
             }
         }
@@ -314,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
         // ---------------------------- MMA issuer ----------------------------
         int step = 0, unit_idx = 0;
         for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
-            const ExecOp op = P.ops[i];
+            const ExecOp &op = P.ops[i];  // read in place: a local copy would live in (L1-starved) local memory
             if (op.type != kOpGemm) continue;
             const uint32_t idesc = idesc_mxf4nvf4(128, op.bn);
             const int rounds = op_rounds(op, teams, C);
@@ -330,20 +394,20 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 // a 64-row W tile reads its half of the 128-row scale atom
                 const uint32_t sub = (op.bn == 64) ? static_cast<uint32_t>(((u.tile * op.bn) & 127) >> 5) : 0u;
                 for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
-                    const int slot = step % kRing, use = step / kRing, sfs = step & 1;
-                    if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull) ||
-                        !mbar_wait(bar_sfr + 8 * sfs, (step >> 1) & 1, abort_flag, P.status, kStatusTimeoutFull))
+                    const int slot = step % kRing, use = step / kRing;
+                    if (!mbar_wait(bar_fw + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull) ||
+                        !mbar_wait(bar_fa + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull) ||
+                        !mbar_wait(bar_sfr + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
                         goto done_m;
                     tc_fence_after();
                     if (kt == u.kt0) stamp(i, 2);
                     const int nkb = nkb_of(op, kt);
                     const uint32_t st = sbase + slot * kStage;
-                    const uint32_t t_sf = tmem + kColSf + sfs * kSfSlot;
+                    const uint32_t t_sf = tmem + kColSf + slot * kSfSlot;
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_mxf4nvf4(t_acc, desc_kmajor_sw128(st + 32 * kb), desc_kmajor_sw128(st + kStageA + 32 * kb),
                                         idesc, t_sf + 4 * kb, t_sf + 16 + 4 * kb + sub, (kt > u.kt0 || kb > 0) ? 1u : 0u);
-                    tc_commit(bar_empty + 8 * slot);  // the stage, once these MMAs have read it
-                    tc_commit(bar_sff + 8 * sfs);     // and the scale slot
+                    tc_commit(bar_empty + 8 * slot);  // the stage and its scale slot, once these MMAs are done
                 }
                 stamp(i, 3);
                 tc_commit(bar_accf + 8 * b);
@@ -351,75 +415,36 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
             }
         }
     done_m:;
-    } else if (warp == 7) {
-        if (lane == 0) {
-            // ---------------------------- scale copier ----------------------------
-            // Same walk of k-tile steps as the MMA issuer; step s uses scale slot s & 1, free
-            // again once the MMAs of step s - 2 have completed.
-            int step = 0;
-            for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
-                const ExecOp op = P.ops[i];
-                if (op.type != kOpGemm) continue;
-                const int rounds = op_rounds(op, teams, C);
-                for (int r = 0; r < rounds; ++r) {
-                    Unit u;
-                    if (!op_unit(op, team, rank, teams, C, r, u)) continue;
-                    for (int kt = u.kt0; kt < u.kt1; ++kt, ++step) {
-                        const int slot = step % kRing, use = step / kRing, sfs = step & 1;
-                        if (!mbar_wait(bar_full + 8 * slot, use & 1, abort_flag, P.status, kStatusTimeoutFull))
-                            goto done_c;
-                        if (step >= 2 && !mbar_wait(bar_sff + 8 * sfs, ((step >> 1) - 1) & 1, abort_flag, P.status,
-                                                    kStatusTimeoutFull))
-                            goto done_c;
-                        tc_fence_after();
-                        const int nkb = nkb_of(op, kt);
-                        const uint32_t st = sbase + slot * kStage;
-                        const uint32_t t_sf = tmem + kColSf + sfs * kSfSlot;
-                        for (int kb = 0; kb < nkb; ++kb) {
-                            tc_cp_32x128b_warpx4(t_sf + 4 * kb, desc_sf_32x128b(st + kStageA + kStageW + kb * kSfAtom));
-                            tc_cp_32x128b_warpx4(t_sf + 16 + 4 * kb,
-                                                 desc_sf_32x128b(st + kStageA + kStageW + kStageSfa + kb * kSfAtom));
-                        }
-                        tc_commit(bar_sfr + 8 * sfs);  // arrives once the copies have landed
-                    }
-                }
-            }
-        done_c:;
-        }
-    } else if (warp >= 3) {
-        // ---------------------------- epilogue / norm workers ----------------------------
+    } else if (warp >= 3 && warp <= 6) {
+        // ---------------------------- workers: epilogues and norm rows ----------------------------
         const int e = threadIdx.x - 96;  // 0..127
-        const int ew = e >> 5;           // worker warp 0..3
         const int q = warp & 3;          // TMEM sub-partition this warp reads
         const int row = q * 32 + lane;
         int unit_idx = 0;
         unsigned int in_expected = 0, free_expected = 0;  // split-group signals expected so far
         for (int i = next_op(opmask, P.n_ops, -1); i < P.n_ops; i = next_op(opmask, P.n_ops, i)) {
-            const ExecOp op = P.ops[i];
+            const ExecOp &op = P.ops[i];  // read in place: a local copy would live in (L1-starved) local memory
             if (op.type == kOpNorm) {
-                const int rows_per_round = gridDim.x * 4;
-                if (blockIdx.x * 4 >= op.norm.M) continue;  // no rows for this CTA
+                // one row at a time on all 128 workers: rows blockIdx.x, blockIdx.x + grid, ...
                 const bool ok = (e != 0) || op.dep < 0 || wait_counter(P.done + op.dep, P.ops[op.dep].units, abort_flag, P.status);
                 if (!bar_epi_and(ok)) goto done_e;
                 if (e == 0) stamp(i, 1);
-                for (int rr = blockIdx.x * 4 + ew; rr < op.norm.M; rr += rows_per_round) {
-                    norm_row_any(op.norm, op.bpt, rr, lane);
-                    __syncwarp();
-                    if (lane == 0 && op.signal) {
-                        __threadfence();
-                        atomicAdd(P.done + i, 1u);
-                    }
+                for (int rr = blockIdx.x; rr < op.norm.M; rr += gridDim.x) norm_row_any(op.norm, op.bpt, rr, e, norm_red);
+                bar_epi();
+                if (e == 0) {
+                    if (op.signal) red_add_release_gpu(P.done + i, 1u);
+                    stamp(i, 7);
                 }
-                if (e == 0) stamp(i, 7);
                 continue;
             }
-            // GEMM op.  Every CTA of a split group finalizes its own slice of bn / S columns
-            // (a multiple of 32): it adds the S partials of those columns in split order, the
-            // first from its own shared memory or a peer's over DSMEM, and runs the epilogue.
+            // GEMM op.  CTA k of a split group owns column slice k (bn / S columns, a multiple of
+            // 32) of the group's tile: every CTA pushes its partial of slice k to CTA k, which
+            // adds the S partials in split order and runs the epilogue of its slice.
             const int rounds = op_rounds(op, teams, C);
             const int S = op.splits;
             const int slice = op.bn / S;
             const int chunks = slice / 32;
+            const int red_ld = slice + 4;
             const bool has_bias = op.bias != nullptr && (op.epi == kEpiBias || op.epi == kEpiBiasResidual ||
                                                          op.epi == kEpiBiasGelu || op.epi == kEpiGeglu);
             const bool has_res = op.residual != nullptr && (op.epi == kEpiResidual || op.epi == kEpiBiasResidual);
@@ -453,118 +478,111 @@ __global__ void __launch_bounds__(kThreads, 1) exec_kernel(const ExecParams P) {
                 if (has_bias && e < slice / 8)
                     *reinterpret_cast<uint4 *>(stg_bias + 8 * e) =
                         __ldg(reinterpret_cast<const uint4 *>(op.bias + n0 + c0 + 8 * e));
+                // before pushing into the group's buffers: every owner is done with this CTA's
+                // previous partials (one thread waits; the barrier orders the others after it)
+                if (!bar_epi_and(e != 0 || S == 1 || free_expected == 0 ||
+                                 wait_smem_counter(red_free_addr, free_expected, abort_flag, P.status)))
+                    goto done_e;
                 const int b = unit_idx & 1, acc_use = unit_idx >> 1;
                 const bool got = mbar_wait(bar_accf + 8 * b, acc_use & 1, abort_flag, P.status,
                                            kStatusTimeoutAccum);
                 if (!bar_epi_and(got)) goto done_e;
                 tc_fence_after();
                 if (e == 0) stamp(i, 4);
-                // peers have finished reading this CTA's previous partial
-                // (one thread waits; the barrier orders the others after its acquire)
-                if (!bar_epi_and(e != 0 || free_expected == 0 ||
-                                 wait_smem_counter(red_free_addr, free_expected, abort_flag, P.status)))
-                    goto done_e;
-                // TMEM -> shared memory (rows_valid rows, all bn columns)
-                if (q * 32 < rows_valid) {
-                    const uint32_t t_row =
-                        tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
-                    for (int cc = 0; cc < op.bn; cc += 32) {
-                        uint32_t rg[32];
-                        tmem_ld_32x32b_x32(t_row + cc, rg);
-                        tmem_ld_wait();
-                        if (row < rows_valid) {
-                            float4 *dst = reinterpret_cast<float4 *>(red + row * kRedLd + cc);
+                const uint32_t t_row = tmem + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(q * 32) << 16);
+                if (S == 1) {
+                    // the whole tile is this CTA's: the epilogue straight from the accumulator
+                    if (q * 32 < rows_valid) {  // warp-uniform: tcgen05.ld is .sync.aligned
+                        for (int cc = 0; cc < op.bn; cc += 32) {
+                            uint32_t rg[32];
+                            tmem_ld_32x32b_x32(t_row + cc, rg);
+                            tmem_ld_wait();
+                            if (row < rows_valid) {
+                                float v[32];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                dst[j] = make_float4(__uint_as_float(rg[4 * j]), __uint_as_float(rg[4 * j + 1]),
-                                                     __uint_as_float(rg[4 * j + 2]), __uint_as_float(rg[4 * j + 3]));
+                                for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(rg[t]);
+                                epilogue_chunk_src(op, row, n0 + cc, v, has_bias ? stg_bias + cc : nullptr,
+                                                   has_res ? stg + row * kStgLd + cc : nullptr);
+                            }
                         }
                     }
-                }
-                tc_fence_before();
-                bar_epi();
-                if (e == 0) {
-                    mbar_arrive(bar_acce + 8 * b);  // the accumulator is free again
-                    stamp(i, 7);
-                }
-                if (S > 1) {
-                    if (e == 0)
-                        for (int sp = 0; sp < S; ++sp)
-                            red_add_release_cluster(mapa_shared(red_in_addr, static_cast<uint32_t>(u.owner_rank + sp)),
-                                                    1u);
+                    tc_fence_before();
+                    bar_epi();
+                    if (e == 0) {
+                        mbar_arrive(bar_acce + 8 * b);  // the accumulator is free again
+                        stamp(i, 7);
+                    }
+                } else {
+                    // push: chunk cc goes to slice owner owner_rank + cc / slice, as split u.split
+                    if (q * 32 < rows_valid) {
+                        for (int cc = 0; cc < op.bn; cc += 32) {
+                            uint32_t rg[32];
+                            tmem_ld_32x32b_x32(t_row + cc, rg);
+                            tmem_ld_wait();
+                            if (row < rows_valid) {
+                                const int k = cc / slice;
+                                const uint32_t dst = mapa_shared(
+                                    smem_u32(red + (u.split * 64 + row) * red_ld + (cc - k * slice)),
+                                    static_cast<uint32_t>(u.owner_rank + k));
+#pragma unroll
+                                for (int j = 0; j < 8; ++j)
+                                    st_dsmem_f4(dst + 16 * j,
+                                                make_float4(__uint_as_float(rg[4 * j]), __uint_as_float(rg[4 * j + 1]),
+                                                            __uint_as_float(rg[4 * j + 2]),
+                                                            __uint_as_float(rg[4 * j + 3])));
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    bar_epi();
+                    if (e == 0) {
+                        mbar_arrive(bar_acce + 8 * b);  // the accumulator is free again
+                        stamp(i, 7);
+                        for (int k = 0; k < S; ++k)
+                            red_add_release_cluster(mapa_shared(red_in_addr, static_cast<uint32_t>(u.owner_rank + k)), 1u);
+                    }
                     in_expected += static_cast<unsigned>(S);
                     if (!bar_epi_and(e != 0 || wait_smem_counter(red_in_addr, in_expected, abort_flag, P.status)))
                         goto done_e;
                     if (e == 0) stamp(i, 5);
-                }
-                for (int item = e;; item += 128) {
-                    const int i_row = item / chunks, ch = item % chunks;
-                    if (i_row >= rows_valid) break;
-                    const int col = c0 + 32 * ch;
-                    float v[32];
-                    if (S == 1) {
-                        const float4 *src4 = reinterpret_cast<const float4 *>(red + i_row * kRedLd + col);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 w = src4[j];
-                            v[4 * j] = w.x;
-                            v[4 * j + 1] = w.y;
-                            v[4 * j + 2] = w.z;
-                            v[4 * j + 3] = w.w;
-                        }
-                    } else {
-                        const uint32_t local = smem_u32(red + i_row * kRedLd + col);
-                        uint32_t src[4];
-#pragma unroll
-                        for (int sp = 0; sp < 4; ++sp)
-                            src[sp] = mapa_shared(local, static_cast<uint32_t>(u.owner_rank + (sp < S ? sp : 0)));
+                    for (int item = e;; item += 128) {
+                        const int i_row = item / chunks, ch = item % chunks;
+                        if (i_row >= rows_valid) break;
+                        float v[32];
 #pragma unroll
                         for (int t = 0; t < 32; ++t) v[t] = 0.0f;
-                        // 16 columns at a time: every partial's loads are in flight together
+                        for (int sp = 0; sp < S; ++sp) {
+                            const float4 *src4 = reinterpret_cast<const float4 *>(red + (sp * 64 + i_row) * red_ld + 32 * ch);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            float4 w4[4][4];
-#pragma unroll
-                            for (int sp = 0; sp < 4; ++sp)
-                                if (sp < S)
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) w4[sp][j] = ld_dsmem_f4(src[sp] + 64 * h + 16 * j);
-#pragma unroll
-                            for (int sp = 0; sp < 4; ++sp)
-                                if (sp < S)
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        float *vv = v + 16 * h + 4 * j;
-                                        vv[0] = __fadd_rn(vv[0], w4[sp][j].x);
-                                        vv[1] = __fadd_rn(vv[1], w4[sp][j].y);
-                                        vv[2] = __fadd_rn(vv[2], w4[sp][j].z);
-                                        vv[3] = __fadd_rn(vv[3], w4[sp][j].w);
-                                    }
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 w4 = src4[j];
+                                v[4 * j] = __fadd_rn(v[4 * j], w4.x);
+                                v[4 * j + 1] = __fadd_rn(v[4 * j + 1], w4.y);
+                                v[4 * j + 2] = __fadd_rn(v[4 * j + 2], w4.z);
+                                v[4 * j + 3] = __fadd_rn(v[4 * j + 3], w4.w);
+                            }
                         }
+                        epilogue_chunk_src(op, i_row, n0 + c0 + 32 * ch, v, has_bias ? stg_bias + 32 * ch : nullptr,
+                                           has_res ? stg + i_row * kStgLd + 32 * ch : nullptr);
                     }
-                    epilogue_chunk_src(op, i_row, n0 + col, v, has_bias ? stg_bias + 32 * ch : nullptr,
-                                       has_res ? stg + i_row * kStgLd + 32 * ch : nullptr);
+                    bar_epi();
+                    if (e == 0)  // this CTA is done with the group's partials of this unit
+                        for (int k = 0; k < S; ++k)
+                            red_add_release_cluster(mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + k)),
+                                                    1u);
+                    free_expected += static_cast<unsigned>(S);
                 }
-                bar_epi();
                 if (e == 0) {
-                    if (S > 1)
-                        for (int sp = 0; sp < S; ++sp)
-                            red_add_release_cluster(
-                                mapa_shared(red_free_addr, static_cast<uint32_t>(u.owner_rank + sp)), 1u);
-                    if (op.signal) {  // only ops that a later op waits for count completions
-                        __threadfence();
-                        atomicAdd(P.done + i, 1u);
-                    }
+                    if (op.signal) red_add_release_gpu(P.done + i, 1u);  // only ops a later op waits for
                     stamp(i, 6);
                 }
-                if (S > 1) free_expected += static_cast<unsigned>(S);
                 ++unit_idx;
             }
         }
     done_e:;
     }
 
-    // teardown: peers may still read this CTA's shared memory until everyone is done
+    // teardown: peers may still write this CTA's shared memory until everyone is done
     __syncwarp();
     if (*abort_flag) {
         // an abandoned run may leave copies or MMAs in flight: give them time to land

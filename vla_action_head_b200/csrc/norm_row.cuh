@@ -27,17 +27,21 @@ namespace nvfp4 {
 
 enum { kNone = 0, kLayerNorm = 1, kRmsNorm = 2, kAdaLN = 3, kAdaRms = 4 };
 
+// Sum of v over the TPR threads of a row (t = the thread's index among them).  TPR = 128:
+// the four warps meet on named barrier 1 (they are the whole CTA of the standalone kernel, or
+// the four worker warps of the layer executor), with `red` four doubles of shared memory.
 template <int TPR>
-__device__ __forceinline__ double row_sum(double v, double *red) {
+__device__ __forceinline__ double row_sum(double v, double *red, int t) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
     if constexpr (TPR == 32) {
         return v;
     } else {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-        __syncthreads();
+        static_assert(TPR == 128, "a row is one warp or four");
+        const int warp = t >> 5, lane = t & 31;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         if (lane == 0) red[warp] = v;
-        __syncthreads();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         double s = 0.0;
 #pragma unroll
         for (int w = 0; w < TPR / 32; ++w) s = __dadd_rn(s, red[w]);
@@ -58,8 +62,8 @@ __device__ __forceinline__ double block_sum16(Elem elem) {
     return v[0];
 }
 
-// Row `row` of p, handled by thread t of TPR (TPR = 32: one warp; TPR = 128: the CTA, with
-// `red` four doubles of shared memory).  TPR, BPT (blocks of 16 per thread) and F32 (fp32
+// Row `row` of p, handled by thread t of TPR (TPR = 32: one warp; TPR = 128: four warps on
+// named barrier 1, with `red` four doubles of shared memory).  TPR, BPT (blocks of 16 per thread) and F32 (fp32
 // input, else bf16) are compile-time; K <= 16 * TPR * BPT.
 //
 // Latency is what matters at tens of rows, so every global load of the row is issued
@@ -185,7 +189,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
         double s = 0.0;
 #pragma unroll
         for (int i = 0; i < BPT; ++i) s = __dadd_rn(s, block_sum16([&](int e) { return elem(i, e); }));
-        s = row_sum<TPR>(s, red);
+        s = row_sum<TPR>(s, red, t);
         const double mu = __ddiv_rn(s, static_cast<double>(K));
         double q = 0.0;
 #pragma unroll
@@ -204,7 +208,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
                 q = __dadd_rn(q, d[0]);
             }
         }
-        q = row_sum<TPR>(q, red);
+        q = row_sum<TPR>(q, red, t);
         mu_f = static_cast<float>(mu);
         rstd_f = static_cast<float>(
             __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(K)), static_cast<double>(eps)))));
@@ -224,7 +228,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
                 for (int e = 0; e < w; ++e) d[e] = __dadd_rn(d[e], d[e + w]);
             q = __dadd_rn(q, d[0]);
         }
-        q = row_sum<TPR>(q, red);
+        q = row_sum<TPR>(q, red, t);
         rstd_f = static_cast<float>(
             __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(q, static_cast<double>(K)), static_cast<double>(eps)))));
     }
