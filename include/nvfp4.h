@@ -164,10 +164,9 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * split-K).  Launches that no longer fit are not traced.  Setting
  * a buffer (or NULL, which turns tracing off) rewinds the cursor.  Host-side state, not
  * thread safe; captured launches keep the slice they got at capture.
- * nvfp4_program_run, when the buffer holds n_ops * grid * 8 words, writes 8 stamps per
- * (op, CTA) at ((op * grid) + cta) * 8: weight tile issued, input ready, first stage
- * landed, last MMA issued, accumulator ready, partials received, op signalled, and norm
- * rows done (norm ops) or accumulator drained to shared memory (GEMM ops). */
+ * nvfp4_program_run (grouped GEMM), when the buffer holds grid * 8 words, writes per CTA
+ * at cta * 8: entry, first stage landed, last MMA issued, exit and per-tile stamps (see
+ * gemm_grouped.cu). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
@@ -334,54 +333,44 @@ nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, 
 
 size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int splits);
 
-/* ---- layer executor: a whole program of ops in one launch --------------------------- */
+/* ---- grouped GEMM (a program of independent GEMMs in one launch) -------------------- */
 
-/* At M <= 64 tokens a transformer layer's linear path is a chain of small dependent steps.
- * Launched as separate kernels, each step pays a launch and a grid completion of several
- * microseconds.  A program runs the chain in ONE persistent cooperative launch:
- *   - every CTA walks the ops in order;
- *   - an op starts consuming its input once the previous op's completion counter is full;
- *   - the weight tiles of later ops stream into shared memory while earlier ops run,
- *     since weights never depend on activations.
- * Results are those of the standalone calls.  The norm op is nvfp4_quantize_norm; the GEMM
- * op is nvfp4_gemm with the same epilogues, its split-K partials added in split order
- * over distributed shared memory.  ([GROOT] §Summary and §What is in the tier: the DiT
- * action head at M = 41 is weight-bandwidth bound and runs as one captured graph; [PI05]
- * §Implemented Path: the whole path is CUDA-graph capturable.) */
+/* A grouped GEMM runs many independent NVFP4 GEMMs -- e.g. the 32 per-frame cross-attention
+ * K / V projections of a DiT ([GROOT] §What is in the tier) -- in ONE launch of the grouped
+ * persistent kernel: one CTA per SM walks all the problems' 128 x 128 output tiles through
+ * one TMA / tensor-core pipeline, so the weight stream does not stop at problem
+ * boundaries.  Results are those of nvfp4_gemm on each problem (one split per tile).
+ * Each op is described by an nvfp4_op of type NVFP4_OP_GEMM with dep = NVFP4_DEP_NONE; the
+ * norm fields and other dep values belong to an earlier interface of this struct and are
+ * rejected (NVFP4_ERR_UNSUPPORTED_SHAPE). */
 typedef enum { NVFP4_OP_QUANTIZE_NORM = 0, NVFP4_OP_GEMM = 1 } nvfp4_op_type;
 
 typedef struct {
-    nvfp4_op_type type;
+    nvfp4_op_type type;  /* NVFP4_OP_GEMM */
     int M, N, K;
-    /* NVFP4_OP_QUANTIZE_NORM: bf16 x [M, K] (ldx) -> out_codes / out_sf (pre-zeroed) */
+    /* unused (must describe no work): */
     const void *x;
     int ldx;
     nvfp4_norm norm;
     const void *gamma, *beta, *mod_scale, *mod_shift;
     float eps;
-    /* NVFP4_OP_GEMM: A (M x K) times W (N x K)^T, epilogue as nvfp4_gemm */
+    /* A (M x K) times W (N x K)^T, epilogue as nvfp4_gemm */
     nvfp4_tensor A, W;
     nvfp4_epilogue epi;
     const void *bias, *residual;
     int ldr;
     void *out_bf16;
     int ldo;
-    /* FP4 output: of the norm op, or of a BIAS_GELU / GEGLU epilogue */
+    /* FP4 output of a BIAS_GELU / GEGLU epilogue (and their rotated forms) */
     uint8_t *out_codes, *out_sf;
     float out_global_scale;
-    /* The earlier op whose results this op reads (its input, and a GEMM's residual):
-     *   NVFP4_DEP_PREVIOUS (0, what a zeroed op gets): the op just before it;
-     *   NVFP4_DEP_NONE (-1): none -- its inputs are ready before the run starts;
-     *   j + 1, for 0 <= j < this op's index: op j.
-     * A run of ops with NVFP4_DEP_NONE is a grouped GEMM: one launch streams every op's
-     * weights with no wait between ops. */
-    int dep;
+    int dep;  /* NVFP4_DEP_NONE: the op's inputs are ready before the launch */
 } nvfp4_op;
 
 #define NVFP4_DEP_PREVIOUS 0
 #define NVFP4_DEP_NONE (-1)
 
-/* Host-side handle of a built program; the device data lives in `buffer`. */
+/* Host-side handle of a built grouped GEMM; the device data lives in `buffer`. */
 typedef struct {
     void *buffer;
     size_t bytes;
@@ -389,31 +378,25 @@ typedef struct {
     int grid;
     int cluster;
     size_t ops_offset, maps_offset, done_offset;
-    int waits;  /* ops that wait for another op (0: the completion counters go unused) */
-    int kind;   /* 0: the layer executor; 1: the grouped GEMM kernel (see nvfp4_program_build) */
-    int epi;    /* kind 1: the epilogue of every op */
-    int tiles;  /* kind 1: output tiles over all ops */
+    int waits;  /* 0 */
+    int kind;   /* 1: the grouped GEMM kernel */
+    int epi;    /* the epilogue of every op */
+    int tiles;  /* output tiles over all ops */
 } nvfp4_program;
 
-/* Device bytes a program of n_ops ops needs. */
+/* Device bytes a grouped GEMM of n_ops problems needs. */
 size_t nvfp4_program_bytes(int n_ops);
 
-/* A program of 2..256 GEMM ops that all have dep = NVFP4_DEP_NONE, the same epilogue and
- * N % 128 == 0 is a grouped GEMM and runs on the grouped kernel: one CTA per SM walks all the
- * problems' 128 x 128 output tiles through one TMA / tensor-core pipeline, so the weight
- * stream does not stop at problem boundaries (kind 1).  Other programs run on the executor.
- * Validates the ops (the rules of the standalone calls, plus: at most 4096 ops (else
- * NVFP4_ERR_UNSUPPORTED_SHAPE); GEMM M <= 64, N % 64 == 0, K % 32 == 0; norm K <= 16384, bf16
- * input; each dep names an earlier op), chooses each GEMM's schedule, encodes the TMA
- * descriptors and copies the program into `buffer` (device, >= nvfp4_program_bytes(n_ops),
- * 256-byte aligned).  Synchronous (set-up time); the buffers the ops name must stay valid
- * for every later run. */
+/* Builds a grouped GEMM of 1..256 GEMM ops that all have dep = NVFP4_DEP_NONE, the same
+ * epilogue and N % 128 == 0 (else NVFP4_ERR_UNSUPPORTED_SHAPE).  Validates each op by the
+ * rules of nvfp4_gemm, encodes the TMA descriptors and copies the problems and their tile
+ * table into `buffer` (device, >= nvfp4_program_bytes(n_ops), 256-byte aligned).
+ * Synchronous (set-up time); the buffers the ops name must stay valid for every later run. */
 nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes,
                                  nvfp4_program *prog);
 
-/* Runs the program on `stream`: zeroes its completion counters (cudaMemsetAsync; skipped
- * when no op waits for another, as in a grouped GEMM) and makes one cooperative launch.  Allocates nothing; capturable in a CUDA graph.  Runs of the same
- * program must not overlap. */
+/* Runs the grouped GEMM on `stream`: one launch.  Allocates nothing; capturable in a CUDA
+ * graph.  Runs of the same program must not overlap. */
 nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream);
 
 #ifdef __cplusplus

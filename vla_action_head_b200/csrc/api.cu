@@ -14,7 +14,6 @@
 #include <vector>
 
 #include "../../include/nvfp4.h"
-#include "exec.h"
 #include "gemm.h"
 #include "norm.h"
 
@@ -677,17 +676,13 @@ nvfp4_status nvfp4_gemm_ex(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, 
                      workspace, ws_bytes, block_n, splits, stream);
 }
 
-// ---- layer executor ---------------------------------------------------------------------
-static constexpr int kExecCluster = 4;
-static constexpr int kExecRing = 6;
-
+// ---- grouped GEMM programs -------------------------------------------------------------------
 size_t nvfp4_program_bytes(int n_ops) {
     if (n_ops <= 0) return 0;
     const size_t maps = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
-    const size_t ops = (static_cast<size_t>(n_ops) * sizeof(ExecOp) + 255) / 256 * 256;
-    // completion counters (executor) or the grouped kernel's tile table (4 n + 1 words)
-    const size_t done = (static_cast<size_t>(n_ops) * 16 + 4 + 255) / 256 * 256;
-    return maps + ops + done;
+    const size_t probs = (static_cast<size_t>(n_ops) * sizeof(GemmArgs) + 255) / 256 * 256;
+    const size_t tab = ((static_cast<size_t>(4 * n_ops + 1)) * sizeof(int) + 255) / 256 * 256;  // the tile table
+    return maps + probs + tab;
 }
 
 static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t maps_off, size_t ops_off,
@@ -695,206 +690,37 @@ static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t 
 
 nvfp4_status nvfp4_program_build(const nvfp4_op *ops, int n_ops, void *buffer, size_t bytes, nvfp4_program *prog) {
     if (ops == nullptr || n_ops <= 0 || buffer == nullptr || prog == nullptr) return NVFP4_ERR_INVALID_ARG;
-    if (n_ops > kExecMaxOps) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (n_ops > kGroupedMaxProblems) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (bytes < nvfp4_program_bytes(n_ops)) return NVFP4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0) return NVFP4_ERR_MISALIGNED;
-    nvfp4_status st = check_device();
-    if (st != NVFP4_OK) return st;
-    {
-        // a grouped GEMM (independent GEMM ops, one epilogue, N % 128 == 0) takes the grouped
-        // kernel; its ops follow the rules of the standalone GEMM (any M)
-        const size_t maps_b = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
-        const size_t ops_b = (static_cast<size_t>(n_ops) * sizeof(ExecOp) + 255) / 256 * 256;
-        nvfp4_status gst = NVFP4_OK;
-        if (build_grouped(ops, n_ops, static_cast<uint8_t *>(buffer), 0, maps_b, maps_b + ops_b, prog, &gst)) {
-            if (gst != NVFP4_OK) return gst;
-            prog->buffer = buffer;
-            prog->bytes = bytes;
-            prog->n_ops = n_ops;
-            prog->cluster = 1;
-            prog->maps_offset = 0;
-            prog->ops_offset = maps_b;
-            prog->done_offset = maps_b + ops_b;
-            return NVFP4_OK;
-        }
-    }
-    int grid = 0;
-    if (exec_grid(kExecCluster, &grid) != cudaSuccess || grid < kExecCluster) return NVFP4_ERR_CUDA;
-    const int teams = grid / kExecCluster;
-
-    std::vector<CUtensorMap> maps(static_cast<size_t>(n_ops) * 2);
-    std::vector<ExecOp> eops(static_cast<size_t>(n_ops));
-    int next_team = 0, waits = 0;
-    // Runs of two or more independent GEMM ops (a grouped GEMM) are scheduled for throughput:
-    // when the run has at least a tile per CTA, no op splits K (a split adds an exchange and
-    // an epilogue pass per unit and buys no parallelism the run does not already have).
-    std::vector<int> run_tiles(static_cast<size_t>(n_ops), 0);
-    for (int i = 0; i < n_ops;) {
-        auto grouped = [&](int k) { return ops[k].type == NVFP4_OP_GEMM && ops[k].dep == NVFP4_DEP_NONE; };
-        if (!grouped(i)) {
-            ++i;
-            continue;
-        }
-        int j = i, tiles = 0;
-        for (; j < n_ops && grouped(j); ++j) tiles += ops[j].N / (ops[j].N % 128 == 0 ? 128 : 64);
-        if (j - i >= 2)
-            for (int k = i; k < j; ++k) run_tiles[k] = tiles;
-        i = j;
-    }
     for (int i = 0; i < n_ops; ++i) {
         const nvfp4_op &o = ops[i];
-        ExecOp &e = eops[i];
-        std::memset(&e, 0, sizeof e);
-        if (o.dep == NVFP4_DEP_PREVIOUS) e.dep = i - 1;  // op 0 has none
-        else if (o.dep == NVFP4_DEP_NONE) e.dep = -1;
-        else if (o.dep >= 1 && o.dep <= i) e.dep = o.dep - 1;
-        else return NVFP4_ERR_INVALID_ARG;  // a later op, itself, or a bad code
-        if (e.dep >= 0) {
-            eops[static_cast<size_t>(e.dep)].signal = 1;
-            ++waits;
-        }
-        if (o.type == NVFP4_OP_QUANTIZE_NORM) {
-            if (o.M <= 0 || o.K <= 0 || o.x == nullptr || o.ldx < o.K) return NVFP4_ERR_INVALID_ARG;
-            if (static_cast<int>(o.norm) < 0 || static_cast<int>(o.norm) > 4) return NVFP4_ERR_INVALID_ARG;
-            if (o.K % 16 != 0 || o.K > 16384) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-            if (o.out_codes == nullptr || o.out_sf == nullptr || !scale_ok(o.out_global_scale))
-                return NVFP4_ERR_INVALID_ARG;
-            if (!(o.eps >= 0.0f) || !std::isfinite(o.eps)) return NVFP4_ERR_INVALID_ARG;
-            if (!aligned16(o.x) || o.ldx % 8 != 0 || !aligned16(o.out_codes) || !aligned16(o.out_sf))
-                return NVFP4_ERR_MISALIGNED;
-            for (const void *pp : {o.gamma, o.beta, o.mod_scale, o.mod_shift})
-                if (pp != nullptr && !aligned16(pp)) return NVFP4_ERR_MISALIGNED;
-            e.type = kOpNorm;
-            e.units = static_cast<unsigned>(std::min(o.M, grid));  // one row per CTA at a time; each CTA signals once
-            e.norm.x = o.x;
-            e.norm.M = o.M;
-            e.norm.K = o.K;
-            e.norm.ldx = o.ldx;
-            e.norm.kind = static_cast<int>(o.norm);
-            e.norm.gamma = static_cast<const uint16_t *>(o.gamma);
-            e.norm.beta = static_cast<const uint16_t *>(o.beta);
-            e.norm.scale = static_cast<const uint16_t *>(o.mod_scale);
-            e.norm.shift = static_cast<const uint16_t *>(o.mod_shift);
-            e.norm.eps = o.eps;
-            e.norm.g = o.out_global_scale;
-            e.norm.codes = o.out_codes;
-            e.norm.sf = o.out_sf;
-            e.bpt = (o.K / 16 + 127) / 128;  // 16-element blocks per worker thread (a row on 128 threads)
-        } else if (o.type == NVFP4_OP_GEMM) {
-            st = validate_gemm(&o.A, &o.W, o.M, o.N, o.K, o.epi, o.bias, o.residual, o.ldr, o.out_bf16, o.ldo,
-                               o.out_codes, o.out_sf, o.out_global_scale);
-            if (st != NVFP4_OK) return st;
-            if (o.M <= 0 || o.M > 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-            const int k_tiles = (o.K + 255) / 256;
-            // schedule: tile width and split factor (dividing the cluster size) that finish the
-            // op in the fewest rounds with the shortest per-CTA K chain
-            double best = 1e30;
-            Schedule sc{64, 1, k_tiles, false};
-            if (run_tiles[i] >= grid) {
-                sc = finish(o.N % 128 == 0 ? 128 : 64, 1, o.K, false);
-                best = -1.0;  // fixed: skip the latency model below
-            }
-            // Latency model (us) of one round at M <= 64: A load 0.8, MMA 0.7 per k-tile,
-            // split exchange 0.8, epilogue 0.6 per pass of 128 threads over 32-column items.
-            for (int bn : {128, 64}) {
-                if (o.N % bn != 0 || best < 0.0) continue;
-                for (int s : {1, 2}) {
-                    const Schedule c = finish(bn, s, o.K, false);
-                    if (kExecCluster % c.splits != 0 || (bn / c.splits) % 32 != 0) continue;
-                    const int n_tiles = o.N / bn;
-                    const int per_round = teams * (kExecCluster / c.splits);
-                    const int rounds = (n_tiles + per_round - 1) / per_round;
-                    const int items = std::min(64, o.M) * (bn / c.splits / 32);
-                    const double cost = rounds * (0.8 + 0.7 * c.kt_per_split + (c.splits > 1 ? 0.8 : 0.0) +
-                                                  0.6 * ((items + 127) / 128)) +
-                                        (c.kt_per_split > kExecRing ? 0.3 * (c.kt_per_split - kExecRing) : 0.0) +
-                                        (bn == 64 ? 0.02 : 0.0);
-                    if (cost < best) {
-                        best = cost;
-                        sc = c;
-                    }
-                }
-            }
-            e.type = kOpGemm;
-            e.M = o.M;
-            e.N = o.N;
-            e.K = o.K;
-            e.k_atoms = (o.K + 63) / 64;
-            e.k_tiles = k_tiles;
-            e.bn = sc.block_n;
-            e.splits = sc.splits;
-            e.kt_per_split = sc.kt_per_split;
-            e.n_tiles = o.N / sc.block_n;
-            {
-                // rotate the op's first tile to the team after the previous GEMM's last one, so
-                // a run of small ops spreads over the whole grid instead of its first teams
-                const int per_team = kExecCluster / e.splits;
-                const int used = std::min(teams, (e.n_tiles + per_team - 1) / per_team);
-                e.team0 = next_team;
-                next_team = (next_team + used) % teams;
-            }
-            e.units = static_cast<unsigned>(e.n_tiles * e.splits);  // every CTA of a group signals its slice
-            e.a_box_rows = static_cast<uint32_t>((o.M + 7) / 8 * 8);
-            e.sfa = o.A.sf;
-            e.sfb = o.W.sf;
-            e.alpha = o.A.global_scale * o.W.global_scale;
-            e.epi = kernel_epi(o.epi);
-            e.out_rotate = epi_rotates(o.epi);
-            e.bias = static_cast<const uint16_t *>(o.bias);
-            e.residual = static_cast<const uint16_t *>(o.residual);
-            e.ldr = o.ldr;
-            e.out = static_cast<uint16_t *>(o.out_bf16);
-            e.ldo = o.ldo;
-            e.out_codes = o.out_codes;
-            e.out_sf = o.out_sf;
-            e.g_out = o.out_global_scale;
-            e.tm_a = 2 * i;
-            e.tm_b = 2 * i + 1;
-            if (getenv("NVFP4_EXEC_DEBUG") != nullptr)
-                fprintf(stderr, "nvfp4 program op %d: GEMM %dx%dx%d block_n %d splits %d k_tiles/split %d tiles %d (grid %d)\n",
-                        i, o.M, o.N, o.K, e.bn, e.splits, e.kt_per_split, e.n_tiles, grid);
-            if (!make_code_map(&maps[2 * i], o.A.codes, o.M, o.K / 2, static_cast<int>(e.a_box_rows)) ||
-                !make_code_map(&maps[2 * i + 1], o.W.codes, o.N, o.K / 2, e.bn))
-                return NVFP4_ERR_CUDA;
-        } else {
-            return NVFP4_ERR_INVALID_ARG;
-        }
+        if (o.type != NVFP4_OP_GEMM) return NVFP4_ERR_UNSUPPORTED_SHAPE;  // norm ops: nvfp4_quantize_norm
+        if (o.dep != NVFP4_DEP_NONE) return NVFP4_ERR_UNSUPPORTED_SHAPE;  // dependent ops: a launch chain
+        if (o.epi != ops[0].epi || o.N % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     }
-    const size_t maps_bytes = maps.size() * sizeof(CUtensorMap);
-    const size_t ops_bytes = (eops.size() * sizeof(ExecOp) + 255) / 256 * 256;
-    uint8_t *base = static_cast<uint8_t *>(buffer);
-    if (cudaMemcpy(base, maps.data(), maps_bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(base + maps_bytes, eops.data(), eops.size() * sizeof(ExecOp), cudaMemcpyHostToDevice) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    const size_t maps_b = static_cast<size_t>(n_ops) * 2 * sizeof(CUtensorMap);
+    const size_t probs_b = (static_cast<size_t>(n_ops) * sizeof(GemmArgs) + 255) / 256 * 256;
+    nvfp4_status gst = NVFP4_OK;
+    build_grouped(ops, n_ops, static_cast<uint8_t *>(buffer), 0, maps_b, maps_b + probs_b, prog, &gst);
+    if (gst != NVFP4_OK) return gst;
     prog->buffer = buffer;
     prog->bytes = bytes;
     prog->n_ops = n_ops;
-    prog->grid = grid;
-    prog->cluster = kExecCluster;
+    prog->cluster = 1;
     prog->maps_offset = 0;
-    prog->ops_offset = maps_bytes;
-    prog->done_offset = maps_bytes + ops_bytes;
-    prog->waits = waits;
-    prog->kind = 0;
-    prog->epi = 0;
-    prog->tiles = 0;
+    prog->ops_offset = maps_b;
+    prog->done_offset = maps_b + probs_b;
     return NVFP4_OK;
 }
 
-// A program of independent GEMM ops with one epilogue kind and N % 128 == 0 (a grouped GEMM)
-// runs on the grouped persistent kernel instead of the executor: the same results (one split
-// per tile, as the executor's grouped schedule), with the weight stream kept running across
-// problem boundaries.  Writes the problems' GemmArgs over the op area, their tensor maps and
-// the tile table; returns false if the program is not such a group.
+// A grouped GEMM (independent GEMM ops, one epilogue kind, N % 128 == 0) for the grouped
+// persistent kernel: one split per tile, the weight stream kept running across problem
+// boundaries.  Writes the problems' GemmArgs, their tensor maps and the tile table.
 static bool build_grouped(const nvfp4_op *ops, int n_ops, uint8_t *base, size_t maps_off, size_t ops_off,
                           size_t tab_off, nvfp4_program *prog, nvfp4_status *st) {
-    if (n_ops < 2 || n_ops > kGroupedMaxProblems) return false;
-    for (int i = 0; i < n_ops; ++i) {
-        const nvfp4_op &o = ops[i];
-        if (o.type != NVFP4_OP_GEMM || o.dep != NVFP4_DEP_NONE || o.epi != ops[0].epi || o.N % 128 != 0)
-            return false;
-    }
-    static_assert(sizeof(GemmArgs) <= sizeof(ExecOp), "the op area holds the grouped problems");
     for (int i = 0; i < n_ops; ++i) {
         const nvfp4_op &o = ops[i];
         *st = validate_gemm(&o.A, &o.W, o.M, o.N, o.K, o.epi, o.bias, o.residual, o.ldr, o.out_bf16, o.ldo,
@@ -986,20 +812,7 @@ nvfp4_status nvfp4_program_run(const nvfp4_program *prog, nvfp4_stream_t stream)
         if (e == cudaSuccess) e = cudaGetLastError();
         return from_cuda(e);
     }
-    ExecParams p;
-    p.ops = reinterpret_cast<const ExecOp *>(base + prog->ops_offset);
-    p.maps = reinterpret_cast<const CUtensorMap *>(base + prog->maps_offset);
-    p.done = reinterpret_cast<unsigned int *>(base + prog->done_offset);
-    p.n_ops = prog->n_ops;
-    p.cluster = prog->cluster;
-    if (device_status_address(&p.status) != cudaSuccess) return NVFP4_ERR_CUDA;
-    p.trace = (g_trace != nullptr && g_trace_words >= static_cast<size_t>(prog->n_ops) * prog->grid * 8) ? g_trace
-                                                                                                          : nullptr;
-    cudaError_t e = prog->waits > 0 ? cudaMemsetAsync(p.done, 0, static_cast<size_t>(prog->n_ops) * 4, stream)
-                                     : cudaSuccess;
-    if (e == cudaSuccess) e = exec_launch(p, prog->grid, stream);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    return from_cuda(e);
+    return NVFP4_ERR_INVALID_ARG;  // not a program this library built
 }
 
 }  // extern "C"

@@ -1,5 +1,5 @@
-// epilogue.cuh — the fused GEMM epilogue, shared by the standalone GEMM and the layer
-// executor: v = acc * gA * gW (+ bias[n]) (+ residual[m, n]), then bf16 out, or tanh-GELU /
+// epilogue.cuh — the fused GEMM epilogue, shared by the GEMM kernels (small-M, persistent,
+// grouped): v = acc * gA * gW (+ bias[n]) (+ residual[m, n]), then bf16 out, or tanh-GELU /
 // GeGLU re-quantized to NVFP4 ("GROOT N1.7 update: Thor NVFP4 + FA4 performance tier",
 // §What is in the tier; "Pi0.5 Thor NVFP4 End-to-End Results", §Half-Width Fused GeGLU
 // Epilogue and §Fused GeGLU FFN in the Decoder: GELU on the fp32 accumulator, gate/up on

@@ -1,5 +1,5 @@
-// norm_row.cuh — one row of the norm -> NVFP4 front-end, shared by the standalone kernel
-// and the layer executor (both must produce the same bytes).
+// norm_row.cuh — one row of the norm -> NVFP4 front-end (the norm_quant_kernel launches: a
+// warp per row for many rows, four warps per row for few).
 //
 // One row is owned by TPR threads.  Each thread loads whole 16-element blocks with 16-byte
 // loads (block b of a row goes to thread b % TPR), keeps them in registers, reduces the row
@@ -28,8 +28,7 @@ namespace nvfp4 {
 enum { kNone = 0, kLayerNorm = 1, kRmsNorm = 2, kAdaLN = 3, kAdaRms = 4 };
 
 // Sum of v over the TPR threads of a row (t = the thread's index among them).  TPR = 128:
-// the four warps meet on named barrier 1 (they are the whole CTA of the standalone kernel, or
-// the four worker warps of the layer executor), with `red` four doubles of shared memory.
+// the CTA's four warps meet on named barrier 1, with `red` four doubles of shared memory.
 template <int TPR>
 __device__ __forceinline__ double row_sum(double v, double *red, int t) {
 #pragma unroll
@@ -77,7 +76,7 @@ __device__ __forceinline__ void norm_row(const NormArgs &p, int row, int t, doub
     constexpr int kWords = F32 ? 16 : 8;  // 32-bit words per 16-element block
     constexpr bool kParamRegs = BPT <= 4;
     // Every field is read once into a local: the byte stores below may alias any memory as
-    // far as the compiler knows, and `p` may live in global memory (executor programs).
+    // far as the compiler knows.
     const int M = p.M, K = p.K, ldx = p.ldx, kind = p.kind;
     const void *const x = p.x;
     const float eps = p.eps, g_arg = p.g;

@@ -16,8 +16,7 @@ enum : uint32_t {
     kStatusTimeoutEmpty = 2,    // producer waited too long for a free stage
     kStatusTimeoutAccum = 3,    // epilogue waited too long for the accumulator
     kStatusTimeoutDrain = 4,    // teardown waited too long for copies / MMAs in flight
-    kStatusTimeoutOp = 5,       // executor: an op's input never completed
-    kStatusTimeoutPeer = 6,     // executor: a split-K partner never delivered / released
+    kStatusTimeoutPeer = 6,     // a split-K partner never delivered its partial
 };
 
 // Wall-clock bound of one wait (ns).  Far above any legitimate wait of these kernels.

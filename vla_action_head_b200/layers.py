@@ -82,18 +82,6 @@ class DiTLayer:
                    workspace=self.ws)
         return y
 
-    def ops(self, x, context, y):
-        """The same forward as a list of executor ops."""
-        return [
-            nvfp4.op_norm(x, self.a1, "adaln", scale=self.ada_scale, shift=self.ada_shift, eps=1e-6),
-            nvfp4.op_gemm(self.a1, self.qkv.w, "bias", bias=self.qkv.bias, out=self.qkv_out),
-            nvfp4.op_norm(context, self.ctx_q, "none"),
-            nvfp4.op_gemm(self.ctx_q, self.o.w, "bias_residual", bias=self.o.bias, residual=x, out=self.h),
-            nvfp4.op_norm(self.h, self.a2, "layernorm", gamma=self.ln_gamma, beta=self.ln_beta, eps=1e-5),
-            nvfp4.op_gemm(self.a2, self.up.w, "bias_gelu", bias=self.up.bias, out=self.u),
-            nvfp4.op_gemm(self.u, self.down.w, "bias_residual", bias=self.down.bias, residual=self.h, out=y),
-        ]
-
     launches = 7
 
 
@@ -132,17 +120,6 @@ class ActionExpertLayer:
         nvfp4.gemm(self.a2, self.gate_up.w, "geglu", out=self.u, workspace=self.ws)
         nvfp4.gemm(self.u, self.down.w, "residual", residual=self.h, out=y, workspace=self.ws)
         return y
-
-    def ops(self, x, context, y):
-        return [
-            nvfp4.op_norm(x, self.a1, "adarms", scale=self.scale1, eps=1e-6),
-            nvfp4.op_gemm(self.a1, self.qkv.w, "none", out=self.qkv_out),
-            nvfp4.op_norm(context, self.ctx_q, "none"),
-            nvfp4.op_gemm(self.ctx_q, self.o.w, "residual", residual=x, out=self.h),
-            nvfp4.op_norm(self.h, self.a2, "adarms", scale=self.scale2, eps=1e-6),
-            nvfp4.op_gemm(self.a2, self.gate_up.w, "geglu", out=self.u),
-            nvfp4.op_gemm(self.u, self.down.w, "residual", residual=self.h, out=y),
-        ]
 
     launches = 7
 

@@ -315,37 +315,13 @@ def device_status():
     _check("nvfp4_get_device_status", lib().nvfp4_get_device_status(_stream()))
 
 
-# ---- layer executor ----------------------------------------------------------------------
-def _dep(dep):
-    """"previous" (the op before), None (no wait) or the index of an earlier op."""
-    if dep == "previous":
-        return 0
-    if dep is None:
-        return -1
-    if isinstance(dep, int) and dep >= 0:
-        return dep + 1
-    raise ValueError(f"dep must be 'previous', None or an op index, got {dep!r}")
-
-
-def op_norm(x, out: NVFP4Tensor, kind="none", gamma=None, beta=None, scale=None, shift=None, eps=1e-6,
-            dep="previous"):
-    """A norm -> FP4 op of a program (bf16 x [M, K] -> out); `dep` names the op it waits for."""
-    M, K = x.shape
-    op = _Op(type=0, M=M, N=0, K=K, x=x.data_ptr(), ldx=x.stride(0), norm=NORM[kind],
-             gamma=_ptr(gamma), beta=_ptr(beta), mod_scale=_ptr(scale), mod_shift=_ptr(shift), eps=eps,
-             out_codes=out.codes.data_ptr(), out_sf=out.sf.data_ptr(), out_global_scale=out.global_scale,
-             dep=_dep(dep))
-    op.keep = (x, out, gamma, beta, scale, shift)  # the program only holds raw pointers
-    return op
-
-
-def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None, out_global_scale=1.0,
-            dep="previous"):
-    """A GEMM op of a program; `out` is bf16 [M, N] or, for FP4 epilogues, an NVFP4Tensor;
-    `dep` names the op whose results it reads ("previous", None or an op index)."""
+# ---- grouped GEMM ------------------------------------------------------------------------
+def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None, out=None, out_global_scale=1.0):
+    """One problem of a grouped GEMM; `out` is bf16 [M, N] or, for FP4 epilogues, an
+    NVFP4Tensor.  Its inputs are ready before the launch (no dependency between problems)."""
     e = EPI[epi]
     op = _Op(type=1, M=a.rows, N=w.rows, K=a.K, A=a.c(), W=w.c(), epi=e, bias=_ptr(bias),
-             residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0, dep=_dep(dep))
+             residual=_ptr(residual), ldr=residual.stride(0) if residual is not None else 0, dep=-1)
     if e in (4, 5, 6, 7):
         op.out_codes, op.out_sf, op.out_global_scale = out.codes.data_ptr(), out.sf.data_ptr(), out_global_scale
     else:
@@ -355,8 +331,8 @@ def op_gemm(a: NVFP4Tensor, w: NVFP4Tensor, epi="none", bias=None, residual=None
 
 
 class Program:
-    """A built program of ops (device buffer owned here); run() makes one launch.  It keeps
-    the ops, and through them every tensor they name, alive."""
+    """A built grouped GEMM of ops (nvfp4_program_build; device buffer owned here); run()
+    makes one launch.  It keeps the ops, and through them every tensor they name, alive."""
 
     def __init__(self, ops, device="cuda"):
         self.ops = list(ops)
@@ -374,15 +350,24 @@ class Program:
         _check("nvfp4_program_run", lib().nvfp4_program_run(C.byref(self.prog), _stream()))
 
 
-class GroupedGemm(Program):
-    """A grouped NVFP4 GEMM: independent problems (a_g, w_g, out_g[, bias_g]) of M <= 64 rows,
-    all run by one launch that streams every problem's weights back to back with no wait
-    between problems.  Problems may differ in N and K; each takes the same epilogue kind."""
+class GroupedGemm:
+    """A grouped NVFP4 GEMM: independent problems (a_g, w_g, out_g[, bias_g]), each taking
+    the same epilogue kind; problems may differ in M, N and K.  When every N is a multiple of
+    128 one launch of the grouped kernel runs them all, streaming the problems' weights back
+    to back (`prog`); otherwise the problems run as standalone nvfp4_gemm launches
+    (`prog` is None)."""
 
-    def __init__(self, problems, epi="none", device="cuda"):
-        ops = []
-        for pr in problems:
-            a, w, out = pr[0], pr[1], pr[2]
-            bias = pr[3] if len(pr) > 3 else None
-            ops.append(op_gemm(a, w, epi, bias=bias, out=out, dep=None))
-        super().__init__(ops, device=device)
+    def __init__(self, problems, epi="none", device="cuda", workspace: Optional["Workspace"] = None):
+        self.problems = [(pr[0], pr[1], pr[2], pr[3] if len(pr) > 3 else None) for pr in problems]
+        self.epi = epi
+        self.workspace = workspace
+        self.prog = None
+        if all(w.rows % 128 == 0 for _, w, _, _ in self.problems):
+            self.prog = Program([op_gemm(a, w, epi, bias=b, out=o) for a, w, o, b in self.problems], device=device)
+
+    def run(self):
+        if self.prog is not None:
+            self.prog.run()
+            return
+        for a, w, o, b in self.problems:
+            gemm(a, w, self.epi, bias=b, out=o, workspace=self.workspace)
