@@ -76,7 +76,8 @@ def parse():
     ap.add_argument("--soak-steps", type=int, default=200,
                     help="untimed steps while the clock sampler starts (0 for profiling runs)")
     ap.add_argument("--profile-case", default=None,
-                    help="run one small case for ncu (dit-gemms | prefill-gemms | grouped | norm) and exit")
+                    help="run one small case for ncu (dit-gemms | prefill-gemms | grouped | norm) or the traced "
+                         "DiT launch chain (dit-chain-trace), and exit")
     return ap.parse_args()
 
 
@@ -544,6 +545,65 @@ def profile_case(name):
         grp = nvfp4.GroupedGemm([(ctxq, l.w, outs[g]) for g, l in enumerate(lins)])
         for _ in range(3):
             grp.run()
+    elif name == "dit-chain-trace":
+        # per-CTA timestamps of the launch chain: a CUDA graph of 8 DiT layers (distinct weights)
+        # with nvfp4_set_gemm_trace; prints, per GEMM launch, the medians over its CTAs of the
+        # stamps and the gap from the previous launch's last exit to this one's first stage
+        import numpy as np
+
+        from vla_action_head_b200 import synth
+        L = nvfp4.lib()
+        R, (M, H, F) = 8, (DIT["M"], DIT["H"], DIT["F"])
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            wsp = nvfp4.Workspace("cuda")
+            lays = [layers.DiTLayer(**DIT, layer=i, ws=wsp) for i in range(R)]
+            x0 = synth.bf16_normal_torch(synth.seed_of(2, synth.X), (M, H), device="cuda")
+            ctx = synth.bf16_normal_torch(synth.seed_of(2, synth.CONTEXT), (M, H), device="cuda")
+            buf = [x0.clone(), torch.empty_like(x0)]
+
+            def fwd():
+                for i, lay in enumerate(lays):
+                    lay.forward(buf[i % 2], ctx, buf[(i + 1) % 2])
+            fwd()
+        torch.cuda.synchronize()
+        gemms = [("qkv", 3 * H, H, "bias"), ("o", H, H, "bias_residual"), ("up", F, H, "bias_gelu"),
+                 ("down", H, F, "bias_residual")]
+        words = [int(L.nvfp4_gemm_trace_words(M, N, K, nvfp4.EPI[e])) for _, N, K, e in gemms]
+        tr = torch.zeros(sum(words) * R, dtype=torch.int64, device="cuda")
+        L.nvfp4_set_gemm_trace(tr.data_ptr(), tr.numel())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fwd()
+        L.nvfp4_set_gemm_trace(None, 0)
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        tr.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        t = tr.cpu().numpy().astype(np.float64)
+        t0 = t[t > 0].min()
+        off, prev_exit = 0, None
+        labels = [(0, "entry"), (3, "first stage"), (4, "last MMA"), (5, "acc ready"), (1, "epilogue done"),
+                  (6, "exit")]
+        print("per launch, us from the first stamp (median over CTAs / max)")
+        for k in range(4 * R):
+            n = words[k % 4]
+            blk = t[off:off + n].reshape(-1, 8)
+            off += n
+            rel = (blk - t0) / 1e3
+            cols = []
+            for c, lab in labels:
+                v = rel[:, c][blk[:, c] > 0]
+                if len(v):
+                    cols.append(f"{lab} {np.median(v):7.2f}/{v.max():7.2f}")
+            first = rel[:, 3][blk[:, 3] > 0]
+            gap = "" if prev_exit is None else f" | gap {np.median(first) - prev_exit:5.2f}"
+            prev_exit = rel[:, 6][blk[:, 6] > 0].max()
+            print(f"{gemms[k % 4][0]:5s} L{k // 4} ({n // 8} CTAs) " + " | ".join(cols) + gap)
+        del g
     elif name == "norm":
         x = torch.randn(968, 2048, device="cuda").to(torch.bfloat16)
         g = torch.ones(2048, device="cuda").to(torch.bfloat16)

@@ -169,6 +169,10 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * gemm_grouped.cu). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
+/* Trace words one nvfp4_gemm launch of this shape and epilogue takes under the default
+ * schedule (8 per CTA of its grid); 0 for a shape nvfp4_gemm does not accept. */
+size_t nvfp4_gemm_trace_words(int M, int N, int K, nvfp4_epilogue epi);
+
 /* ---- norm -> NVFP4 quantize (fused front-end) --------------------------------------- */
 
 /* Per row of x [M, K] (leading dimension ldx, bf16 or fp32): the norm `kind`, then the

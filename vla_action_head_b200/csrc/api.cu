@@ -494,6 +494,18 @@ size_t nvfp4_gemm_workspace_bytes_ex(int M, int N, int K, int block_n, int split
     return workspace_for(M, N, sc);
 }
 
+size_t nvfp4_gemm_trace_words(int M, int N, int K, nvfp4_epilogue epi) {
+    if (M <= 0 || N <= 0 || K <= 0 || N % 64 != 0) return 0;
+    if (static_cast<int>(epi) < 0 || static_cast<int>(epi) > 7) return 0;
+    const size_t m_tiles = static_cast<size_t>((M + 127) / 128);
+    if (M > 128) {
+        const ManyRows many = choose_persistent(M, N, K);
+        if (many.block_n > 0) return 8 * m_tiles * static_cast<size_t>(N / many.block_n) * many.splits;
+    }
+    const Schedule sc = choose(M, N, K, kernel_epi(epi) == kEpiBiasGelu || kernel_epi(epi) == kEpiGeglu);
+    return 8 * m_tiles * static_cast<size_t>(N / sc.block_n) * sc.splits;
+}
+
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
     g_trace = buf;
     g_trace_words = buf ? words : 0;

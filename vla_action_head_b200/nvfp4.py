@@ -79,6 +79,7 @@ def lib():
             "nvfp4_gemm_workspace_bytes_ex": (SZ, [I, I, I, I, I]),
             "nvfp4_get_device_status": (I, [P]),
             "nvfp4_set_gemm_trace": (I, [P, SZ]),
+            "nvfp4_gemm_trace_words": (SZ, [I, I, I, I]),
             "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
             "nvfp4_residual_quantize_norm": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, P, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
@@ -354,20 +355,22 @@ class GroupedGemm:
     """A grouped NVFP4 GEMM: independent problems (a_g, w_g, out_g[, bias_g]), each taking
     the same epilogue kind; problems may differ in M, N and K.  When every N is a multiple of
     128 one launch of the grouped kernel runs them all, streaming the problems' weights back
-    to back (`prog`); otherwise the problems run as standalone nvfp4_gemm launches
-    (`prog` is None)."""
+    to back (`program`, whose built handle is `prog`); otherwise the problems run as standalone
+    nvfp4_gemm launches (`program` and `prog` are None)."""
 
     def __init__(self, problems, epi="none", device="cuda", workspace: Optional["Workspace"] = None):
         self.problems = [(pr[0], pr[1], pr[2], pr[3] if len(pr) > 3 else None) for pr in problems]
         self.epi = epi
         self.workspace = workspace
-        self.prog = None
+        self.program = self.prog = None
         if all(w.rows % 128 == 0 for _, w, _, _ in self.problems):
-            self.prog = Program([op_gemm(a, w, epi, bias=b, out=o) for a, w, o, b in self.problems], device=device)
+            self.program = Program([op_gemm(a, w, epi, bias=b, out=o) for a, w, o, b in self.problems],
+                                   device=device)
+            self.prog = self.program.prog
 
     def run(self):
-        if self.prog is not None:
-            self.prog.run()
+        if self.program is not None:
+            self.program.run()
             return
         for a, w, o, b in self.problems:
             gemm(a, w, self.epi, bias=b, out=o, workspace=self.workspace)
