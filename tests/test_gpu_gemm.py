@@ -1,7 +1,7 @@
 """GPU parity of the block-scaled NVFP4 GEMM and its fused epilogues against the oracle.
 
 Operands are quantized by the oracle and uploaded, so the GEMM is checked alone: bf16
-outputs meet the spec bar (relative error <= 1e-2 where |ref| > 1e-2 max|ref|,
+outputs meet the acceptance bar (relative error <= 1e-2 where |ref| > 1e-2 max|ref|,
 cosine >= 0.99999); FP4 outputs meet the boundary-only mismatch bar in parity.py.  Every
 tile width (64/128/256) and several split-K factors are pinned explicitly, over shapes
 that span several tiles and ragged M / K tails."""

@@ -1,6 +1,6 @@
 """GPU parity of the norm -> NVFP4 front-end and the weight quantizer against the oracle.
 
-Encodings are compared byte for byte.  The spec bar allows fused-norm code
+Encodings are compared byte for byte.  The acceptance bar allows fused-norm code
 mismatches only within one fp32 ulp of a rounding boundary, at most 1e-4 of the elements;
 the kernel's fp64 row statistics make them identical in practice, which is asserted too
 where it holds by construction (plain quantizer, weights)."""
