@@ -586,8 +586,8 @@ def profile_case(name):
         t = tr.cpu().numpy().astype(np.float64)
         t0 = t[t > 0].min()
         off, prev_exit = 0, None
-        labels = [(0, "entry"), (3, "first stage"), (4, "last MMA"), (5, "acc ready"), (1, "epilogue done"),
-                  (6, "exit")]
+        labels = [(0, "entry"), (3, "first stage"), (4, "last MMA"), (5, "acc ready"), (7, "partials in"),
+                  (1, "epilogue done"), (6, "exit")]
         print("per launch, us from the first stamp (median over CTAs / max)")
         for k in range(4 * R):
             n = words[k % 4]

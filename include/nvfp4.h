@@ -288,6 +288,10 @@ nvfp4_status nvfp4_quantize_weight_ex(const void *w_bf16, int N, int K, int ldw,
  *   workspace: >= nvfp4_gemm_workspace_bytes(M, N, K) bytes, zeroed once at allocation;
  *   used by one GEMM at a time (GEMMs that may run concurrently, e.g. on two streams, each
  *   need their own).
+ * Launch overlap: the kernel starts while the previous kernel of `stream` still runs when
+ * that kernel is one of this library's (programmatic dependent launch), and may read W, its
+ * scales and bias before waiting for it; A, its scales and residual are read after.  So W
+ * and bias must not be written by the library call immediately before on the same stream.
  * Constraints: M >= 0 (0 is a no-op), K % 32 == 0 (TMA 16-byte rows; a K % 64 tail is
  * covered by the zero scale padding, [PI05] §Encoder Attention QKV NVFP4 + Scale-Factor
  * Zero-Init), N % 64 == 0. */

@@ -339,7 +339,6 @@ nvfp4_status gemm_impl(const nvfp4_tensor *A, const nvfp4_tensor *W, int M, int 
     p.out_sf = out_sf;
     p.g_out = out_global_scale;
     if (need > 0) {
-        const size_t tiles = static_cast<size_t>((M + 127) / 128) * p.n_tiles;
         p.tickets = static_cast<uint32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + kTicketRegion);
     }

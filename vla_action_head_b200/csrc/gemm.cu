@@ -402,7 +402,6 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             // threads need to meet (every one reads the accumulator-valid word below)
             if constexpr (!S::kSepRed) cluster_sync_all();
             else __syncthreads();
-            if (trace != nullptr && threadIdx.x == 64) trace[7] = globaltimer_ns();
             const bool acc_ok = misc[3] != 0u;
             if (warp >= 2 && acc_ok) {
                 const int q = warp & 3;
@@ -427,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
             }
             __syncwarp();
             cluster_sync_all();  // (3)
+            if (trace != nullptr && threadIdx.x == 64) trace[7] = globaltimer_ns();
             if (!acc_ok) return;
             for (int item = e;; item += kThreads) {
                 const int li = item / kChunks, ch = item % kChunks;
