@@ -41,8 +41,8 @@ DIT = dict(M=41, H=1536, F=6144)
 # of the kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                 "sha256": "17b02ebe159326c26105abd88f5fe361ab7e1d70e67ca2be63b934508da5e1ed",
-                 "bytes": 4213440},  # mean of the 4 DiT GEMM launches (case dit-gemms)
+                 "sha256": "bbb01126a6ef704b83f71c00539d073b176b9c6cef1bb89748375d59d971902f",
+                 "bytes": 4213568},  # mean of the 4 DiT GEMM launches (case dit-gemms)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
                         "sha256": "054c613d536e86440b88b4be1cb5a5eee56c8a38970de0a92c7033de96f37689",
                         "bytes": 38966528},  # the gate/up launch of case prefill-gemms
@@ -1051,6 +1051,25 @@ def side_measurements(stack, wsp, stream, dev, pk, pk_kind):
                                                "unit": "GB/s", "frac": round(gbs_t / pk["hbm_gbs"], 4),
                                                "bytes": tb, "peak_kind": pk_kind},
                                   "l2": "48 distinct weight copies (L2-warm: 3.6 MB in total)"}
+    # ---- the block-scaled MMA's issue rate on one SM (nvfp4_mma_rate): the ceiling of the
+    # GEMM kernels' MMA phases; cycles per K step of 256 (4 MMAs of 128 x n x 64), MMAs alone
+    # (mode 0) and with the step's scale-atom copies from the same thread (mode 1) ----
+    torch.cuda.synchronize()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    rate = {}
+    out["mma_rate"] = rate
+    with clocked("mma_rate"):
+        for n in (64, 128, 256):
+            _, c0 = nvfp4.mma_rate(n, 0, 256)
+            _, c1 = nvfp4.mma_rate(n, 1, 256)
+            flop_per_cycle = 4 * 2.0 * 128 * n * 64 / c0
+            rate[f"n{n}"] = {"mma_cycles_per_kstep": round(c0, 1), "copies_and_mma_cycles_per_kstep": round(c1, 1),
+                             "fp4_flop_per_sm_cycle": round(flop_per_cycle, 1)}
+    max_mhz = rate["clocks"].get("sm_max_mhz") or 0.0
+    rate["implied_fp4_tflops_at_max_clock"] = round(rate["n256"]["fp4_flop_per_sm_cycle"] * sms * max_mhz * 1e6 / 1e12,
+                                                    1)
+    rate["note"] = ("one CTA, one issuing thread, operands resident in shared memory; the implied figure is the "
+                    "256-wide MMA rate x SMs x the maximum SM clock, context for the FP4 peak, not its denominator")
     torch.cuda.synchronize()
     nvfp4.device_status()
     return out

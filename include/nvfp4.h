@@ -169,6 +169,18 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream);
  * gemm_grouped.cu). */
 nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words);
 
+/* Diagnostics: the issue rate of the block-scaled MMA on one SM.  One CTA, one issuing
+ * thread, operands resident in shared memory, accumulator and scale factors in tensor
+ * memory, runs `ksteps` K steps of 256, each four tcgen05.mma kind::mxf4nvf4 block16
+ * (M = 128, N = n, K = 64) -- mode 0 -- or each its scale-atom copies (tcgen05.cp: 4 for A,
+ * 4 per 128-row group of W) followed by its four MMAs -- mode 1.  Writes SM clock cycles
+ * per K step until the last instruction was issued (*issue_cycles) and until all of them
+ * completed (*complete_cycles; host pointers).  n: 64, 128 or 256; mode 0 or 1;
+ * 1 <= ksteps <= 4096 (else NVFP4_ERR_INVALID_ARG).  Uses 512 tensor-memory columns and
+ * ~57 KB of shared memory on one SM; synchronises the device.  The data are meaningless;
+ * only the cycle counts are. */
+nvfp4_status nvfp4_mma_rate(int n, int mode, int ksteps, double *issue_cycles, double *complete_cycles);
+
 /* Trace words one nvfp4_gemm launch of this shape and epilogue takes under the default
  * schedule (8 per CTA of its grid); 0 for a shape nvfp4_gemm does not accept. */
 size_t nvfp4_gemm_trace_words(int M, int N, int K, nvfp4_epilogue epi);

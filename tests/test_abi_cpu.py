@@ -92,6 +92,13 @@ def test_gemm_validation(L):
     assert call() in (5, 6)
 
 
+def test_mma_rate_validation(L):
+    out1, out2 = C.c_double(), C.c_double()
+    for n, mode, ksteps in ((96, 0, 64), (64, 2, 64), (128, 0, 0), (256, 1, 4097)):
+        assert L.nvfp4_mma_rate(n, mode, ksteps, C.byref(out1), C.byref(out2)) == 1
+    assert L.nvfp4_mma_rate(64, 0, 64, None, C.byref(out2)) == 1
+
+
 def test_norm_and_weight_validation(L):
     q = L.nvfp4_quantize_norm
     x, c, s = C.c_void_p(0x1000), C.c_void_p(0x2000), C.c_void_p(0x4000)

@@ -279,3 +279,18 @@ def test_split_k_wait_expires_and_context_survives(orc):
     torch.cuda.synchronize()
     nvfp4.device_status()
     check_gemm_bf16(got, ref["v"], what=("after timeout", M, N, K))
+
+
+def test_mma_rate_diagnostic():
+    """The MMA issue-rate diagnostic (nvfp4_mma_rate) runs at every width and both modes, its
+    completion count is at least its issue count, the scale copies add cycles (mode 1 over
+    mode 0), and a 256-wide MMA is not cheaper than a 64-wide one."""
+    rates = {}
+    for n in (64, 128, 256):
+        for mode in (0, 1):
+            issue, done = nvfp4.mma_rate(n, mode, 64)
+            assert 10.0 < issue <= done < 1e6, (n, mode, issue, done)
+            rates[n, mode] = done
+    for n in (64, 128, 256):
+        assert rates[n, 1] > rates[n, 0]
+    assert rates[256, 0] >= rates[64, 0]

@@ -5,7 +5,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["api.cu", "gemm.cu", "gemm_persistent.cu", "gemm_grouped.cu", "norm_quant.cu"]
+SOURCES = ["api.cu", "gemm.cu", "gemm_persistent.cu", "gemm_grouped.cu", "norm_quant.cu", "mma_rate.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-Xcompiler", "-Wall"]

@@ -17,6 +17,11 @@
 #include "gemm.h"
 #include "norm.h"
 
+namespace nvfp4 {
+// mma_rate.cu: one CTA issues `ksteps` K steps of block-scaled MMAs (mode 0) or of scale
+// copies + MMAs (mode 1) at width n; out = issue cycles, completion cycles, timeout flag.
+cudaError_t run_mma_rate(int n, int mode, int ksteps, unsigned long long out[3]);
+}  // namespace nvfp4
 
 using namespace nvfp4;
 
@@ -509,6 +514,21 @@ nvfp4_status nvfp4_set_gemm_trace(unsigned long long *buf, size_t words) {
     g_trace = buf;
     g_trace_words = buf ? words : 0;
     g_trace_cursor = 0;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_mma_rate(int n, int mode, int ksteps, double *issue_cycles, double *complete_cycles) {
+    if ((n != 64 && n != 128 && n != 256) || (mode != 0 && mode != 1) || ksteps < 1 || ksteps > 4096 ||
+        issue_cycles == nullptr || complete_cycles == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    unsigned long long out[3] = {0, 0, 0};
+    const cudaError_t e = run_mma_rate(n, mode, ksteps, out);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (out[2] != 0) return NVFP4_ERR_TIMEOUT;
+    *issue_cycles = static_cast<double>(out[0]) / ksteps;
+    *complete_cycles = static_cast<double>(out[1]) / ksteps;
     return NVFP4_OK;
 }
 

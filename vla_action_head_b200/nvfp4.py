@@ -80,6 +80,7 @@ def lib():
             "nvfp4_get_device_status": (I, [P]),
             "nvfp4_set_gemm_trace": (I, [P, SZ]),
             "nvfp4_gemm_trace_words": (SZ, [I, I, I, I]),
+            "nvfp4_mma_rate": (I, [I, I, I, P, P]),
             "nvfp4_quantize_norm": (I, [P, I, I, I, I, I, P, P, P, P, F, F, P, P, P]),
             "nvfp4_residual_quantize_norm": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, F, F, P, P, P, P]),
             "nvfp4_norm_f32": (I, [P, I, I, I, I, I, P, P, P, P, F, P, P]),
@@ -314,6 +315,14 @@ def probe():
 def device_status():
     """Raises NVFP4Error(TIMEOUT) if a kernel's bounded wait expired since the last check."""
     _check("nvfp4_get_device_status", lib().nvfp4_get_device_status(_stream()))
+
+
+def mma_rate(n=256, mode=0, ksteps=64):
+    """Diagnostics: SM cycles per K step of 256 (four block-scaled MMAs of 128 x n x 64; mode 1
+    adds the step's scale-atom copies from the same thread), as (issued, completed)."""
+    issue, done = C.c_double(), C.c_double()
+    _check("nvfp4_mma_rate", lib().nvfp4_mma_rate(n, mode, ksteps, C.byref(issue), C.byref(done)))
+    return issue.value, done.value
 
 
 # ---- grouped GEMM ------------------------------------------------------------------------
