@@ -88,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // ---------------------------------------------------------------------------------------
 // TMA: 2-D tiled load (tensor map in param space) and 1-D bulk load, both completing on an
-// mbarrier by transaction bytes.  No multicast: every CTA fetches its own tiles.
+// mbarrier by transaction bytes.  Every CTA fetches its own tiles; no load is shared across a cluster.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y,
                                             uint32_t bar, uint64_t policy) {
     asm volatile(
