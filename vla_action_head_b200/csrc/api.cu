@@ -55,16 +55,21 @@ nvfp4_status from_cuda(cudaError_t e) {
     return NVFP4_ERR_CUDA;
 }
 
+// The driver's tensor-map encoder, looked up once (host threads racing on the first call
+// each look it up and store the same pointer).
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+    if (f == nullptr) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            fn.store(f, std::memory_order_release);
+        }
     }
-    return fn;
+    return f;
 }
 
 // 2-D uint8 view [rows, row_bytes] of FP4 codes, box 128 bytes x box_rows, 128-byte swizzle.
@@ -95,22 +100,28 @@ constexpr int kMaxClusterSplits = 8;  // portable cluster size
 
 // Device address of the library's status word on the current device (looked up once).
 uint32_t *status_word() {
-    constexpr int kMaxDevices = 64;
-    static uint32_t *addr[kMaxDevices] = {};
+    static std::atomic<uint32_t *> addr[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (addr[dev] == nullptr && device_status_address(&addr[dev]) != cudaSuccess) addr[dev] = nullptr;
-    return addr[dev];
+    uint32_t *a = addr[dev].load(std::memory_order_acquire);
+    if (a == nullptr) {
+        if (device_status_address(&a) != cudaSuccess) return nullptr;
+        addr[dev].store(a, std::memory_order_release);
+    }
+    return a;
 }
 
+// SM count of the current device (148 on a B200), looked up once per device.
 int sm_count_cached() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            sms = 148;
+    static std::atomic<int> sms[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    int n = sms[dev].load(std::memory_order_acquire);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        sms[dev].store(n, std::memory_order_release);
     }
-    return sms;
+    return n;
 }
 
 // Normalises a (block_n, splits) request so that every split owns >= 1 K tile.  Split

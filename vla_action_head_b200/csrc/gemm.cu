@@ -471,13 +471,10 @@ __global__ void __launch_bounds__(kThreads, SMALL_A ? 2 : 1)
 template <int BN, int STAGES, bool SMALL_A>
 cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
     using S = Smem<BN, STAGES, SMALL_A>;
-    static bool attr_set = false;  // per process; the attribute is idempotent
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, STAGES, SMALL_A>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e =
+        set_smem_limit_once(reinterpret_cast<const void *>(gemm_kernel<BN, STAGES, SMALL_A>), S::kBytes, attr_set);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.n_tiles, (p.M + 127) / 128, p.splits);
     cfg.blockDim = dim3(kThreads);
@@ -510,7 +507,6 @@ cudaError_t launch_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmAr
 // atomics: host threads making their first calls at once each look the address up and
 // store the same value.
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes) {
-    constexpr int kMaxDevices = 64;
     static std::atomic<void *> addr[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -525,6 +521,17 @@ cudaError_t noalloc_scratch(void **ptr, size_t *bytes) {
     *ptr = a;
     *bytes = kNoAllocScratchBytes;
     return cudaSuccess;
+}
+
+cudaError_t set_smem_limit_once(const void *func, int bytes, std::atomic<bool> *done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_release);
+    return e;
 }
 
 bool pdl_enabled() {

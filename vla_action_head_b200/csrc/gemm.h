@@ -4,10 +4,20 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
 namespace nvfp4 {
+
+// Host-side caches that hold per-device state (addresses, function attributes) have one
+// entry per device index below this bound.
+constexpr int kMaxDevices = 64;
+
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device (the attribute belongs to the device's context; `done` has kMaxDevices entries).
+// Safe to call from several host threads: a race only repeats the idempotent call.
+cudaError_t set_smem_limit_once(const void *func, int bytes, std::atomic<bool> *done);
 
 enum { kEpiNone = 0, kEpiBias = 1, kEpiResidual = 2, kEpiBiasResidual = 3, kEpiBiasGelu = 4, kEpiGeglu = 5 };
 

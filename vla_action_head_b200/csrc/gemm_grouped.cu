@@ -327,13 +327,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_grouped_kernel(const Grouped
 
 template <int EPI>
 cudaError_t launch_epi(const GroupedParams &p, int grid, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_grouped_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e =
+        set_smem_limit_once(reinterpret_cast<const void *>(gemm_grouped_kernel<EPI>), kSmemBytes, attr_set);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);

@@ -596,13 +596,10 @@ int gemm_persistent_grid(int M, int n_tiles, int splits) {
 
 template <int BN, int EPI, bool SPLIT>
 static cudaError_t launch_split(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &p, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_persistent_kernel<BN, EPI, SPLIT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, PCfg<BN>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const cudaError_t e = set_smem_limit_once(reinterpret_cast<const void *>(gemm_persistent_kernel<BN, EPI, SPLIT>),
+                                              PCfg<BN>::kSmemBytes, attr_set);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(gemm_persistent_grid(p.M, p.n_tiles, p.splits));
     cfg.blockDim = dim3(kThreads);
