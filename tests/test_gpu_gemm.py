@@ -127,6 +127,42 @@ def test_k_tail_zero_padding(orc):
     _run(orc, 41, 128, 4320, "bias", bn=128, sp=2)
 
 
+@pytest.mark.parametrize("M,bn,sp", [(80, 0, 0), (80, 64, 2), (80, 128, 1), (200, 0, 0)])
+def test_extreme_block_scales(orc, M, bn, sp):
+    """Operands whose blocks take subnormal, normal and saturated UE4M3 scales.  Activation
+    rows of magnitude 1e-2 .. 1e2 in five bands (with g = 1 the 1e-2 band's block scales are
+    E4M3 subnormals) and two rows with +-1e4 outliers (saturated scales: the other values of
+    those blocks round to small codes or zero); weight rows spanning 1e-6 .. 1 of the
+    tensor's amax in four bands (below ~3.5e-5 of the amax a block's scale is subnormal).
+    The tensor core must decode every scale byte as the format defines it, which is how the
+    oracle decodes it; the output is checked block by block (activation band x weight
+    band, outlier rows apart), so that small values are not hidden behind large ones.
+    M = 200 runs the persistent kernel (256-wide tiles, two W scale groups per stage)."""
+    N, K = 256, 1024
+    outl = [3, 42]
+    band = np.arange(M) % 5
+    x = synth.bf16_bits_to_f32(synth.bf16_normal(synth.seed_of(61, synth.X), (M, K)))
+    x = x * (10.0 ** (band - 2.0))[:, None].astype(np.float32)
+    x[3, 17], x[3, 500], x[42, 1000] = 1e4, -1e4, 1e4
+    w = synth.bf16_bits_to_f32(synth.bf16_normal(synth.seed_of(61, synth.W0), (N, K), 0.0, 0.02))
+    w = w * np.logspace(-6, 0, N, dtype=np.float32)[:, None]
+    xb, wb = synth.f32_to_bf16_bits(x), synth.f32_to_bf16_bits(w)
+    ac, asf = orc.quantize_norm(xb, "none", g=1.0)
+    wc, wsf, gw = orc.quantize_weight(wb)
+    # the operands do take subnormal (0 < byte < 8) and saturated (0x7E) scale bytes
+    assert ((asf > 0) & (asf < 8)).any() and (asf == 0x7E).any() and ((wsf > 0) & (wsf < 8)).any()
+    ref = orc.gemm(ac, asf, 1.0, M, wc, wsf, gw, N, K, epi="none")["v"]
+    got = host(nvfp4.gemm(to_gpu_fp4(ac, asf, 1.0, M, K), to_gpu_fp4(wc, wsf, gw, N, K), "none",
+                          block_n=bn, splits=sp))
+    for b in range(5):
+        rows = np.array([r for r in np.nonzero(band == b)[0] if r not in outl])
+        for c in range(4):
+            cols = np.arange(c * N // 4, (c + 1) * N // 4)
+            check_gemm_bf16(got[np.ix_(rows, cols)], ref[np.ix_(rows, cols)], what=("band", b, c, bn, sp))
+    for r in outl:
+        check_gemm_bf16(got[[r]], ref[[r]], what=("outlier row", r, bn, sp))
+
+
 def test_zero_activations_give_bias(orc):
     M, N, K = 41, 256, 512
     ac = np.zeros((M, K // 2), np.uint8)
