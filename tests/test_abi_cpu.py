@@ -90,6 +90,12 @@ def test_gemm_validation(L):
     assert call(ldo=68) == 3                   # ld not a multiple of 8
     # valid arguments reach the device check: no GPU here
     assert call() in (5, 6)
+    # M == 0 is a no-op: valid shapes and scales are enough (no pointer is read, no device
+    # call is made), while a malformed call with M == 0 is still rejected
+    empty = _t(rows=0, K=64, codes=0, sf=0)
+    assert call(a=empty, M=0, out=None, ldo=0, epi=3) == 0
+    assert call(a=empty, M=0, epi=9) == 1
+    assert call(a=empty, M=0, N=32, w=_t(rows=32, K=64)) == 2
 
 
 def test_mma_rate_validation(L):
