@@ -41,11 +41,11 @@ DIT = dict(M=41, H=1536, F=6144)
 # of the kernel sources they were taken on: once a source changes the figure is reported as null.
 TRAFFIC = {
     "dit_gemm": {"sources": ["gemm.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                 "sha256": "f2bc3d5193e6f38dc067ddd816a42020debac10081680e8a4b9a5502166753b5",
-                 "bytes": 4213568},  # mean of the 4 DiT GEMM launches (case dit-gemms)
+                 "sha256": "e533d6ba7a6374968bbe10c65e2504292a354537b26dbd3bd82c9cbf495935a7",
+                 "bytes": 4213888},  # mean of the 4 DiT GEMM launches (case dit-gemms)
     "prefill_gate_up": {"sources": ["gemm_persistent.cu", "gemm.h", "epilogue.cuh", "quant.cuh", "sm100.cuh"],
-                        "sha256": "a713df3f33f559394d6ec514bb61f5fb9b24258aaf90c2d9e37c2dc8d51b6764",
-                        "bytes": 38964224},  # the gate/up launch of case prefill-gemms
+                        "sha256": "31ab8efdad49dbafc019494c7a579955034a47b345434bb78976656d20918f52",
+                        "bytes": 38947072},  # the gate/up launch of case prefill-gemms
 }
 
 
