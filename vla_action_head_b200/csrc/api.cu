@@ -144,7 +144,9 @@ Schedule finish(int block_n, int splits, int K, bool use_cluster = true) {
 //   30 GB/s per CTA (up to one CTA per SM), + 2e-4 per element of a re-quantizing epilogue
 //   (bias+GELU or GeGLU -> FP4) on the owner CTA.  Grids above 1.35 CTAs per SM (1.5 for a
 //   re-quantizing epilogue), or above what one wave of the kernel holds, measured slow and
-//   are not used.
+//   are not used; with 16 or more K tiles a grid stays within one CTA per SM (measured in
+//   the DiT chain at 41 x 1536 x 6144: 6 splits on 144 CTAs 30.92 us per layer against 8
+//   splits on 192 CTAs 31.24, the model's own pick).
 Schedule choose(int M, int N, int K, bool fp4_out) {
     const int sms = sm_count_cached();
     const int k_tiles = (K + 255) / 256;
@@ -166,6 +168,7 @@ Schedule choose(int M, int N, int K, bool fp4_out) {
                 const int wave = M > 64 ? gemm_wave_ctas(false, bn, c.splits) : 0;
                 if (wave > 0 && ctas > wave) continue;
                 if (fp4_out && 2 * ctas > 3 * sms) continue;
+                if (k_tiles >= 16 && ctas > sms) continue;
                 const int owner_rows = (std::min(M, 128) + c.splits - 1) / c.splits;
                 const double cost = 0.3 * c.kt_per_split + (c.splits > 1 ? 0.3 + 0.004 * bn : 0.0) +
                                     bytes / (std::min(ctas, sms) * 30e3) +
