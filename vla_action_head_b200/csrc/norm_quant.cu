@@ -10,6 +10,11 @@
 
 namespace nvfp4 {
 
+// Brings the line holding p into L2 (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 // TPR threads per row, BPT blocks of 16 per thread, F32: fp32 input (else bf16).
 template <int TPR, int BPT, bool F32>
 __global__ void __launch_bounds__(128) norm_quant_kernel(const NormArgs p) {
@@ -18,6 +23,28 @@ __global__ void __launch_bounds__(128) norm_quant_kernel(const NormArgs p) {
     // Let the next kernel launch now (it prefetches its weights), then wait for our input,
     // which may be the previous kernel's output (programmatic dependent launch).
     pdl_launch_dependents();
+    if constexpr (TPR == 128) {
+        // A CTA per row (tens to hundreds of rows, latency-bound): bring this thread's blocks of
+        // the per-column parameters into L2 while the previous kernel finishes, so that their
+        // loads after the wait are L2 hits.  Only L2 is touched, which stays coherent: a
+        // parameter that the previous kernel writes is still read fresh after the wait.
+        // (Measured: 0.2 us off a DiT layer.  With a warp per row, hundreds of warps would
+        // prefetch the same lines: 0.4 us slower at 968 rows, so not there.)
+        const int t = threadIdx.x, nblk = p.K >> 4;
+        const bool ada = (p.kind == kAdaLN || p.kind == kAdaRms);
+        const uint16_t *pa = ada ? p.scale : p.gamma;
+        const uint16_t *pb = (p.kind == kLayerNorm) ? p.beta : p.shift;
+        const uint16_t *pg = F32 ? nullptr : p.res_gate;
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) {
+            const int b = t + i * TPR;
+            if (b < nblk) {
+                if (pa != nullptr) prefetch_l2(pa + static_cast<size_t>(b) * 16);
+                if (pb != nullptr) prefetch_l2(pb + static_cast<size_t>(b) * 16);
+                if (pg != nullptr) prefetch_l2(pg + static_cast<size_t>(b) * 16);
+            }
+        }
+    }
     pdl_wait();
     norm_row<TPR, BPT, F32>(p, blockIdx.x * kRowsPerCta + threadIdx.x / TPR, threadIdx.x % TPR, red);
 }
