@@ -120,3 +120,25 @@ def test_norm_and_weight_validation(L):
     assert w(x, 64, 64, 64, 0, c, s, None, x, None) == 1
     assert w(x, 63, 64, 64, 1, c, s, C.byref(gs), x, None) == 2  # interleave needs even N
     assert w(x, 64, 64, 64, 0, c, s, C.byref(gs), x, None) in (5, 6)
+
+
+def test_default_schedules_of_the_workload_gemms(L):
+    """The latency model's picks for the small-M GEMMs of the benchmarked layers, as CTA
+    counts (trace words / 8) on a 148-SM device: the choices the in-chain A/B measurements
+    settled on (64-wide tiles; the DiT FFN-down GEMM on 6 splits, one CTA per SM, rather
+    than 8).  Host logic only: no device call is made for M <= 64."""
+    if L.nvfp4_gemm_trace_words(41, 4608, 1536, 1) == 0:
+        pytest.skip("schedule query unavailable")
+    picks = {  # (M, N, K, epilogue) -> CTAs
+        (41, 4608, 1536, 1): 72 * 2,   # DiT qkv: 64-wide x 2 splits
+        (41, 1536, 1536, 3): 24 * 6,   # DiT attention-out: 64 x 6
+        (41, 6144, 1536, 4): 96 * 2,   # DiT FFN-up (bias+GELU -> FP4): 64 x 2
+        (41, 1536, 6144, 3): 24 * 6,   # DiT FFN-down: 64 x 6 (K tiles >= 16: <= one CTA per SM)
+        (50, 2560, 1024, 0): 40 * 4,   # action-expert qkv: 64 x 4
+        (50, 1024, 2048, 2): 16 * 8,   # action-expert attention-out
+        (50, 8192, 1024, 5): 128,      # action-expert gate/up (GeGLU)
+        (50, 1024, 4096, 2): 16 * 8,   # action-expert down
+    }
+    for (M, N, K, epi), ctas in picks.items():
+        assert L.nvfp4_gemm_trace_words(M, N, K, epi) == 8 * ctas, (M, N, K, epi)
+
